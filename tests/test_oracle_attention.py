@@ -1,0 +1,114 @@
+"""Pins for the oracle's masked attention (CPU only)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import attention, select, tiling
+
+
+def test_all_kept_equals_torch_sdpa_fp64():
+    rng = np.random.default_rng(0)
+    L, D = 96, 16
+    q, k, v = (rng.standard_normal((L, D)) for _ in range(3))
+    o, lse = attention.dense_masked(q, k, v, np.ones((L, L), bool), 1 / math.sqrt(D))
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        *(torch.from_numpy(t)[None, None] for t in (q, k, v)))[0, 0].numpy()
+    np.testing.assert_allclose(o, ref, rtol=1e-12, atol=1e-13)
+    mask = rng.random((L, L)) < 0.3
+    mask[np.arange(L), np.arange(L)] = True
+    o2, _ = attention.dense_masked(q, k, v, mask, 0.25)
+    ref2 = torch.nn.functional.scaled_dot_product_attention(
+        *(torch.from_numpy(t)[None, None] for t in (q, k, v)),
+        attn_mask=torch.from_numpy(mask)[None, None], scale=0.25)[0, 0].numpy()
+    np.testing.assert_allclose(o2, ref2, rtol=1e-12, atol=1e-13)
+
+
+def test_brute_force_triple_loop():
+    rng = np.random.default_rng(1)
+    Lq, Lk, D = 5, 7, 3
+    q, k, v = rng.standard_normal((Lq, D)), rng.standard_normal((Lk, D)), rng.standard_normal((Lk, D))
+    mask = rng.random((Lq, Lk)) < 0.6
+    mask[:, 0] = True
+    o, lse = attention.dense_masked(q, k, v, mask, 0.7)
+    for n in range(Lq):
+        w = [math.exp(0.7 * sum(q[n, d] * k[m, d] for d in range(D))) if mask[n, m] else 0.0
+             for m in range(Lk)]
+        z = sum(w)
+        assert lse[n] == pytest.approx(math.log(z), rel=1e-13)
+        for d in range(D):
+            assert o[n, d] == pytest.approx(sum(w[m] * v[m, d] for m in range(Lk)) / z,
+                                            rel=1e-12, abs=1e-14)
+
+
+def test_rows_normalised():
+    rng = np.random.default_rng(2)
+    q, k = rng.standard_normal((40, 8)) * 3, rng.standard_normal((40, 8)) * 3
+    mask = rng.random((40, 40)) < 0.5
+    mask[:, 3] = True
+    o, _ = attention.dense_masked(q, k, np.ones((40, 8)), mask, 1.0)
+    np.testing.assert_allclose(o, 1.0, rtol=1e-14)
+
+
+def test_single_valid_key_returns_its_value():
+    """Grid 5x1x1: tile 1 holds only token t=4; attending only tile 1 copies v[4]."""
+    T, H, W = 5, 1, 1
+    rng = np.random.default_rng(3)
+    q, k, v = (rng.standard_normal((1, 5, 1, 4)) for _ in range(3))
+    lists = [np.array([1]), np.array([1])]
+    o, lse = attention.attention_full(q, k, v, lists, T, H, W)
+    np.testing.assert_array_equal(o[0, :, 0], np.repeat(v[0, 4:5, 0], 5, axis=0))
+    np.testing.assert_allclose(lse[0, 0], 0.5 * q[0, :, 0] @ k[0, 4, 0], rtol=1e-14)
+
+
+def test_in_tile_permutation_invariance():
+    T, H, W = 8, 4, 8
+    rng = np.random.default_rng(4)
+    q, k, v = (rng.standard_normal((1, T * H * W, 2, 8)) for _ in range(3))
+    nb = tiling.n_blocks(T, H, W)
+    lists = [np.sort(rng.choice(nb, 2, replace=False)) for _ in range(2 * nb)]
+    o, _ = attention.attention_full(q, k, v, lists, T, H, W)
+    tid, _ = tiling.token_tile_and_row(T, H, W)
+    perm = np.arange(T * H * W)
+    for j in range(nb):
+        mem = np.nonzero(tid == j)[0]
+        perm[mem] = rng.permutation(mem)
+    o2, _ = attention.attention_full(q[:, perm], k[:, perm], v[:, perm], lists, T, H, W)
+    np.testing.assert_allclose(o2, o[:, perm], rtol=1e-12, atol=1e-13)
+
+
+def test_rows_form_equals_full_mask_form():
+    T, H, W = 6, 5, 9
+    rng = np.random.default_rng(5)
+    q, k, v = (rng.standard_normal((2, T * H * W, 2, 8)) for _ in range(3))
+    nb = tiling.n_blocks(T, H, W)
+    lists = [np.sort(rng.choice(nb, rng.integers(1, nb + 1), replace=False)) for _ in range(4 * nb)]
+    o, lse = attention.attention_full(q, k, v, lists, T, H, W)
+    rows = attention.attention_rows(q, k, v, lists, T, H, W)
+    for (b, h, i), (tok, oi, li) in rows.items():
+        np.testing.assert_allclose(oi, o[b, tok, h], rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(li, lse[b, h, tok], rtol=1e-13)
+
+
+def test_all_tiles_kept_is_dense_attention_over_valid_tokens():
+    T, H, W = 5, 6, 7
+    rng = np.random.default_rng(6)
+    q, k, v = (rng.standard_normal((1, T * H * W, 1, 8)) for _ in range(3))
+    nb = tiling.n_blocks(T, H, W)
+    lists = [np.arange(nb)] * nb
+    o, _ = attention.attention_full(q, k, v, lists, T, H, W)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        *(torch.from_numpy(t[0, :, 0])[None, None] for t in (q, k, v)))[0, 0].numpy()
+    np.testing.assert_allclose(o[0, :, 0], ref, rtol=1e-12, atol=1e-13)
+
+
+def test_fp8_qk_uses_tile_scales():
+    T, H, W = 4, 4, 8
+    rng = np.random.default_rng(7)
+    q = rng.standard_normal((1, T * H * W, 1, 16)).astype(np.float32)
+    k = q * 3
+    qd, kd, (qc, qs), (kc, ks) = attention.fp8_qk(q, k, T, H, W)
+    np.testing.assert_array_equal(qc, kc)  # scaling by 3 scales amax and scale alike
+    assert qs.shape == (1, 1, 2)
+    np.testing.assert_allclose(qd, q, rtol=2 ** -4, atol=float(qs.max()) * 2 ** -9)
