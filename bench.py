@@ -1,0 +1,465 @@
+"""Benchmark of the block-sparse attention layer on one or more B200s.
+
+A step is one whole layer through the C ABI (attn_layer): tile reorder with
+fused pooling (and e4m3 quantisation on the FP8 workload), block scores,
+key-tile selection, block-sparse attention, unreorder. Inputs are seeded
+synthetic video-latent Q/K/V already resident in HBM; L2 is flushed between
+timed steps. Prints one JSON line (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference ...   # the fp64 CPU oracle on host cores
+
+For N > 1 launch under torch.distributed.run: every rank runs its own layer
+(independent problems, weak scaling, no data-path collective); the step
+time is the max over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from block_sparse_attention_reorder_b200.datagen import WORKLOADS, make_qkv  # noqa: E402
+
+METRIC = "sparse attn fwd ms/layer & achieved TFLOP/s on kept blocks vs B200 BF16 peak"
+DEFAULT_WORKLOAD = "wan1.3b"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+def kept_pairs_from_counts(cnt: torch.Tensor) -> int:
+    return int(cnt.to(torch.int64).sum().item())
+
+
+def pair_flops(head_dim: int) -> float:
+    # QK^T and PV on one 64x64 tile pair: 2 * (2 * 64 * 64 * D)
+    return 4.0 * 64 * 64 * head_dim
+
+
+def launches_per_step(wl) -> int:
+    pooled = wl.rule != "window"
+    return 3 + (2 if pooled else 1) + 2  # reorder x3, [scores], select, attention, unreorder
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while work runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(device_index)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def cpu_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+_CPU_INPUTS = {}
+
+
+def cpu_inputs(wl):
+    """Seeded CPU inputs of one head of the workload, fp64 (drawn once)."""
+    import dataclasses
+
+    if wl.name not in _CPU_INPUTS:
+        one = dataclasses.replace(wl, heads=1)
+        _CPU_INPUTS[wl.name] = tuple(x.to(torch.float64).numpy() for x in make_qkv(one, "cpu"))
+    return _CPU_INPUTS[wl.name]
+
+
+def oracle_sample(wl, seconds_target: float = 12.0):
+    """Time the oracle (as it stands) on a bounded sample of the workload.
+
+    Sample: one head of the layer. Routing (pool, scores, rule) over the whole
+    grid, then attention of that head's query tiles in seeded order until
+    about `seconds_target` seconds have passed. Returns (kept FLOP, seconds,
+    description).
+    """
+    import numpy as np
+    from oracle import attention
+
+    qn, kn, vn = cpu_inputs(wl)
+    t0 = time.perf_counter()
+    if wl.qk_fp8:
+        qn, kn, _, _ = attention.fp8_qk(qn, kn, wl.T, wl.H, wl.W)
+    _, _, _, lists = attention.route(qn, kn, wl.T, wl.H, wl.W, wl.rule, k=wl.k, p=wl.p,
+                                     half=wl.win)
+    N = len(lists)
+    order = np.random.default_rng(0).permutation(N)
+    pairs, done = 0, 0
+    for i in order:
+        attention.attention_rows(qn, kn, vn, lists, wl.T, wl.H, wl.W, rows=[(0, 0, int(i))])
+        pairs += len(lists[i])
+        done += 1
+        if time.perf_counter() - t0 > seconds_target:
+            break
+    secs = time.perf_counter() - t0
+    text = (f"one head of {wl.heads}: routing over all {N} tiles, then attention of {done} of "
+            f"{N} query tiles ({pairs} kept tile pairs), fp64 numpy")
+    return pairs * pair_flops(wl.head_dim), secs, text
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    wl = WORKLOADS[args.workload]
+    total_flops, total_s, text = 0.0, 0.0, ""
+    per_step_target = max(0.05, 90.0 / max(1, args.steps + args.warmup))
+    for s in range(args.warmup + args.steps):
+        f, secs, text = oracle_sample(wl, seconds_target=per_step_target)
+        if s >= args.warmup:
+            total_flops += f
+            total_s += secs
+    tflops = total_flops / total_s / 1e12 if total_s > 0 else None
+    line = {"impl": "reference", "metric": METRIC, "value": tflops, "unit": "TFLOP/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": total_s / max(1, args.steps) * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(wl),
+            "cpu_baseline": {"value": tflops, "unit": "TFLOP/s", "cores": cpu_threads(),
+                             "kind": "oracle", "sample": text + " (each step)"},
+            "e2e": {"value": tflops, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+def workload_config(wl, extra=None):
+    Tp, Hp, Wp = (-(-n // t) * t for n, t in zip((wl.T, wl.H, wl.W), wl.tile))
+    cfg = {"workload": wl.name, "B": wl.B, "heads": wl.heads, "head_dim": wl.head_dim,
+           "grid": [wl.T, wl.H, wl.W], "padded": [Tp, Hp, Wp], "tile": list(wl.tile),
+           "rule": wl.rule, "qk": "e4m3" if wl.qk_fp8 else "bf16",
+           "l2": "flushed between timed steps (256 MiB write)",
+           "data": "seeded synthetic " + ("iid N(0,1)" if wl.recipe == "iid" else
+                                          "Gaussian-blurred field (sigma 2) + N(0,0.5^2) noise")}
+    if wl.rule in ("topk", "topp"):
+        cfg["k"] = wl.k
+    if wl.rule == "topp":
+        cfg["p"] = wl.p
+    if wl.rule == "window":
+        cfg["window_half"] = list(wl.win)
+    if extra:
+        cfg.update(extra)
+    return cfg
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    from block_sparse_attention_reorder_b200 import bsattn
+
+    wl = WORKLOADS[args.workload]
+    plan = bsattn.Plan.for_workload(wl)
+    q, k, v = make_qkv(wl, "cuda", batch_offset=rank)
+    o = torch.empty_like(q)
+    ws = plan.workspace("layer")
+    si, sc = plan.list_shapes()
+    idx = torch.empty(si, dtype=torch.int32, device="cuda")
+    cnt = torch.empty(sc, dtype=torch.int32, device="cuda")
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step():
+        bsattn.attn_layer(plan, q, k, v, o, ws, idx=idx, cnt=cnt, stream=stream)
+
+    step()
+    if bsattn.attn_check_device_status(plan) != 0:
+        raise SystemExit("device error word set")
+    kept = kept_pairs_from_counts(cnt)
+    flops = kept * pair_flops(wl.head_dim)
+
+    sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        step()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    for s in range(args.steps):
+        flush.fill_(float(s))
+        ev[s][0].record(stream)
+        step()
+        ev[s][1].record(stream)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks = sampler.stop() if sampler else None
+    total_ms = sum(a.elapsed_time(b) for a, b in ev)
+    if dist:
+        t = torch.tensor([total_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+
+    # Per-kernel breakdown: the same layer as its C-ABI components, with
+    # events between launches on the launching stream.
+    comp = component_timing(bsattn, plan, wl, q, k, v, flush, stream, reps=min(args.steps, 50))
+
+    # End to end through the public API with host buffers: pinned host
+    # inputs copied in, the layer, the output copied back, every step.
+    e2e = e2e_timing(bsattn, plan, q, k, v, ws, idx, cnt, stream, steps=args.e2e_steps,
+                     warmup=3, dist=dist)
+
+    if dist:
+        dist.barrier()
+    if rank != 0:
+        if dist:
+            dist.destroy_process_group()
+        return 0
+
+    pk = peaks()
+    attn_ms = comp["attention"]
+    achieved = flops / (attn_ms * 1e-3) / 1e12
+    line = {
+        "metric": METRIC,
+        "value": world * flops / (ms_per_step * 1e-3) / 1e12,
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_per_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16+e4m3" if wl.qk_fp8 else "bf16",
+        "data": "synthetic",
+        "config": workload_config(wl, {"kept_pairs": kept, "kept_tflop": flops / 1e12,
+                                        "parallelism": f"independent layer per GPU x{world}"}),
+        "ms_per_layer": ms_per_step,
+        "kernels_ms": comp,
+        "roofline": {"bound": "tensor", "kernel": "attention", "achieved": achieved,
+                     "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": achieved / pk["bf16_tflops"],
+                     "peak_note": f"{pk['source']} bf16 burst (kernel timed alone)",
+                     "traffic": None},
+        "memory_kernels": memory_kernel_rates(wl, plan, comp, pk),
+        "e2e": e2e,
+        "gpu_launches": launches_per_step(wl) * args.steps,
+        "clocks": clocks,
+    }
+    if not args.no_cpu_baseline and world == 1:
+        f, secs, text = oracle_sample(wl)
+        line["cpu_baseline"] = {"value": f / secs / 1e12, "unit": "TFLOP/s",
+                                "cores": cpu_threads(), "kind": "oracle", "sample": text}
+    print(json.dumps(line))
+    if dist:
+        dist.destroy_process_group()
+    return 0
+
+
+def component_timing(bsattn, plan, wl, q, k, v, flush, stream, reps=20):
+    """Average device time of each step of the layer, launched one by one."""
+    tiled = [torch.empty(plan.tiled_shape(), dtype=torch.bfloat16, device="cuda") for _ in range(3)]
+    pq = torch.empty((wl.B, wl.heads, plan.N, wl.head_dim), dtype=torch.float32, device="cuda")
+    pk = torch.empty_like(pq)
+    S = torch.empty((wl.B, wl.heads, plan.N, plan.N), dtype=torch.float32, device="cuda") \
+        if wl.rule != "window" else None
+    si, sc = plan.list_shapes()
+    idx = torch.empty(si, dtype=torch.int32, device="cuda")
+    cnt = torch.empty(sc, dtype=torch.int32, device="cuda")
+    o_t = torch.empty(plan.tiled_shape(), dtype=torch.bfloat16, device="cuda")
+    o = torch.empty_like(q)
+    if wl.qk_fp8:
+        codes = [torch.empty(plan.tiled_shape(), dtype=torch.uint8, device="cuda") for _ in range(2)]
+        scales = [torch.empty((wl.B, wl.heads, plan.N), dtype=torch.float32, device="cuda")
+                  for _ in range(2)]
+    names = ["reorder_qk", "reorder_v", "block_scores", "select", "quantize", "attention",
+             "unreorder"]
+    acc = {n: 0.0 for n in names}
+
+    def timed(name, fn):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        return name, a, b
+
+    for r in range(reps + 2):
+        marks = []
+        flush.fill_(1.0)
+        pooled = wl.rule != "window"
+        marks.append(timed("reorder_qk", lambda: (
+            bsattn.attn_reorder(plan, q, tiled[0], pq if pooled else None, stream),
+            bsattn.attn_reorder(plan, k, tiled[1], pk if pooled else None, stream))))
+        marks.append(timed("reorder_v", lambda: bsattn.attn_reorder(plan, v, tiled[2], None, stream)))
+        if pooled:
+            marks.append(timed("block_scores", lambda: bsattn.attn_block_scores(plan, pq, pk, S, stream)))
+        marks.append(timed("select", lambda: bsattn.attn_select_from_scores(plan, S, idx, cnt, stream)))
+        if wl.qk_fp8:
+            marks.append(timed("quantize", lambda: (
+                bsattn.attn_quantize_e4m3(plan, tiled[0], codes[0], scales[0], stream),
+                bsattn.attn_quantize_e4m3(plan, tiled[1], codes[1], scales[1], stream))))
+            qa, ka, qs, ks = codes[0], codes[1], scales[0], scales[1]
+        else:
+            qa, ka, qs, ks = tiled[0], tiled[1], None, None
+        flush.fill_(2.0)
+        marks.append(timed("attention", lambda: bsattn.attn_forward(
+            plan, qa, ka, tiled[2], idx, cnt, o_t, q_scale=qs, k_scale=ks, stream=stream)))
+        marks.append(timed("unreorder", lambda: bsattn.attn_unreorder(plan, o_t, o, stream)))
+        torch.cuda.synchronize()
+        if r >= 2:
+            for n, a, b in marks:
+                acc[n] += a.elapsed_time(b)
+    return {n: acc[n] / reps for n in names if acc[n] > 0}
+
+
+def memory_kernel_rates(wl, plan, comp, pk):
+    """Algorithmic bytes / time for the HBM-bound steps."""
+    bh = wl.B * wl.heads
+    nat = wl.B * wl.L * wl.heads * wl.head_dim * 2
+    til = bh * plan.N * 64 * wl.head_dim * 2
+    pooled = bh * plan.N * wl.head_dim * 4
+    out = {}
+    if "reorder_qk" in comp:
+        b = 2 * (nat + til) + (2 * pooled if wl.rule != "window" else 0)
+        out["reorder_qk"] = b / (comp["reorder_qk"] * 1e-3) / 1e9
+    if "reorder_v" in comp:
+        out["reorder_v"] = (nat + til) / (comp["reorder_v"] * 1e-3) / 1e9
+    if "select" in comp and wl.rule != "window":
+        rows = bh * plan.N
+        b = rows * plan.N * 4 + rows * 4 + rows * (wl.k if wl.rule == "topk" else plan.N / 4) * 4
+        out["select"] = b / (comp["select"] * 1e-3) / 1e9
+    if "unreorder" in comp:
+        out["unreorder"] = (nat + til) / (comp["unreorder"] * 1e-3) / 1e9
+    res = {n: {"GB/s": round(x, 1), "frac": round(x / pk["hbm_gbs"], 3)} for n, x in out.items()}
+    res["peak_GBs"] = pk["hbm_gbs"]
+    res["note"] = "algorithmic bytes / kernel time; of " + pk["source"] + " HBM copy bandwidth"
+    return res
+
+
+def e2e_timing(bsattn, plan, q, k, v, ws, idx, cnt, stream, steps=10, warmup=3, dist=None):
+    hq = [x.cpu().pin_memory() for x in (q, k, v)]
+    ho = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+    dq = [torch.empty_like(x) for x in (q, k, v)]
+    do = torch.empty_like(q)
+    flops_per = kept_pairs_from_counts(cnt) * pair_flops(plan.D)
+
+    def one():
+        for h, d in zip(hq, dq):
+            d.copy_(h, non_blocking=True)
+        bsattn.attn_layer(plan, dq[0], dq[1], dq[2], do, ws, idx=idx, cnt=cnt, stream=stream)
+        ho.copy_(do, non_blocking=True)
+
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        one()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    world = 1
+    if dist:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+        world = dist.get_world_size()
+    h2d = sum(x.numel() * x.element_size() for x in hq)
+    d2h = ho.numel() * ho.element_size()
+    return {"value": world * flops_per / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "ms_per_step": ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,80 @@
+// Internal declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+#include <stddef.h>
+
+#include "bsattn.h"
+
+// Device error word bits (plan->d_err).
+enum : int {
+  BSATTN_DEVERR_BAD_INDEX = 1,  // a kept-list entry or count outside [0, N]
+  BSATTN_DEVERR_TIMEOUT = 2,    // a bounded wait gave up
+};
+
+struct bsattn_plan {
+  bsattn_desc desc;
+  bsattn_rule rule;
+  int device;
+  int Tp, Hp, Wp, nT, nH, nW, N, V, L, kmax;
+  float scale;
+  int* d_err;        // device error word
+  int32_t* d_win_idx;  // window rule: [N, kmax]
+  int32_t* d_win_cnt;  // window rule: [N]
+};
+
+// Geometry passed by value to kernels.
+struct Geom {
+  int B, Hh, D;
+  int T, H, W;
+  int tt, th, tw;
+  int nT, nH, nW, N, L;
+};
+
+static inline Geom make_geom(const bsattn_plan* p) {
+  Geom g;
+  g.B = p->desc.B; g.Hh = p->desc.heads; g.D = p->desc.head_dim;
+  g.T = p->desc.T; g.H = p->desc.H; g.W = p->desc.W;
+  g.tt = p->desc.tile_t; g.th = p->desc.tile_h; g.tw = p->desc.tile_w;
+  g.nT = p->nT; g.nH = p->nH; g.nW = p->nW; g.N = p->N; g.L = p->L;
+  return g;
+}
+
+static inline bool aligned16(const void* ptr) { return (((uintptr_t)ptr) & 15u) == 0; }
+
+#define BSATTN_CUDA_TRY(expr)                         \
+  do {                                                \
+    cudaError_t e_ = (expr);                          \
+    if (e_ != cudaSuccess) return BSATTN_ERR_CUDA;    \
+  } while (0)
+
+// Launch wrappers (each returns BSATTN_OK or BSATTN_ERR_CUDA).
+// flags for launch_reorder
+enum : int {
+  RO_WRITE_TILED = 1,  // write the tiled bf16 copy
+  RO_POOL = 2,         // write fp32 tile means
+  RO_QUANT = 4,        // write e4m3 codes + tile scales instead of/in addition to bf16
+};
+bsattn_status launch_reorder(const Geom& g, const __nv_bfloat16* x_nat, __nv_bfloat16* x_tiled,
+                             float* pooled, uint8_t* codes, float* scales, int flags,
+                             cudaStream_t st);
+bsattn_status launch_unreorder(const Geom& g, const __nv_bfloat16* x_tiled, __nv_bfloat16* x_nat,
+                               const float* lse_tiled, float* lse_nat, cudaStream_t st);
+bsattn_status launch_quant_tiled(const Geom& g, const __nv_bfloat16* x_tiled, uint8_t* codes,
+                                 float* scales, cudaStream_t st);
+bsattn_status launch_block_scores(const Geom& g, const float* pq, const float* pk, float scale,
+                                  float* S, cudaStream_t st);
+bsattn_status launch_select_topk(int rows, int N, int k, const float* S, int32_t* idx,
+                                 int32_t* cnt, int kmax, cudaStream_t st);
+bsattn_status launch_select_topp(int rows, int N, int k, double p, const float* S, int32_t* idx,
+                                 int32_t* cnt, int kmax, cudaStream_t st);
+bsattn_status launch_broadcast_lists(int bh, int N, int kmax, const int32_t* src_idx,
+                                     const int32_t* src_cnt, int32_t* idx, int32_t* cnt,
+                                     cudaStream_t st);
+bsattn_status launch_attention(const bsattn_plan* p, const void* q, const void* k,
+                               const float* qs, const float* ks, const __nv_bfloat16* v,
+                               const int32_t* idx, const int32_t* cnt, __nv_bfloat16* o,
+                               float* lse, void* ws, size_t ws_bytes, cudaStream_t st);
+size_t attention_workspace_bytes(const bsattn_plan* p);

@@ -1,0 +1,381 @@
+// Plans, argument checking and the C ABI entry points. Host code only: every
+// step of the computation runs in the kernels of the other translation units.
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <new>
+#include <vector>
+
+#include "internal.h"
+
+namespace {
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Carves sub-buffers out of a caller-provided workspace, 256-byte aligned.
+struct Carve {
+  char* base;
+  size_t off = 0;
+  explicit Carve(void* b) : base(static_cast<char*>(b)) {}
+  void* take(size_t bytes) {
+    off = align_up(off, 256);
+    void* p = base ? base + off : nullptr;
+    off += bytes;
+    return p;
+  }
+};
+
+struct SelectWs {
+  float* pq;
+  float* pk;
+  float* S;
+};
+
+SelectWs carve_select(const bsattn_plan* p, Carve& c) {
+  size_t bh = (size_t)p->desc.B * p->desc.heads;
+  SelectWs w;
+  w.pq = (float*)c.take(bh * p->N * p->desc.head_dim * sizeof(float));
+  w.pk = (float*)c.take(bh * p->N * p->desc.head_dim * sizeof(float));
+  w.S = (float*)c.take(bh * p->N * p->N * sizeof(float));
+  return w;
+}
+
+struct LayerWs {
+  void* qt;  // bf16 tiled or e4m3 codes
+  void* kt;
+  __nv_bfloat16* vt;
+  float* qs;
+  float* ks;
+  SelectWs sel;
+  int32_t* idx;
+  int32_t* cnt;
+  __nv_bfloat16* ot;
+  float* lse_t;
+  void* attn_ws;
+};
+
+LayerWs carve_layer(const bsattn_plan* p, Carve& c) {
+  size_t bh = (size_t)p->desc.B * p->desc.heads;
+  size_t elems = bh * p->N * p->V * p->desc.head_dim;
+  size_t qk_elt = p->desc.qk_fp8 ? 1 : 2;
+  LayerWs w;
+  w.qt = c.take(elems * qk_elt);
+  w.kt = c.take(elems * qk_elt);
+  w.vt = (__nv_bfloat16*)c.take(elems * 2);
+  w.qs = (float*)c.take(p->desc.qk_fp8 ? bh * p->N * sizeof(float) : 0);
+  w.ks = (float*)c.take(p->desc.qk_fp8 ? bh * p->N * sizeof(float) : 0);
+  if (p->rule.kind == BSATTN_RULE_WINDOW) {
+    w.sel.pq = w.sel.pk = w.sel.S = nullptr;
+  } else {
+    w.sel = carve_select(p, c);
+  }
+  w.idx = (int32_t*)c.take(bh * p->N * p->kmax * sizeof(int32_t));
+  w.cnt = (int32_t*)c.take(bh * p->N * sizeof(int32_t));
+  w.ot = (__nv_bfloat16*)c.take(elems * 2);
+  w.lse_t = (float*)c.take(bh * p->N * p->V * sizeof(float));
+  w.attn_ws = c.take(attention_workspace_bytes(p));
+  return w;
+}
+
+bool ok_ptr(const void* x) { return x != nullptr && aligned16(x); }
+
+bsattn_status set_device(const bsattn_plan* p) {
+  int cur = -1;
+  BSATTN_CUDA_TRY(cudaGetDevice(&cur));
+  if (cur != p->device) BSATTN_CUDA_TRY(cudaSetDevice(p->device));
+  return BSATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* attn_status_string(bsattn_status s) {
+  switch (s) {
+    case BSATTN_OK: return "ok";
+    case BSATTN_ERR_INVALID_ARG: return "invalid argument";
+    case BSATTN_ERR_UNSUPPORTED: return "unsupported configuration";
+    case BSATTN_ERR_CUDA: return "CUDA error";
+    case BSATTN_ERR_TIMEOUT: return "device wait timed out";
+    case BSATTN_ERR_INTERNAL: return "device reported a bad kept-list entry";
+    case BSATTN_ERR_WORKSPACE: return "workspace missing or too small";
+  }
+  return "unknown status";
+}
+
+bsattn_status attn_plan_create(const bsattn_desc* d, const bsattn_rule* r, bsattn_plan** out) {
+  if (!d || !r || !out) return BSATTN_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (d->B < 1 || d->heads < 1 || d->T < 1 || d->H < 1 || d->W < 1 || d->tile_t < 1 ||
+      d->tile_h < 1 || d->tile_w < 1 || d->head_dim < 1)
+    return BSATTN_ERR_INVALID_ARG;
+  if (d->head_dim != 64 && d->head_dim != 128) return BSATTN_ERR_UNSUPPORTED;
+  if (d->tile_t * d->tile_h * d->tile_w != 64) return BSATTN_ERR_UNSUPPORTED;
+  if (d->qk_fp8 != 0 && d->qk_fp8 != 1) return BSATTN_ERR_INVALID_ARG;
+  long long Tp = (d->T + d->tile_t - 1) / d->tile_t * (long long)d->tile_t;
+  long long Hp = (d->H + d->tile_h - 1) / d->tile_h * (long long)d->tile_h;
+  long long Wp = (d->W + d->tile_w - 1) / d->tile_w * (long long)d->tile_w;
+  long long N = (Tp / d->tile_t) * (Hp / d->tile_h) * (Wp / d->tile_w);
+  long long L = (long long)d->T * d->H * d->W;
+  if (N > (1 << 20) || L > (1LL << 30) / d->heads) return BSATTN_ERR_UNSUPPORTED;
+
+  int kmax = 0;
+  switch (r->kind) {
+    case BSATTN_RULE_TOPK:
+      if (r->k < 1 || r->k > N) return BSATTN_ERR_INVALID_ARG;
+      if (N > 2048) return BSATTN_ERR_UNSUPPORTED;
+      kmax = r->k;
+      break;
+    case BSATTN_RULE_TOPP:
+      if (r->k < 0 || r->k > N || !(r->p > 0.0 && r->p <= 1.0)) return BSATTN_ERR_INVALID_ARG;
+      if (N > 2048) return BSATTN_ERR_UNSUPPORTED;
+      kmax = (int)N;
+      break;
+    case BSATTN_RULE_WINDOW: {
+      if (r->win_t < 0 || r->win_h < 0 || r->win_w < 0) return BSATTN_ERR_INVALID_ARG;
+      long long a = 2LL * r->win_t + 1, b = 2LL * r->win_h + 1, c = 2LL * r->win_w + 1;
+      long long nt = Tp / d->tile_t, nh = Hp / d->tile_h, nw = Wp / d->tile_w;
+      kmax = (int)((a < nt ? a : nt) * (b < nh ? b : nh) * (c < nw ? c : nw));
+      break;
+    }
+    default:
+      return BSATTN_ERR_INVALID_ARG;
+  }
+
+  bsattn_plan* p = new (std::nothrow) bsattn_plan();
+  if (!p) return BSATTN_ERR_INTERNAL;
+  p->desc = *d;
+  p->rule = *r;
+  p->Tp = (int)Tp; p->Hp = (int)Hp; p->Wp = (int)Wp;
+  p->nT = (int)(Tp / d->tile_t); p->nH = (int)(Hp / d->tile_h); p->nW = (int)(Wp / d->tile_w);
+  p->N = (int)N; p->V = 64; p->L = (int)L; p->kmax = kmax;
+  p->scale = d->softmax_scale > 0.f ? d->softmax_scale : (float)(1.0 / sqrt((double)d->head_dim));
+  if (cudaGetDevice(&p->device) != cudaSuccess) { delete p; return BSATTN_ERR_CUDA; }
+  if (cudaMalloc(&p->d_err, sizeof(int)) != cudaSuccess) { delete p; return BSATTN_ERR_CUDA; }
+  if (cudaMemset(p->d_err, 0, sizeof(int)) != cudaSuccess) {
+    attn_plan_destroy(p);
+    return BSATTN_ERR_CUDA;
+  }
+  if (r->kind == BSATTN_RULE_WINDOW) {
+    // Closed-form clipped window lists, ascending because j grows with
+    // (t, h, w) in row-major tile order.
+    std::vector<int32_t> idx((size_t)N * kmax, -1), cnt((size_t)N, 0);
+    for (int i = 0; i < N; ++i) {
+      int ti = i / (p->nH * p->nW), hi = (i / p->nW) % p->nH, wi = i % p->nW;
+      int c = 0;
+      for (int t = ti - r->win_t; t <= ti + r->win_t; ++t)
+        for (int h = hi - r->win_h; h <= hi + r->win_h; ++h)
+          for (int w = wi - r->win_w; w <= wi + r->win_w; ++w) {
+            if (t < 0 || h < 0 || w < 0 || t >= p->nT || h >= p->nH || w >= p->nW) continue;
+            idx[(size_t)i * kmax + c++] = (t * p->nH + h) * p->nW + w;
+          }
+      cnt[i] = c;
+    }
+    if (cudaMalloc(&p->d_win_idx, idx.size() * 4) != cudaSuccess ||
+        cudaMalloc(&p->d_win_cnt, cnt.size() * 4) != cudaSuccess ||
+        cudaMemcpy(p->d_win_idx, idx.data(), idx.size() * 4, cudaMemcpyHostToDevice) != cudaSuccess ||
+        cudaMemcpy(p->d_win_cnt, cnt.data(), cnt.size() * 4, cudaMemcpyHostToDevice) != cudaSuccess) {
+      attn_plan_destroy(p);
+      return BSATTN_ERR_CUDA;
+    }
+  }
+  *out = p;
+  return BSATTN_OK;
+}
+
+void attn_plan_destroy(bsattn_plan* p) {
+  if (!p) return;
+  int cur = -1;
+  cudaGetDevice(&cur);
+  if (cur != p->device) cudaSetDevice(p->device);
+  if (p->d_err) cudaFree(p->d_err);
+  if (p->d_win_idx) cudaFree(p->d_win_idx);
+  if (p->d_win_cnt) cudaFree(p->d_win_cnt);
+  if (cur >= 0 && cur != p->device) cudaSetDevice(cur);
+  delete p;
+}
+
+bsattn_status attn_plan_info(const bsattn_plan* p, bsattn_info* o) {
+  if (!p || !o) return BSATTN_ERR_INVALID_ARG;
+  memset(o, 0, sizeof(*o));
+  o->Tp = p->Tp; o->Hp = p->Hp; o->Wp = p->Wp;
+  o->nT = p->nT; o->nH = p->nH; o->nW = p->nW;
+  o->n_blocks = p->N; o->tile_volume = p->V; o->kmax = p->kmax;
+  o->softmax_scale = p->scale;
+  {
+    Carve c(nullptr);
+    if (p->rule.kind != BSATTN_RULE_WINDOW) carve_select(p, c);
+    o->select_workspace_bytes = align_up(c.off, 256);
+  }
+  o->forward_workspace_bytes = attention_workspace_bytes(p);
+  {
+    Carve c(nullptr);
+    carve_layer(p, c);
+    o->layer_workspace_bytes = align_up(c.off, 256);
+  }
+  return BSATTN_OK;
+}
+
+bsattn_status attn_reorder(const bsattn_plan* p, const void* x_nat, void* x_tiled, float* pooled,
+                           void* stream) {
+  if (!p || !ok_ptr(x_nat) || !ok_ptr(x_tiled) || (pooled && !aligned16(pooled)))
+    return BSATTN_ERR_INVALID_ARG;
+  bsattn_status s = set_device(p);
+  if (s) return s;
+  return launch_reorder(make_geom(p), (const __nv_bfloat16*)x_nat, (__nv_bfloat16*)x_tiled, pooled,
+                        nullptr, nullptr, RO_WRITE_TILED | (pooled ? RO_POOL : 0),
+                        (cudaStream_t)stream);
+}
+
+bsattn_status attn_pool(const bsattn_plan* p, const void* x_nat, float* pooled, void* stream) {
+  if (!p || !ok_ptr(x_nat) || !ok_ptr(pooled)) return BSATTN_ERR_INVALID_ARG;
+  bsattn_status s = set_device(p);
+  if (s) return s;
+  return launch_reorder(make_geom(p), (const __nv_bfloat16*)x_nat, nullptr, pooled, nullptr,
+                        nullptr, RO_POOL, (cudaStream_t)stream);
+}
+
+bsattn_status attn_unreorder(const bsattn_plan* p, const void* x_tiled, void* x_nat,
+                             void* stream) {
+  if (!p || !ok_ptr(x_tiled) || !ok_ptr(x_nat)) return BSATTN_ERR_INVALID_ARG;
+  bsattn_status s = set_device(p);
+  if (s) return s;
+  return launch_unreorder(make_geom(p), (const __nv_bfloat16*)x_tiled, (__nv_bfloat16*)x_nat,
+                          nullptr, nullptr, (cudaStream_t)stream);
+}
+
+bsattn_status attn_block_scores(const bsattn_plan* p, const float* pq, const float* pk,
+                                float* S, void* stream) {
+  if (!p || !ok_ptr(pq) || !ok_ptr(pk) || !ok_ptr(S)) return BSATTN_ERR_INVALID_ARG;
+  bsattn_status s = set_device(p);
+  if (s) return s;
+  return launch_block_scores(make_geom(p), pq, pk, p->scale, S, (cudaStream_t)stream);
+}
+
+static bsattn_status select_core(const bsattn_plan* p, const float* S, int32_t* idx,
+                                 int32_t* cnt, cudaStream_t st) {
+  int rows = p->desc.B * p->desc.heads * p->N;
+  switch (p->rule.kind) {
+    case BSATTN_RULE_TOPK:
+      return launch_select_topk(rows, p->N, p->rule.k, S, idx, cnt, p->kmax, st);
+    case BSATTN_RULE_TOPP:
+      return launch_select_topp(rows, p->N, p->rule.k, p->rule.p, S, idx, cnt, p->kmax, st);
+    default:
+      return launch_broadcast_lists(p->desc.B * p->desc.heads, p->N, p->kmax, p->d_win_idx,
+                                    p->d_win_cnt, idx, cnt, st);
+  }
+}
+
+bsattn_status attn_select_from_scores(const bsattn_plan* p, const float* S, int32_t* idx,
+                                      int32_t* cnt, void* stream) {
+  if (!p || !ok_ptr(idx) || !ok_ptr(cnt)) return BSATTN_ERR_INVALID_ARG;
+  if (p->rule.kind != BSATTN_RULE_WINDOW && !ok_ptr(S)) return BSATTN_ERR_INVALID_ARG;
+  bsattn_status s = set_device(p);
+  if (s) return s;
+  return select_core(p, S, idx, cnt, (cudaStream_t)stream);
+}
+
+bsattn_status attn_select(const bsattn_plan* p, const void* q_nat, const void* k_nat,
+                          int32_t* idx, int32_t* cnt, void* ws, size_t ws_bytes, void* stream) {
+  if (!p || !ok_ptr(idx) || !ok_ptr(cnt)) return BSATTN_ERR_INVALID_ARG;
+  bsattn_info info;
+  attn_plan_info(p, &info);
+  cudaStream_t st = (cudaStream_t)stream;
+  bsattn_status s = set_device(p);
+  if (s) return s;
+  if (p->rule.kind == BSATTN_RULE_WINDOW) return select_core(p, nullptr, idx, cnt, st);
+  if (!ok_ptr(q_nat) || !ok_ptr(k_nat)) return BSATTN_ERR_INVALID_ARG;
+  if (!ws || !aligned16(ws) || ws_bytes < info.select_workspace_bytes) return BSATTN_ERR_WORKSPACE;
+  Carve c(ws);
+  SelectWs w = carve_select(p, c);
+  Geom g = make_geom(p);
+  if ((s = launch_reorder(g, (const __nv_bfloat16*)q_nat, nullptr, w.pq, nullptr, nullptr, RO_POOL, st)))
+    return s;
+  if ((s = launch_reorder(g, (const __nv_bfloat16*)k_nat, nullptr, w.pk, nullptr, nullptr, RO_POOL, st)))
+    return s;
+  if ((s = launch_block_scores(g, w.pq, w.pk, p->scale, w.S, st))) return s;
+  return select_core(p, w.S, idx, cnt, st);
+}
+
+bsattn_status attn_quantize_e4m3(const bsattn_plan* p, const void* x_tiled, uint8_t* codes,
+                                 float* scales, void* stream) {
+  if (!p || !ok_ptr(x_tiled) || !ok_ptr(codes) || !ok_ptr(scales)) return BSATTN_ERR_INVALID_ARG;
+  bsattn_status s = set_device(p);
+  if (s) return s;
+  return launch_quant_tiled(make_geom(p), (const __nv_bfloat16*)x_tiled, codes, scales,
+                            (cudaStream_t)stream);
+}
+
+bsattn_status attn_forward(const bsattn_plan* p, const void* q, const void* k, const float* qs,
+                           const float* ks, const void* v, const int32_t* idx, const int32_t* cnt,
+                           void* o, float* lse, void* ws, size_t ws_bytes, void* stream) {
+  if (!p || !ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(idx) || !ok_ptr(cnt) || !ok_ptr(o) ||
+      (lse && !aligned16(lse)))
+    return BSATTN_ERR_INVALID_ARG;
+  if (p->desc.qk_fp8 && (!ok_ptr(qs) || !ok_ptr(ks))) return BSATTN_ERR_INVALID_ARG;
+  size_t need = attention_workspace_bytes(p);
+  if (need && (!ws || !aligned16(ws) || ws_bytes < need)) return BSATTN_ERR_WORKSPACE;
+  bsattn_status s = set_device(p);
+  if (s) return s;
+  return launch_attention(p, q, k, qs, ks, (const __nv_bfloat16*)v, idx, cnt, (__nv_bfloat16*)o,
+                          lse, ws, ws_bytes, (cudaStream_t)stream);
+}
+
+bsattn_status attn_layer(const bsattn_plan* p, const void* q_nat, const void* k_nat,
+                         const void* v_nat, void* o_nat, float* lse_nat, int32_t* idx_out,
+                         int32_t* cnt_out, void* ws, size_t ws_bytes, void* stream) {
+  if (!p || !ok_ptr(q_nat) || !ok_ptr(k_nat) || !ok_ptr(v_nat) || !ok_ptr(o_nat) ||
+      (lse_nat && !aligned16(lse_nat)) || (idx_out && !aligned16(idx_out)) ||
+      (cnt_out && !aligned16(cnt_out)) || ((idx_out == nullptr) != (cnt_out == nullptr)))
+    return BSATTN_ERR_INVALID_ARG;
+  bsattn_info info;
+  attn_plan_info(p, &info);
+  if (!ws || !aligned16(ws) || ws_bytes < info.layer_workspace_bytes) return BSATTN_ERR_WORKSPACE;
+  bsattn_status s = set_device(p);
+  if (s) return s;
+  cudaStream_t st = (cudaStream_t)stream;
+  Carve c(ws);
+  LayerWs w = carve_layer(p, c);
+  Geom g = make_geom(p);
+  int32_t* idx = idx_out ? idx_out : w.idx;
+  int32_t* cnt = cnt_out ? cnt_out : w.cnt;
+  bool pool = p->rule.kind != BSATTN_RULE_WINDOW;
+  if (p->desc.qk_fp8) {
+    int f = RO_QUANT | (pool ? RO_POOL : 0);
+    if ((s = launch_reorder(g, (const __nv_bfloat16*)q_nat, nullptr, w.sel.pq, (uint8_t*)w.qt, w.qs, f, st)))
+      return s;
+    if ((s = launch_reorder(g, (const __nv_bfloat16*)k_nat, nullptr, w.sel.pk, (uint8_t*)w.kt, w.ks, f, st)))
+      return s;
+  } else {
+    int f = RO_WRITE_TILED | (pool ? RO_POOL : 0);
+    if ((s = launch_reorder(g, (const __nv_bfloat16*)q_nat, (__nv_bfloat16*)w.qt, w.sel.pq, nullptr, nullptr, f, st)))
+      return s;
+    if ((s = launch_reorder(g, (const __nv_bfloat16*)k_nat, (__nv_bfloat16*)w.kt, w.sel.pk, nullptr, nullptr, f, st)))
+      return s;
+  }
+  if ((s = launch_reorder(g, (const __nv_bfloat16*)v_nat, w.vt, nullptr, nullptr, nullptr, RO_WRITE_TILED, st)))
+    return s;
+  if (pool && (s = launch_block_scores(g, w.sel.pq, w.sel.pk, p->scale, w.sel.S, st))) return s;
+  if ((s = select_core(p, w.sel.S, idx, cnt, st))) return s;
+  if ((s = launch_attention(p, w.qt, w.kt, w.qs, w.ks, w.vt, idx, cnt, w.ot,
+                            lse_nat ? w.lse_t : nullptr, w.attn_ws,
+                            attention_workspace_bytes(p), st)))
+    return s;
+  return launch_unreorder(g, w.ot, (__nv_bfloat16*)o_nat, lse_nat ? w.lse_t : nullptr, lse_nat, st);
+}
+
+bsattn_status attn_check_device_status(const bsattn_plan* p, void* stream) {
+  if (!p) return BSATTN_ERR_INVALID_ARG;
+  bsattn_status s = set_device(p);
+  if (s) return s;
+  BSATTN_CUDA_TRY(cudaStreamSynchronize((cudaStream_t)stream));
+  int h = 0;
+  BSATTN_CUDA_TRY(cudaMemcpy(&h, p->d_err, sizeof(int), cudaMemcpyDeviceToHost));
+  if (h) BSATTN_CUDA_TRY(cudaMemset(p->d_err, 0, sizeof(int)));
+  if (h & BSATTN_DEVERR_TIMEOUT) return BSATTN_ERR_TIMEOUT;
+  if (h & BSATTN_DEVERR_BAD_INDEX) return BSATTN_ERR_INTERNAL;
+  return BSATTN_OK;
+}
+
+}  // extern "C"

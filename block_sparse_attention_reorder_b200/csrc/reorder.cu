@@ -1,0 +1,243 @@
+// Tile reorder (natural -> tiled) with fused tile-mean pooling and per-tile
+// e4m3 quantisation, the inverse scatter, and standalone tile quantisation.
+//
+// These steps move bytes: one CTA per (batch, head, tile) moves the tile's
+// 64 rows of D bf16 with 16-byte vector accesses. Reads are 64 row segments
+// of 2*D bytes (the natural layout interleaves heads), writes are one
+// contiguous 64*D*2-byte block, so both sides use full 32-byte sectors.
+#include <cuda_fp8.h>
+
+#include "internal.h"
+
+namespace {
+
+constexpr int kThreads = 256;
+
+struct TileCoord {
+  int t0, h0, w0;     // first token coordinate of the tile
+  int vt, vh, vw;     // real extent along each axis (<= tile)
+};
+
+__device__ __forceinline__ TileCoord tile_coord(const Geom& g, int j) {
+  TileCoord c;
+  int bt = j / (g.nH * g.nW), bh = (j / g.nW) % g.nH, bw = j % g.nW;
+  c.t0 = bt * g.tt; c.h0 = bh * g.th; c.w0 = bw * g.tw;
+  c.vt = min(g.tt, g.T - c.t0); c.vh = min(g.th, g.H - c.h0); c.vw = min(g.tw, g.W - c.w0);
+  return c;
+}
+
+// Natural token index of in-tile row r, or -1 for a padded slot.
+__device__ __forceinline__ int row_token(const Geom& g, const TileCoord& c, int r) {
+  int dt = r / (g.th * g.tw), dh = (r / g.tw) % g.th, dw = r % g.tw;
+  if (dt >= c.vt || dh >= c.vh || dw >= c.vw) return -1;
+  return ((c.t0 + dt) * g.H + (c.h0 + dh)) * g.W + (c.w0 + dw);
+}
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float* f) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float2 x = __bfloat1622float2(h[i]);
+    f[2 * i] = x.x;
+    f[2 * i + 1] = x.y;
+  }
+}
+
+__device__ __forceinline__ float block_max(float v, float* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  int w = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0) red[w] = v;
+  __syncthreads();
+  float m = red[0];
+#pragma unroll
+  for (int i = 1; i < kThreads / 32; ++i) m = fmaxf(m, red[i]);
+  return m;
+}
+
+// e4m3 codes of 8 values divided by `scale` (IEEE fp32 division), RNE, satfinite.
+__device__ __forceinline__ uint2 quant8(const float* f, float scale) {
+  uint32_t w[2];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    uint32_t acc = 0;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      float2 x = make_float2(__fdiv_rn(f[4 * h + 2 * i], scale), __fdiv_rn(f[4 * h + 2 * i + 1], scale));
+      __nv_fp8x2_storage_t p = __nv_cvt_float2_to_fp8x2(x, __NV_SATFINITE, __NV_E4M3);
+      acc |= (uint32_t)p << (16 * i);
+    }
+    w[h] = acc;
+  }
+  return make_uint2(w[0], w[1]);
+}
+
+__device__ __forceinline__ float tile_scale_from_amax(float amax) {
+  return amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads)
+reorder_kernel(Geom g, const __nv_bfloat16* __restrict__ x_nat, __nv_bfloat16* __restrict__ x_tiled,
+               float* __restrict__ pooled, uint8_t* __restrict__ codes, float* __restrict__ scales,
+               int flags) {
+  constexpr int CH = D / 8;                 // 16-byte chunks per row
+  constexpr int ITER = 64 * CH / kThreads;  // chunks per thread
+  constexpr int RSTEP = kThreads / CH;      // row stride between a thread's chunks
+  __shared__ float red[RSTEP][D + 1];
+  __shared__ float wred[kThreads / 32];
+
+  const int j = blockIdx.x, head = blockIdx.y, b = blockIdx.z;
+  const int c = threadIdx.x % CH;
+  const int r0 = threadIdx.x / CH;
+  const TileCoord tc = tile_coord(g, j);
+  const size_t tile_off = (((size_t)b * g.Hh + head) * g.N + j) * 64;
+
+  uint4 v[ITER];
+#pragma unroll
+  for (int i = 0; i < ITER; ++i) {
+    int r = r0 + RSTEP * i;
+    int n = row_token(g, tc, r);
+    if (n >= 0) {
+      const uint4* src = reinterpret_cast<const uint4*>(x_nat + (((size_t)b * g.L + n) * g.Hh + head) * D) + c;
+      v[i] = __ldg(src);
+    } else {
+      v[i] = make_uint4(0, 0, 0, 0);
+    }
+  }
+  if (flags & RO_WRITE_TILED) {
+#pragma unroll
+    for (int i = 0; i < ITER; ++i) {
+      int r = r0 + RSTEP * i;
+      reinterpret_cast<uint4*>(x_tiled + (tile_off + r) * D)[c] = v[i];
+    }
+  }
+  if (flags & RO_POOL) {
+    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+#pragma unroll
+    for (int i = 0; i < ITER; ++i) {
+      float f[8];
+      bf16x8_to_f32(v[i], f);  // padded slots hold zeros
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] += f[e];
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) red[r0][c * 8 + e] = acc[e];
+    __syncthreads();
+    if (threadIdx.x < D) {
+      float s = 0.f;
+#pragma unroll
+      for (int q = 0; q < RSTEP; ++q) s += red[q][threadIdx.x];
+      float nvalid = (float)(tc.vt * tc.vh * tc.vw);
+      pooled[(((size_t)b * g.Hh + head) * g.N + j) * D + threadIdx.x] = __fdiv_rn(s, nvalid);
+    }
+  }
+  if (flags & RO_QUANT) {
+    float m = 0.f;
+#pragma unroll
+    for (int i = 0; i < ITER; ++i) {
+      float f[8];
+      bf16x8_to_f32(v[i], f);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(f[e]));
+    }
+    float scale = tile_scale_from_amax(block_max(m, wred));
+#pragma unroll
+    for (int i = 0; i < ITER; ++i) {
+      int r = r0 + RSTEP * i;
+      float f[8];
+      bf16x8_to_f32(v[i], f);
+      reinterpret_cast<uint2*>(codes + (tile_off + r) * D)[c] = quant8(f, scale);
+    }
+    if (threadIdx.x == 0) scales[((size_t)b * g.Hh + head) * g.N + j] = scale;
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads)
+unreorder_kernel(Geom g, const __nv_bfloat16* __restrict__ x_tiled, __nv_bfloat16* __restrict__ x_nat,
+                 const float* __restrict__ lse_tiled, float* __restrict__ lse_nat) {
+  constexpr int CH = D / 8;
+  constexpr int ITER = 64 * CH / kThreads;
+  constexpr int RSTEP = kThreads / CH;
+  const int j = blockIdx.x, head = blockIdx.y, b = blockIdx.z;
+  const int c = threadIdx.x % CH;
+  const int r0 = threadIdx.x / CH;
+  const TileCoord tc = tile_coord(g, j);
+  const size_t tile_off = (((size_t)b * g.Hh + head) * g.N + j) * 64;
+#pragma unroll
+  for (int i = 0; i < ITER; ++i) {
+    int r = r0 + RSTEP * i;
+    int n = row_token(g, tc, r);
+    if (n < 0) continue;
+    uint4 v = __ldg(reinterpret_cast<const uint4*>(x_tiled + (tile_off + r) * D) + c);
+    reinterpret_cast<uint4*>(x_nat + (((size_t)b * g.L + n) * g.Hh + head) * D)[c] = v;
+  }
+  if (lse_tiled && threadIdx.x < 64) {
+    int n = row_token(g, tc, threadIdx.x);
+    if (n >= 0) lse_nat[((size_t)b * g.Hh + head) * g.L + n] = lse_tiled[tile_off + threadIdx.x];
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads)
+quant_tiled_kernel(Geom g, const __nv_bfloat16* __restrict__ x_tiled, uint8_t* __restrict__ codes,
+                   float* __restrict__ scales) {
+  constexpr int CH = D / 8;
+  constexpr int ITER = 64 * CH / kThreads;
+  __shared__ float wred[kThreads / 32];
+  const size_t tile = ((size_t)blockIdx.z * g.Hh + blockIdx.y) * g.N + blockIdx.x;
+  const uint4* src = reinterpret_cast<const uint4*>(x_tiled + tile * 64 * D);
+  uint4 v[ITER];
+  float m = 0.f;
+#pragma unroll
+  for (int i = 0; i < ITER; ++i) {
+    v[i] = __ldg(src + threadIdx.x + kThreads * i);
+    float f[8];
+    bf16x8_to_f32(v[i], f);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(f[e]));
+  }
+  float scale = tile_scale_from_amax(block_max(m, wred));
+  uint2* dst = reinterpret_cast<uint2*>(codes + tile * 64 * D);
+#pragma unroll
+  for (int i = 0; i < ITER; ++i) {
+    float f[8];
+    bf16x8_to_f32(v[i], f);
+    dst[threadIdx.x + kThreads * i] = quant8(f, scale);
+  }
+  if (threadIdx.x == 0) scales[tile] = scale;
+}
+
+}  // namespace
+
+bsattn_status launch_reorder(const Geom& g, const __nv_bfloat16* x_nat, __nv_bfloat16* x_tiled,
+                             float* pooled, uint8_t* codes, float* scales, int flags,
+                             cudaStream_t st) {
+  dim3 grid(g.N, g.Hh, g.B);
+  if (g.D == 128)
+    reorder_kernel<128><<<grid, kThreads, 0, st>>>(g, x_nat, x_tiled, pooled, codes, scales, flags);
+  else
+    reorder_kernel<64><<<grid, kThreads, 0, st>>>(g, x_nat, x_tiled, pooled, codes, scales, flags);
+  return cudaGetLastError() == cudaSuccess ? BSATTN_OK : BSATTN_ERR_CUDA;
+}
+
+bsattn_status launch_unreorder(const Geom& g, const __nv_bfloat16* x_tiled, __nv_bfloat16* x_nat,
+                               const float* lse_tiled, float* lse_nat, cudaStream_t st) {
+  dim3 grid(g.N, g.Hh, g.B);
+  if (g.D == 128)
+    unreorder_kernel<128><<<grid, kThreads, 0, st>>>(g, x_tiled, x_nat, lse_tiled, lse_nat);
+  else
+    unreorder_kernel<64><<<grid, kThreads, 0, st>>>(g, x_tiled, x_nat, lse_tiled, lse_nat);
+  return cudaGetLastError() == cudaSuccess ? BSATTN_OK : BSATTN_ERR_CUDA;
+}
+
+bsattn_status launch_quant_tiled(const Geom& g, const __nv_bfloat16* x_tiled, uint8_t* codes,
+                                 float* scales, cudaStream_t st) {
+  dim3 grid(g.N, g.Hh, g.B);
+  if (g.D == 128)
+    quant_tiled_kernel<128><<<grid, kThreads, 0, st>>>(g, x_tiled, codes, scales);
+  else
+    quant_tiled_kernel<64><<<grid, kThreads, 0, st>>>(g, x_tiled, codes, scales);
+  return cudaGetLastError() == cudaSuccess ? BSATTN_OK : BSATTN_ERR_CUDA;
+}

@@ -1,0 +1,192 @@
+/*
+ * bsattn.h — C ABI of the block-sparse attention library for 3D-tiled video
+ * latent tokens (sm_100a).
+ *
+ * The method (sources named per entry point below):
+ *   1. reorder the tokens of a T x H x W latent grid into (t, h, w) tiles
+ *      ("video-aware block organisation", FVAttn summary page, Summary;
+ *      "shared 3D tile granularity", FPSAttention page, Approach);
+ *   2. mean-pool Q and K per tile and score tile pairs;
+ *   3. keep, per query tile, a set of key tiles: top-k, top-p with a top-k
+ *      floor (FVAttn summary page, Summary and Abstract), or a fixed 3D tile
+ *      window (FPSAttention page, ablation rows on sparsity windows);
+ *   4. run softmax attention over the kept tile pairs only (FPSAttention
+ *      page, Approach; trainable sparse attention record, Research Type and
+ *      Hardware Specification rows), optionally with Q/K quantised to e4m3
+ *      per tile (FPSAttention page, Approach).
+ *
+ * Conventions for every entry point:
+ *   - Device pointers are owned by the caller; the library never allocates
+ *     on the hot path. A plan owns only host metadata plus a few small
+ *     device buffers made at create time (window lists, error word).
+ *   - All device pointers must be 16-byte aligned. Tensors are dense,
+ *     row-major, with the layouts stated below.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream). Calls enqueue work and return; nothing synchronises except
+ *     attn_check_device_status.
+ *   - Argument errors are reported before anything is enqueued. A failed
+ *     launch returns BSATTN_ERR_CUDA. Kernels never trap: an out-of-range
+ *     list entry or an exhausted bounded wait sets the plan's device error
+ *     word and the affected work is skipped; attn_check_device_status
+ *     reports it.
+ *   - A plan is bound to the device that was current at attn_plan_create
+ *     and is immutable afterwards, so it may be used from several streams
+ *     at once (calls that share output buffers must still be ordered by the
+ *     caller).
+ *   - Block scores containing NaN give unspecified (but in-bounds) lists.
+ *
+ * Layouts (B batch, Hh heads, D head_dim, L = T*H*W, N = number of tiles,
+ * V = tile volume = tile_t*tile_h*tile_w = 64):
+ *   natural   [B, L, Hh, D] bf16, token n = (t*H + h)*W + w
+ *   tiled     [B, Hh, N, V, D] (bf16, or u8 e4m3 codes), tile id
+ *             j = ((t/tile_t)*nH + h/tile_h)*nW + w/tile_w, in-tile row
+ *             ((t%tile_t)*tile_h + h%tile_h)*tile_w + w%tile_w; padded
+ *             slots (t>=T, h>=H or w>=W) are zero
+ *   pooled    [B, Hh, N, D] fp32, mean over the tile's real tokens
+ *   scores    [B, Hh, N, N] fp32, S[i][j] = softmax_scale * qbar_i . kbar_j
+ *   idx       [B, Hh, N, kmax] int32, ascending kept key tiles of each query
+ *             tile; entries at and beyond cnt are unspecified
+ *   cnt       [B, Hh, N] int32
+ *   tile scale [B, Hh, N] fp32 (e4m3 path)
+ *   lse       natural [B, Hh, L] fp32 (attn_layer) or tiled [B, Hh, N, V]
+ *             fp32 (attn_forward); natural-log sum of exp(scaled scores)
+ */
+#ifndef BSATTN_H
+#define BSATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  BSATTN_OK = 0,
+  BSATTN_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad size or rule */
+  BSATTN_ERR_UNSUPPORTED = 2,  /* valid request outside the supported set   */
+  BSATTN_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed      */
+  BSATTN_ERR_TIMEOUT = 4,      /* a bounded device wait ran out             */
+  BSATTN_ERR_INTERNAL = 5,     /* device error word: bad list entry etc.    */
+  BSATTN_ERR_WORKSPACE = 6     /* workspace pointer null or too small       */
+} bsattn_status;
+
+typedef enum {
+  BSATTN_RULE_TOPK = 0,   /* k largest scores, ties to the lower tile index */
+  BSATTN_RULE_TOPP = 1,   /* smallest prefix with softmax mass >= p, >= k   */
+  BSATTN_RULE_WINDOW = 2  /* |dt|<=win_t, |dh|<=win_h, |dw|<=win_w in tiles */
+} bsattn_rule_kind;
+
+typedef struct {
+  int kind;              /* bsattn_rule_kind                                 */
+  int k;                 /* top-k: count (1..N); top-p: floor (0..N)          */
+  double p;              /* top-p: mass threshold in (0, 1]                   */
+  int win_t, win_h, win_w; /* window half-widths in tiles (>= 0)             */
+} bsattn_rule;
+
+typedef struct {
+  int B, heads, head_dim;       /* head_dim in {64, 128}                      */
+  int T, H, W;                  /* latent grid, each >= 1                     */
+  int tile_t, tile_h, tile_w;   /* tile shape; volume must be 64              */
+  float softmax_scale;          /* <= 0 selects 1/sqrt(head_dim)              */
+  int qk_fp8;                   /* 1: attn_forward takes per-tile e4m3 Q/K    */
+} bsattn_desc;
+
+typedef struct {
+  int Tp, Hp, Wp;               /* padded grid                                */
+  int nT, nH, nW;               /* tiles per axis                             */
+  int n_blocks;                 /* N = nT*nH*nW                               */
+  int tile_volume;              /* V = 64                                     */
+  int kmax;                     /* idx row capacity                           */
+  float softmax_scale;          /* resolved scale                             */
+  size_t select_workspace_bytes;  /* attn_select                              */
+  size_t forward_workspace_bytes; /* attn_forward                             */
+  size_t layer_workspace_bytes;   /* attn_layer                               */
+} bsattn_info;
+
+typedef struct bsattn_plan bsattn_plan;
+
+/* Validate a problem and rule and build a plan (host metadata; for the
+ * window rule also the closed-form kept lists, copied once to the device;
+ * a 4-byte device error word). The current CUDA device is bound to the plan.
+ * Errors: INVALID_ARG (null, non-positive sizes, k outside its range,
+ * p outside (0,1], negative half-widths), UNSUPPORTED (head_dim not 64/128,
+ * tile volume != 64, N above 2048 for top-k/top-p), CUDA. */
+bsattn_status attn_plan_create(const bsattn_desc* desc, const bsattn_rule* rule,
+                               bsattn_plan** out);
+void attn_plan_destroy(bsattn_plan* plan);
+bsattn_status attn_plan_info(const bsattn_plan* plan, bsattn_info* out);
+const char* attn_status_string(bsattn_status s);
+
+/* Step 1 (+2): gather natural bf16 tokens into the tiled layout with zero
+ * pads; if `pooled` is non-NULL also write the fp32 tile means over real
+ * tokens (pooling for the block scores; the pages leave the pooling function
+ * open, the mean is this library's reading). */
+bsattn_status attn_reorder(const bsattn_plan* plan, const void* x_nat, void* x_tiled,
+                           float* pooled, void* stream);
+
+/* Step 2 alone: fp32 tile means of natural bf16 tokens, no tiled copy. */
+bsattn_status attn_pool(const bsattn_plan* plan, const void* x_nat, float* pooled,
+                        void* stream);
+
+/* Inverse of step 1: scatter tiled bf16 rows of real tokens back to the
+ * natural layout (padded slots are dropped). */
+bsattn_status attn_unreorder(const bsattn_plan* plan, const void* x_tiled, void* x_nat,
+                             void* stream);
+
+/* Step 2: block scores S = softmax_scale * pooled_q . pooled_k^T per
+ * (batch, head), fp32, accumulated in order d = 0..D-1. */
+bsattn_status attn_block_scores(const bsattn_plan* plan, const float* pooled_q,
+                                const float* pooled_k, float* scores, void* stream);
+
+/* Step 3 on a given score matrix: the plan's rule applied row by row.
+ * Top-k: the k largest by (score descending, index ascending); -0.0 and
+ * +0.0 tie. Top-p: in that order, the shortest prefix whose softmax mass
+ * (fp64 exp, sum and scan) reaches p, then at least k and at most N tiles.
+ * Window: the plan's closed-form lists (scores unused, may be NULL).
+ * Lists come out ascending. */
+bsattn_status attn_select_from_scores(const bsattn_plan* plan, const float* scores,
+                                      int32_t* idx, int32_t* cnt, void* stream);
+
+/* Steps 2-3 from natural Q and K: pool, score, select. `ws` must hold
+ * info.select_workspace_bytes (pooled Q/K and the score matrix). */
+bsattn_status attn_select(const bsattn_plan* plan, const void* q_nat, const void* k_nat,
+                          int32_t* idx, int32_t* cnt, void* ws, size_t ws_bytes,
+                          void* stream);
+
+/* Per-tile e4m3 quantisation of a tiled bf16 tensor: per (b, head, tile)
+ * scale = fp32(amax)/448 (amax 0 -> 1), code = e4m3(x/scale) rounded to
+ * nearest even with finite saturation (OCP E4M3). */
+bsattn_status attn_quantize_e4m3(const bsattn_plan* plan, const void* x_tiled,
+                                 uint8_t* codes, float* scales, void* stream);
+
+/* Step 4: block-sparse attention on tiled inputs. q/k are bf16, or e4m3
+ * codes with per-tile scales when the plan has qk_fp8 (q_scale/k_scale are
+ * then required, else ignored). For every query tile i and j in
+ * idx[..., i, :cnt]: S = scale * Q_i K_j^T (times q_scale_i * k_scale_j on
+ * the e4m3 path), padded keys masked, fp32 online softmax, P rounded to
+ * bf16, O += P V_j; O /= row sum. Writes tiled bf16 O (padded rows too) and,
+ * if non-NULL, tiled fp32 lse. `ws`: info.forward_workspace_bytes (may be 0). */
+bsattn_status attn_forward(const bsattn_plan* plan, const void* q, const void* k,
+                           const float* q_scale, const float* k_scale, const void* v,
+                           const int32_t* idx, const int32_t* cnt, void* o_tiled,
+                           float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/* The whole layer on natural tensors: reorder + pool (+ e4m3 quantisation),
+ * block scores, selection, block-sparse attention, unreorder. Writes natural
+ * bf16 O and, if non-NULL, natural fp32 lse [B, Hh, L]. If idx_out/cnt_out
+ * are non-NULL the kept lists are also copied there. `ws` must hold
+ * info.layer_workspace_bytes. */
+bsattn_status attn_layer(const bsattn_plan* plan, const void* q_nat, const void* k_nat,
+                         const void* v_nat, void* o_nat, float* lse_nat, int32_t* idx_out,
+                         int32_t* cnt_out, void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronise `stream`, read and clear the plan's device error word.
+ * Returns OK, TIMEOUT or INTERNAL (bad list entry), or CUDA. */
+bsattn_status attn_check_device_status(const bsattn_plan* plan, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BSATTN_H */

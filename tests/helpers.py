@@ -1,0 +1,68 @@
+"""Shared test utilities: small ragged workloads, tensor conversion, and
+oracle-side list checks. Test infrastructure only."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from block_sparse_attention_reorder_b200.datagen import Workload
+from oracle import select
+
+# Small cases the oracle finishes in seconds that still span several tiles
+# and a ragged tail along every axis.
+SMALL = {
+    "tiny_d64": Workload("tiny_d64", 1, 2, 64, 8, 16, 16, "topk", k=8, recipe="iid", seed=0),
+    "ragged_topk": Workload("ragged_topk", 2, 3, 128, 7, 10, 13, "topk", k=5, seed=11),
+    "ragged_topp": Workload("ragged_topp", 1, 3, 128, 7, 10, 13, "topp", k=3, p=0.9, seed=12,
+                            temperature=(0.3, 3.0)),
+    "ragged_window_fp8": Workload("ragged_window_fp8", 1, 2, 128, 9, 10, 13, "window",
+                                  win=(1, 1, 0), qk_fp8=True, seed=13),
+    "ragged_d64_fp8": Workload("ragged_d64_fp8", 1, 2, 64, 5, 9, 6, "topk", k=4, qk_fp8=True,
+                               seed=14),
+    "ragged_bf16_window": Workload("ragged_bf16_window", 1, 2, 128, 6, 6, 9, "window",
+                                   win=(1, 0, 1), seed=15),
+}
+
+
+def to64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
+def lists_from_device(idx: torch.Tensor, cnt: torch.Tensor):
+    idx = idx.cpu().numpy().reshape(-1, idx.shape[-1])
+    cnt = cnt.cpu().numpy().reshape(-1)
+    return [idx[r, :cnt[r]].astype(np.int64) for r in range(cnt.size)]
+
+
+def lists_to_device(lists, kmax: int, device="cuda"):
+    rows = len(lists)
+    idx = np.full((rows, kmax), -1, dtype=np.int32)
+    cnt = np.zeros((rows,), dtype=np.int32)
+    for r, l in enumerate(lists):
+        idx[r, :len(l)] = l
+        cnt[r] = len(l)
+    return torch.from_numpy(idx).to(device), torch.from_numpy(cnt).to(device)
+
+
+def assert_topp_equal(got, S_row, p, k):
+    """GPU top-p list vs the oracle's on the same fp32 row; a count that differs
+    by one is accepted only at an fp64 rounding tie (|c_m - p| < 1e-12)."""
+    want_cnt, c = select.topp_count(S_row, p, k)
+    order = select.rank_order(S_row)
+    n = len(got)
+    if n != want_cnt:
+        lo = min(n, want_cnt)
+        assert abs(n - want_cnt) == 1 and lo >= k and abs(c[lo - 1] - p) < 1e-12, (n, want_cnt)
+    np.testing.assert_array_equal(np.asarray(got), np.sort(order[:n]))
+
+
+def assert_valid_selection(got, S_row64, rule, k=0, p=0.0, eps=1e-5):
+    """Lists computed from fp32 scores are a valid selection under the oracle's
+    fp64 scores up to `eps` (only near-ties may be decided differently)."""
+    got = np.asarray(got)
+    n = S_row64.shape[0]
+    dropped = np.setdiff1d(np.arange(n), got)
+    if rule == "topk":
+        assert got.size == min(k, n)
+    if rule in ("topk", "topp") and got.size and dropped.size:
+        assert S_row64[got].min() >= S_row64[dropped].max() - eps

@@ -1,0 +1,72 @@
+"""Host-side checks of the C ABI: the library loads, exports every declared
+entry point, and rejects bad arguments before touching the device (CPU only)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "bsattn.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(attn_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_api():
+    names = declared_functions()
+    for must in ("attn_plan_create", "attn_select", "attn_forward", "attn_layer"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol():
+    from block_sparse_attention_reorder_b200 import bsattn
+    lib = ctypes.CDLL(bsattn.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert set(declared_functions()) == set(bsattn.EXPORTED)
+
+
+def test_status_strings():
+    from block_sparse_attention_reorder_b200 import bsattn
+    for code in range(7):
+        assert bsattn.attn_status_string(code) == bsattn.STATUS[code]
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(head_dim=96), 2),                     # unsupported head_dim
+    (dict(tile=(4, 4, 8)), 2),                  # tile volume 128
+    (dict(T=0), 1),                             # empty grid
+    (dict(B=0), 1),
+    (dict(k=0), 1),                             # top-k needs k >= 1
+    (dict(k=33), 1),                            # k > N (N = 32)
+    (dict(rule="topp", k=2, p=0.0), 1),         # p outside (0, 1]
+    (dict(rule="topp", k=2, p=1.5), 1),
+    (dict(rule="topp", k=-1, p=0.5), 1),
+    (dict(rule="window", win=(-1, 0, 0)), 1),
+    (dict(rule=7), 1),
+    (dict(T=4 * 32, H=4 * 8, W=4 * 9, k=8), 2),  # N = 2304 > 2048 for top-k
+])
+def test_plan_rejects_bad_arguments_before_any_device_call(kw, code):
+    from block_sparse_attention_reorder_b200 import bsattn
+    args = dict(B=1, heads=2, head_dim=64, T=8, H=16, W=16, rule="topk", k=8)
+    args.update(kw)
+    with pytest.raises(bsattn.BsattnError) as e:
+        bsattn.Plan(**args)
+    assert e.value.code == code
+
+
+def test_null_plan_and_null_pointers_are_invalid():
+    from block_sparse_attention_reorder_b200 import bsattn
+    lib = bsattn._lib
+    assert lib.attn_plan_create(None, None, None) == 1
+    assert lib.attn_reorder(None, None, None, None, None) == 1
+    assert lib.attn_forward(None, None, None, None, None, None, None, None, None, None, None, 0,
+                            None) == 1
+    assert lib.attn_layer(None, None, None, None, None, None, None, None, None, 0, None) == 1
+    assert lib.attn_check_device_status(None, None) == 1
+    assert lib.attn_plan_info(None, None) == 1
+    lib.attn_plan_destroy(None)  # no-op

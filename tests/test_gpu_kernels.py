@@ -1,0 +1,211 @@
+"""Kernel-level parity: each C-ABI step against the oracle on the same inputs."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_attention_reorder_b200.datagen import make_qkv, random_scores
+from oracle import attention, e4m3, select, tiling
+from tests.helpers import (SMALL, assert_topp_equal, lists_from_device, lists_to_device, to64)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def bs():
+    from block_sparse_attention_reorder_b200 import bsattn
+    assert torch.cuda.is_available()
+    return bsattn
+
+
+def _plan(bs, wl, **over):
+    args = dict(rule=wl.rule, k=wl.k, p=wl.p, win=wl.win, tile=wl.tile, qk_fp8=wl.qk_fp8)
+    args.update(over)
+    return bs.Plan(wl.B, wl.heads, wl.head_dim, wl.T, wl.H, wl.W, **args)
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_reorder_pool_unreorder(bs, name):
+    wl = SMALL[name]
+    plan = _plan(bs, wl)
+    q, _, _ = make_qkv(wl, "cuda")
+    xt = torch.empty(plan.tiled_shape(), dtype=torch.bfloat16, device="cuda")
+    pooled = torch.empty((wl.B, wl.heads, plan.N, wl.head_dim), dtype=torch.float32, device="cuda")
+    bs.attn_reorder(plan, q, xt, pooled)
+    qn = to64(q)
+    np.testing.assert_array_equal(to64(xt), tiling.reorder(qn, wl.T, wl.H, wl.W, wl.tile))
+    ref = tiling.pool_mean(qn, wl.T, wl.H, wl.W, wl.tile)
+    np.testing.assert_allclose(to64(pooled), ref, rtol=1e-5, atol=2e-6)
+    pooled2 = torch.zeros_like(pooled)
+    bs.attn_pool(plan, q, pooled2)
+    torch.testing.assert_close(pooled2, pooled, rtol=0, atol=0)
+    back = torch.empty_like(q)
+    bs.attn_unreorder(plan, xt, back)
+    assert torch.equal(back, q)
+    assert bs.attn_check_device_status(plan) == 0
+
+
+@pytest.mark.parametrize("name", ["ragged_topk", "tiny_d64"])
+def test_block_scores(bs, name):
+    wl = SMALL[name]
+    plan = _plan(bs, wl)
+    q, k, _ = make_qkv(wl, "cuda")
+    pq = tiling.pool_mean(to64(q), wl.T, wl.H, wl.W).astype(np.float32)
+    pk = tiling.pool_mean(to64(k), wl.T, wl.H, wl.W).astype(np.float32)
+    S = torch.empty((wl.B, wl.heads, plan.N, plan.N), dtype=torch.float32, device="cuda")
+    bs.attn_block_scores(plan, torch.from_numpy(pq).cuda(), torch.from_numpy(pk).cuda(), S)
+    scale = 1 / math.sqrt(wl.head_dim)
+    ref = select.block_scores(pq, pk, scale)
+    bound = 1e-5 * scale * np.matmul(np.abs(pq).astype(np.float64),
+                                     np.swapaxes(np.abs(pk).astype(np.float64), -1, -2)) + 1e-30
+    assert np.all(np.abs(to64(S) - ref) <= bound)
+
+
+@pytest.mark.parametrize("N,k", [(32, 8), (364, 46), (1440, 144), (37, 37), (2048, 1),
+                                 (100, 99), (5, 2), (1000, 500)])
+def test_select_topk_bit_exact(bs, N, k):
+    rows = 2 * 3 * N if N <= 400 else 2 * N
+    S = random_scores(rows, N, seed=N * 7 + k)
+    # A plan whose N matches: grid of N tiles along w (4 x 4 x 4N)
+    plan = bs.Plan(1, rows // N, 64, 4, 4, 4 * N, rule="topk", k=k)
+    assert plan.N == N
+    idx = torch.empty((1, rows // N, N, k), dtype=torch.int32, device="cuda")
+    cnt = torch.empty((1, rows // N, N), dtype=torch.int32, device="cuda")
+    bs.attn_select_from_scores(plan, S.view(1, rows // N, N, N).cuda(), idx, cnt)
+    got = lists_from_device(idx, cnt)
+    Sn = S.numpy()
+    for r in range(rows):
+        np.testing.assert_array_equal(got[r], select.topk_row(Sn[r], k))
+
+
+@pytest.mark.parametrize("N,k,p", [(32, 8, 0.9), (364, 16, 0.9), (1440, 16, 0.9), (50, 0, 0.5),
+                                   (700, 3, 0.99), (2048, 16, 0.9), (17, 17, 0.3), (9, 1, 1.0)])
+@pytest.mark.parametrize("sharp", [1.0, 8.0])
+def test_select_topp_bit_exact(bs, N, k, p, sharp):
+    rows = 2 * N if N <= 400 else N
+    S = random_scores(rows, N, seed=N * 13 + k) * sharp
+    plan = bs.Plan(1, rows // N, 64, 4, 4, 4 * N, rule="topp", k=k, p=p)
+    idx = torch.empty((1, rows // N, N, N), dtype=torch.int32, device="cuda")
+    cnt = torch.empty((1, rows // N, N), dtype=torch.int32, device="cuda")
+    bs.attn_select_from_scores(plan, S.view(1, rows // N, N, N).cuda(), idx, cnt)
+    got = lists_from_device(idx, cnt)
+    Sn = S.numpy()
+    for r in range(rows):
+        assert_topp_equal(got[r], Sn[r], p, k)
+
+
+@pytest.mark.parametrize("name", ["ragged_window_fp8", "ragged_bf16_window"])
+def test_window_lists(bs, name):
+    wl = SMALL[name]
+    plan = _plan(bs, wl)
+    si, sc = plan.list_shapes()
+    idx = torch.empty(si, dtype=torch.int32, device="cuda")
+    cnt = torch.empty(sc, dtype=torch.int32, device="cuda")
+    bs.attn_select_from_scores(plan, None, idx, cnt)
+    got = lists_from_device(idx, cnt)
+    grid = tiling.tile_grid(wl.T, wl.H, wl.W)
+    for r, l in enumerate(got):
+        np.testing.assert_array_equal(l, select.window_row(r % plan.N, grid, wl.win))
+
+
+@pytest.mark.parametrize("name", ["ragged_window_fp8", "ragged_d64_fp8", "tiny_d64"])
+def test_quantize_e4m3_bytes(bs, name):
+    wl = SMALL[name]
+    plan = _plan(bs, wl)
+    q, _, _ = make_qkv(wl, "cuda")
+    q = q * 37.0  # exercise larger magnitudes too
+    q = q.to(torch.bfloat16)
+    xt = torch.empty(plan.tiled_shape(), dtype=torch.bfloat16, device="cuda")
+    bs.attn_reorder(plan, q, xt)
+    codes = torch.empty(plan.tiled_shape(), dtype=torch.uint8, device="cuda")
+    scales = torch.empty((wl.B, wl.heads, plan.N), dtype=torch.float32, device="cuda")
+    bs.attn_quantize_e4m3(plan, xt, codes, scales)
+    rc, rs = e4m3.quantize_tiled(tiling.reorder(to64(q).astype(np.float32), wl.T, wl.H, wl.W))
+    np.testing.assert_array_equal(scales.cpu().numpy(), rs)
+    np.testing.assert_array_equal(codes.cpu().numpy(), rc)
+
+
+def _oracle_inputs(wl):
+    q, k, v = make_qkv(wl, "cpu")
+    return q, k, v, to64(q), to64(k), to64(v)
+
+
+@pytest.mark.parametrize("name", ["tiny_d64", "ragged_topk", "ragged_topp", "ragged_bf16_window"])
+def test_forward_bf16_against_oracle(bs, name):
+    wl = SMALL[name]
+    plan = _plan(bs, wl, qk_fp8=False)
+    q, k, v, qn, kn, vn = _oracle_inputs(wl)
+    _, _, _, lists = attention.route(qn, kn, wl.T, wl.H, wl.W, wl.rule, k=wl.k, p=wl.p,
+                                     half=wl.win, score_dtype=np.float32)
+    idx, cnt = lists_to_device(lists, plan.kmax)
+    tiled = []
+    for x in (q, k, v):
+        t = torch.empty(plan.tiled_shape(), dtype=torch.bfloat16, device="cuda")
+        bs.attn_reorder(plan, x.cuda(), t)
+        tiled.append(t)
+    o = torch.empty(plan.tiled_shape(), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((wl.B, wl.heads, plan.N, 64), dtype=torch.float32, device="cuda")
+    si, sc = plan.list_shapes()
+    bs.attn_forward(plan, tiled[0], tiled[1], tiled[2], idx.view(si), cnt.view(sc), o, lse)
+    assert bs.attn_check_device_status(plan) == 0
+    o_ref, lse_ref = attention.attention_full(qn, kn, vn, lists, wl.T, wl.H, wl.W)
+    o_nat = tiling.unreorder(to64(o), wl.T, wl.H, wl.W)
+    err = np.abs(o_nat - o_ref)
+    assert err.max() <= 2e-2 and err.mean() <= 2e-3, (err.max(), err.mean())
+    lse_nat = np.stack([tiling.unreorder(to64(lse)[:, h:h + 1, :, :, None], wl.T, wl.H, wl.W)[..., 0, 0]
+                        for h in range(wl.heads)], axis=1)
+    np.testing.assert_allclose(lse_nat, lse_ref, rtol=0, atol=2e-2)
+
+
+@pytest.mark.parametrize("name", ["ragged_window_fp8", "ragged_d64_fp8"])
+def test_forward_fp8_against_oracle(bs, name):
+    wl = SMALL[name]
+    plan = _plan(bs, wl)
+    q, k, v, qn, kn, vn = _oracle_inputs(wl)
+    qd, kd, (qc, qs), (kc, ks) = attention.fp8_qk(qn, kn, wl.T, wl.H, wl.W)
+    _, _, _, lists = attention.route(qn, kn, wl.T, wl.H, wl.W, wl.rule, k=wl.k, p=wl.p,
+                                     half=wl.win, score_dtype=np.float32)
+    idx, cnt = lists_to_device(lists, plan.kmax)
+    vt = torch.empty(plan.tiled_shape(), dtype=torch.bfloat16, device="cuda")
+    bs.attn_reorder(plan, v.cuda(), vt)
+    o = torch.empty(plan.tiled_shape(), dtype=torch.bfloat16, device="cuda")
+    si, sc = plan.list_shapes()
+    bs.attn_forward(plan, torch.from_numpy(qc).cuda(), torch.from_numpy(kc).cuda(), vt,
+                    idx.view(si), cnt.view(sc), o, q_scale=torch.from_numpy(qs).cuda(),
+                    k_scale=torch.from_numpy(ks).cuda())
+    assert bs.attn_check_device_status(plan) == 0
+    o_ref, _ = attention.attention_full(qd, kd, vn, lists, wl.T, wl.H, wl.W)
+    o_nat = tiling.unreorder(to64(o), wl.T, wl.H, wl.W)
+    rel = np.linalg.norm(o_nat - o_ref) / np.linalg.norm(o_ref)
+    assert rel <= 1e-2, rel
+
+
+def test_bad_list_entry_sets_error_word_and_is_skipped(bs):
+    wl = SMALL["ragged_topk"]
+    plan = _plan(bs, wl)
+    q, k, v = make_qkv(wl, "cuda")
+    tiled = []
+    for x in (q, k, v):
+        t = torch.empty(plan.tiled_shape(), dtype=torch.bfloat16, device="cuda")
+        bs.attn_reorder(plan, x, t)
+        tiled.append(t)
+    si, sc = plan.list_shapes()
+    idx = torch.zeros(si, dtype=torch.int32, device="cuda")
+    idx[..., 1] = plan.N + 3          # out of range: must be skipped, not read
+    idx[0, 0, 0, 2] = -7
+    cnt = torch.full(sc, 3, dtype=torch.int32, device="cuda")
+    o = torch.empty(plan.tiled_shape(), dtype=torch.bfloat16, device="cuda")
+    bs.attn_forward(plan, *tiled, idx, cnt, o)
+    assert bs.attn_check_device_status(plan) == bs.BsattnError(5, "").code
+    assert bs.attn_check_device_status(plan) == 0  # cleared
+    # result equals attending tile 0 only (listed twice counts as two passes of the same keys)
+    idx2 = torch.zeros(si, dtype=torch.int32, device="cuda")
+    cnt2 = torch.ones(sc, dtype=torch.int32, device="cuda")
+    o2 = torch.empty_like(o)
+    bs.attn_forward(plan, *tiled, idx2, cnt2, o2)
+    rows = (idx[..., 2] == 0)
+    torch.testing.assert_close(o[rows], o2[rows], rtol=2e-2, atol=2e-2)
+    cnt_bad = torch.full(sc, plan.kmax + 1, dtype=torch.int32, device="cuda")
+    bs.attn_forward(plan, *tiled, idx2, cnt_bad, o2)
+    assert bs.attn_check_device_status(plan) == 5
