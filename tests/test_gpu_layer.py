@@ -102,8 +102,8 @@ def test_attn_select_equals_component_chain(bs, name):
     bs.attn_block_scores(plan, pq, pk, S)
     idx2, cnt2 = torch.empty_like(idx), torch.empty_like(cnt)
     bs.attn_select_from_scores(plan, S, idx2, cnt2)
-    assert lists_from_device(idx, cnt) == lists_from_device(idx2, cnt2) or all(
-        np.array_equal(a, b) for a, b in zip(lists_from_device(idx, cnt), lists_from_device(idx2, cnt2)))
+    a_l, b_l = lists_from_device(idx, cnt), lists_from_device(idx2, cnt2)
+    assert len(a_l) == len(b_l) and all(np.array_equal(a, b) for a, b in zip(a_l, b_l))
 
 
 def _sample_rows(wl, N, n_heads=3, n_tiles=6, seed=0):
