@@ -72,7 +72,7 @@ def test_layer_small(bs, name):
             assert wl.rule != "window"
             assert_valid_selection(g, Sf[r], wl.rule, k=wl.k, p=wl.p)
     assert np.mean(same) >= 0.9
-    o_ref, lse_ref = attention.attention_full(qa, ka, vn, got if all(same) else lists,
+    o_ref, lse_ref = attention.attention_full(qa, ka, vn, lists,
                                               wl.T, wl.H, wl.W)
     if all(same):
         _check_outputs(wl, to64(o), o_ref, to64(lse), lse_ref)
