@@ -1,0 +1,522 @@
+// Block-sparse attention forward over kept tile pairs on the 5th-generation
+// tensor cores (tcgen05, TMEM accumulators, TMA-fed shared memory).
+//
+// Work unit: two adjacent query tiles i0 = 2p, i1 = 2p + 1 of one (batch,
+// head), stacked into one 128-row query block so that every QK^T and PV
+// product is an M = 128 tcgen05.mma. The block walks the union of the two
+// tiles' kept key-tile lists in ascending order; a key tile kept by only one
+// of the two query tiles gives zero probabilities to the other tile's rows.
+// Adjacent query tiles of a smooth video latent keep mostly the same key
+// tiles, so little work is wasted.
+//
+// Roles (192 threads):
+//   warps 0-3  softmax: thread r owns query row r (TMEM lane r). Per key
+//              tile: read S from TMEM, scale (and e4m3 tile scales), mask
+//              padded keys, online softmax in fp32 with lazy rescaling
+//              (the running max is only moved when it grows by more than
+//              2^8, which keeps O and l exact up to rounding), write P as
+//              bf16 into the TMEM columns S came from.
+//   warp 4     TMA producer: Q block once, then K_j / V_j per step into a
+//              two-stage ring.
+//   warp 5     MMA issuer (one thread): S_{n+2} = Q K^T is issued right
+//              after PV_n so it overlaps softmax n+1; O += P_n V_n reads P
+//              from TMEM (A operand) and V from shared memory (MN-major B).
+// TMEM: columns [0,64) and [64,128) hold S/P double buffers, [128,128+D) O.
+// Every mbarrier wait is bounded: on expiry the CTA sets the device error
+// word, raises a CTA-wide abort flag, lets in-flight TMA copies land and
+// frees its TMEM before returning.
+#include <cudaTypedefs.h>
+#include <math.h>
+
+
+#include "internal.h"
+#include "tc_common.cuh"
+
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int kStages = 2;
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kColS0 = 0, kColS1 = 64, kColO = 128;
+constexpr long long kWaitLimit = 4000000000LL;  // SM cycles (~2 s)
+constexpr float kRescaleThreshold = 8.0f;        // log2 units
+
+struct TcParams {
+  Geom g;
+  const float* qs;
+  const float* ks;
+  const int32_t* idx;
+  const int32_t* cnt;
+  int kmax;
+  __nv_bfloat16* o;
+  float* lse;
+  float scale_log2;
+  int* err;
+  int umax;      // union list capacity (entries)
+  int bm_words;  // bitmap words per list
+};
+
+template <int D, bool FP8>
+struct Cfg {
+  static constexpr int ESZ = FP8 ? 1 : 2;
+  static constexpr int QRB = D * ESZ;                 // Q/K row bytes
+  static constexpr int SWB = QRB >= 128 ? 128 : 64;   // swizzle span
+  static constexpr uint32_t LAYOUT = SWB == 128 ? tc::kLayoutSW128 : tc::kLayoutSW64;
+  static constexpr int QBLK = QRB / SWB;              // column blocks of Q/K
+  static constexpr int NKS = QRB / 32;                // S MMAs (32 bytes of K each)
+  static constexpr int KS_PER_BLK = SWB / 32;
+  static constexpr int Q_BYTES = 128 * QRB;
+  static constexpr int K_BYTES = 64 * QRB;
+  static constexpr int V_BYTES = 64 * D * 2;
+  static constexpr int VBLK = D / 64;                 // 64-column blocks of V
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + Q_BYTES;
+  static constexpr int OFF_V = OFF_K + kStages * K_BYTES;
+  static constexpr int OFF_BAR = OFF_V + kStages * V_BYTES;
+  // barriers: q, full[2], empty[2], sfull[2], pfull[2], pvdone[2], final
+  static constexpr int NBAR = 1 + 2 * kStages + 7;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base, abort, L, pad
+  static constexpr int OFF_COL = OFF_MISC + 16;         // 64 packed column coords
+  static constexpr int OFF_SCAN = OFF_COL + 256;        // block-scan scratch
+  static constexpr int OFF_DYN = OFF_SCAN + 64;         // bitmaps, union list
+  static constexpr int O_PITCH = D * 2 + 16;            // epilogue staging row pitch
+  static_assert(OFF_Q % 1024 == 0 && OFF_K % 1024 == 0 && OFF_V % 1024 == 0, "alignment");
+  static_assert(128 * O_PITCH <= OFF_BAR - OFF_K, "epilogue staging fits in the ring");
+};
+
+__device__ __forceinline__ void record_timeout(volatile int* abort_flag, int* err) {
+  *abort_flag = 1;
+  atomicOr(err, BSATTN_DEVERR_TIMEOUT);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi, float& sum) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  float2 f = __bfloat1622float2(h);
+  sum += f.x + f.y;
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+template <int D, bool FP8>
+__global__ void __launch_bounds__(kThreads, 2)
+attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+               const __grid_constant__ CUtensorMap tmV, TcParams P) {
+  using C = Cfg<D, FP8>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t sb = tc::smem_addr(smem);
+  const uint32_t bar_q = sb + C::OFF_BAR;
+  auto bar_full = [&](int s) { return sb + C::OFF_BAR + 8u * (1 + s); };
+  auto bar_empty = [&](int s) { return sb + C::OFF_BAR + 8u * (1 + kStages + s); };
+  auto bar_sfull = [&](int b) { return sb + C::OFF_BAR + 8u * (1 + 2 * kStages + b); };
+  auto bar_pfull = [&](int b) { return sb + C::OFF_BAR + 8u * (3 + 2 * kStages + b); };
+  auto bar_pvdone = [&](int b) { return sb + C::OFF_BAR + 8u * (5 + 2 * kStages + b); };
+  const uint32_t bar_final = sb + C::OFF_BAR + 8u * (7 + 2 * kStages);
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
+  volatile int* never = reinterpret_cast<volatile int*>(misc + 3);  // stays 0: waits that ignore abort
+  uint32_t* colc = reinterpret_cast<uint32_t*>(smem + C::OFF_COL);
+  int* scan = reinterpret_cast<int*>(smem + C::OFF_SCAN);
+  uint32_t* bmA = reinterpret_cast<uint32_t*>(smem + C::OFF_DYN);
+  uint32_t* bmB = bmA + P.bm_words;
+  uint32_t* ulist = bmB + P.bm_words;
+
+  const Geom& g = P.g;
+  const int i0 = 2 * blockIdx.x, i1 = i0 + 1;
+  const int head = blockIdx.y, b = blockIdx.z;
+  const size_t bh = (size_t)b * g.Hh + head;
+  const bool has1 = i1 < g.N;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  // ------------------------------------------------------------ setup
+  if (tid == 0) {
+    tc::mbar_init(bar_q, 1);
+    for (int s = 0; s < kStages; ++s) {
+      tc::mbar_init(bar_full(s), 1);
+      tc::mbar_init(bar_empty(s), 1);
+    }
+    for (int x = 0; x < 2; ++x) {
+      tc::mbar_init(bar_sfull(x), 1);
+      tc::mbar_init(bar_pfull(x), 128);
+      tc::mbar_init(bar_pvdone(x), 1);
+    }
+    tc::mbar_init(bar_final, 1);
+    misc[1] = 0;
+    misc[3] = 0;
+    tc::mbar_fence_init();
+  }
+  if (warp == 5) {
+    tc::tmem_alloc(sb + C::OFF_MISC, kTmemCols);
+    tc::tmem_relinquish();
+  }
+  if (tid < 64) {
+    int dt = tid / (g.th * g.tw), dh = (tid / g.tw) % g.th, dw = tid % g.tw;
+    colc[tid] = (uint32_t)dt | ((uint32_t)dh << 8) | ((uint32_t)dw << 16);
+  }
+  for (int w = tid; w < 2 * P.bm_words; w += kThreads) bmA[w] = 0u;
+  __syncthreads();
+
+  // Union of the two kept lists as a bitmap pair, then compacted ascending.
+  int nA = P.cnt[bh * g.N + i0];
+  int nB = has1 ? P.cnt[bh * g.N + i1] : 0;
+  if (nA < 0 || nA > P.kmax || nB < 0 || nB > P.kmax) {
+    if (tid == 0) atomicOr(P.err, BSATTN_DEVERR_BAD_INDEX);
+    nA = min(max(nA, 0), P.kmax);
+    nB = min(max(nB, 0), P.kmax);
+  }
+  {
+    const int32_t* lA = P.idx + (bh * g.N + i0) * (size_t)P.kmax;
+    const int32_t* lB = lA + P.kmax;
+    for (int e = tid; e < nA + nB; e += kThreads) {
+      int j = e < nA ? __ldg(lA + e) : __ldg(lB + (e - nA));
+      if (j < 0 || j >= g.N) {
+        atomicOr(P.err, BSATTN_DEVERR_BAD_INDEX);
+        continue;
+      }
+      atomicOr(e < nA ? &bmA[j >> 5] : &bmB[j >> 5], 1u << (j & 31));
+    }
+  }
+  __syncthreads();
+  {
+    const int wpt = (P.bm_words + kThreads - 1) / kThreads;
+    const int w0 = min(tid * wpt, P.bm_words), w1 = min(w0 + wpt, P.bm_words);
+    int mine = 0;
+    for (int w = w0; w < w1; ++w) mine += __popc(bmA[w] | bmB[w]);
+    int x = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) scan[warp] = x;
+    __syncthreads();
+    int off = 0, tot = 0;
+#pragma unroll
+    for (int i = 0; i < kThreads / 32; ++i) {
+      off += i < warp ? scan[i] : 0;
+      tot += scan[i];
+    }
+    int pos = off + x - mine;
+    for (int w = w0; w < w1; ++w) {
+      uint32_t a = bmA[w], bb = bmB[w], bits = a | bb;
+      while (bits) {
+        int bit = __ffs(bits) - 1;
+        bits &= bits - 1;
+        uint32_t e = (uint32_t)(w * 32 + bit) | (((a >> bit) & 1u) << 30) | (((bb >> bit) & 1u) << 31);
+        if (pos < P.umax) ulist[pos] = e;
+        ++pos;
+      }
+    }
+    if (tid == 0) misc[2] = (uint32_t)min(tot, P.umax);
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = misc[0];
+  const int L = (int)misc[2];
+
+  // ------------------------------------------------------------ roles
+  if (warp == 4) {
+    if (lane == 0 && L > 0) {
+      tc::tma_prefetch_desc(&tmQ);
+      tc::tma_prefetch_desc(&tmK);
+      tc::tma_prefetch_desc(&tmV);
+      const int qrow = (int)((bh * g.N + i0) * 64);
+      tc::mbar_arrive_expect_tx(bar_q, C::Q_BYTES);
+#pragma unroll
+      for (int cb = 0; cb < C::QBLK; ++cb)
+        tc::tma_load_2d(sb + C::OFF_Q + cb * 128 * C::SWB, &tmQ, bar_q, cb * C::SWB / C::ESZ, qrow);
+      int last[kStages];
+#pragma unroll
+      for (int s = 0; s < kStages; ++s) last[s] = -1;
+      for (int n = 0; n < L; ++n) {
+        const int s = n % kStages;
+        if (n >= kStages && !tc::mbar_wait(bar_empty(s), ((n / kStages) - 1) & 1, abort_flag, kWaitLimit)) {
+          record_timeout(abort_flag, P.err);
+          break;
+        }
+        const int j = (int)(ulist[n] & 0x3FFFFFFFu);
+        const int krow = (int)((bh * g.N + j) * 64);
+        tc::mbar_arrive_expect_tx(bar_full(s), C::K_BYTES + C::V_BYTES);
+#pragma unroll
+        for (int cb = 0; cb < C::QBLK; ++cb)
+          tc::tma_load_2d(sb + C::OFF_K + s * C::K_BYTES + cb * 64 * C::SWB, &tmK, bar_full(s),
+                          cb * C::SWB / C::ESZ, krow);
+#pragma unroll
+        for (int vb = 0; vb < C::VBLK; ++vb)
+          tc::tma_load_2d(sb + C::OFF_V + s * C::V_BYTES + vb * 8192, &tmV, bar_full(s), vb * 64, krow);
+        last[s] = n;
+      }
+      if (*abort_flag) {
+        // Let copies already issued land before the CTA's memory goes away.
+        tc::mbar_wait(bar_q, 0, never, kWaitLimit);
+        for (int s = 0; s < kStages; ++s)
+          if (last[s] >= 0) tc::mbar_wait(bar_full(s), (last[s] / kStages) & 1, never, kWaitLimit);
+      }
+    }
+  } else if (warp == 5) {
+    if (lane == 0 && L > 0) {
+      constexpr uint32_t idS = FP8 ? tc::instr_desc(0, 0, 0, 0, 64, 128)
+                                   : tc::instr_desc(1, 1, 0, 0, 64, 128);
+      constexpr uint32_t idPV = tc::instr_desc(1, 1, 0, 1, D, 128);
+      bool ok = tc::mbar_wait(bar_q, 0, abort_flag, kWaitLimit);
+      auto issue_S = [&](int m) -> bool {
+        const int s = m % kStages;
+        if (!tc::mbar_wait(bar_full(s), (m / kStages) & 1, abort_flag, kWaitLimit)) return false;
+        tc::fence_after_sync();
+        const uint32_t dS = tmem + ((m & 1) ? kColS1 : kColS0);
+#pragma unroll
+        for (int kk = 0; kk < C::NKS; ++kk) {
+          const int cb = kk / C::KS_PER_BLK, within = kk % C::KS_PER_BLK;
+          const uint64_t da = tc::smem_desc(sb + C::OFF_Q + cb * 128 * C::SWB + within * 32, 16,
+                                            8 * C::SWB, C::LAYOUT);
+          const uint64_t db = tc::smem_desc(sb + C::OFF_K + s * C::K_BYTES + cb * 64 * C::SWB + within * 32,
+                                            16, 8 * C::SWB, C::LAYOUT);
+          if (FP8)
+            tc::mma_ss_f8(dS, da, db, idS, kk > 0 ? 1u : 0u);
+          else
+            tc::mma_ss_f16(dS, da, db, idS, kk > 0 ? 1u : 0u);
+        }
+        tc::mma_commit(bar_sfull(m & 1));
+        return true;
+      };
+      if (ok) ok = issue_S(0);
+      if (ok && L > 1) ok = issue_S(1);
+      for (int n = 0; ok && n < L; ++n) {
+        const int s = n % kStages;
+        if (!tc::mbar_wait(bar_pfull(n & 1), (n >> 1) & 1, abort_flag, kWaitLimit)) {
+          ok = false;
+          break;
+        }
+        tc::fence_after_sync();
+        const uint32_t pA = tmem + ((n & 1) ? kColS1 : kColS0);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t dv = tc::smem_desc(sb + C::OFF_V + s * C::V_BYTES + kk * 2048, 8192, 1024,
+                                            tc::kLayoutSW128);
+          tc::mma_ts_f16(tmem + kColO, pA + kk * 8, dv, idPV, (n > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc::mma_commit(bar_pvdone(n & 1));
+        tc::mma_commit(bar_empty(s));
+        if (n + 2 < L && !issue_S(n + 2)) {
+          ok = false;
+          break;
+        }
+      }
+      if (!ok) record_timeout(abort_flag, P.err);
+      // Every MMA issued so far has finished before TMEM is released.
+      tc::mma_commit(bar_final);
+      tc::mbar_wait(bar_final, 0, never, kWaitLimit);
+    }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------- softmax
+    const int r = tid;              // query row of the 128-row block
+    const int half = r >> 6;        // 0: tile i0, 1: tile i1
+    const bool row_exists = half == 0 || has1;
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const float qsc = (FP8 && row_exists) ? P.qs[bh * g.N + (half ? i1 : i0)] : 1.f;
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int n = 0; n < L; ++n) {
+      const uint32_t e = ulist[n];
+      const int j = (int)(e & 0x3FFFFFFFu);
+      const bool keep = ((e >> (30 + half)) & 1u) != 0;  // uniform within the warp
+      if (!__all_sync(0xffffffffu, tc::mbar_wait(bar_sfull(n & 1), (n >> 1) & 1, abort_flag, kWaitLimit))) {
+        ok = false;
+        break;
+      }
+      tc::fence_after_sync();
+      const uint32_t sbuf = tmem + lane_base + ((n & 1) ? kColS1 : kColS0);
+      uint32_t pk[32];
+      bool need = false;
+      float alpha = 1.f;
+      if (keep) {
+        uint32_t sr[64];
+        tc::tmem_ld64_wait(sbuf, sr);
+        const float c = P.scale_log2 * (FP8 ? qsc * __ldg(P.ks + bh * g.N + j) : 1.f);
+        const int bt = j / (g.nH * g.nW), bhh = (j / g.nW) % g.nH, bw = j % g.nW;
+        const int vt = g.T - bt * g.tt, vh = g.H - bhh * g.th, vw = g.W - bw * g.tw;
+        const bool partial = vt < g.tt || vh < g.th || vw < g.tw;
+        float mx = -INFINITY;
+#pragma unroll
+        for (int q = 0; q < 64; ++q) {
+          float x = __uint_as_float(sr[q]) * c;
+          if (partial) {
+            const uint32_t cc = colc[q];
+            if ((int)(cc & 0xffu) >= vt || (int)((cc >> 8) & 0xffu) >= vh || (int)((cc >> 16) & 0xffu) >= vw)
+              x = -INFINITY;
+          }
+          sr[q] = __float_as_uint(x);
+          mx = fmaxf(mx, x);
+        }
+        const float m_new = fmaxf(m, mx);
+        if (m == -INFINITY) {
+          m = m_new;  // first kept tile of this row: O row is still zero
+        } else if (m_new - m > kRescaleThreshold) {
+          alpha = exp2f(m - m_new);
+          m = m_new;
+          l *= alpha;
+          need = true;
+        }
+        float ls = 0.f;
+#pragma unroll
+        for (int q = 0; q < 32; ++q)
+          pk[q] = pack_bf16x2(exp2f(__uint_as_float(sr[2 * q]) - m),
+                              exp2f(__uint_as_float(sr[2 * q + 1]) - m), ls);
+        l += ls;
+      } else {
+#pragma unroll
+        for (int q = 0; q < 32; ++q) pk[q] = 0u;
+      }
+      tc::tmem_st32(sbuf, pk);  // P_n over the first 32 columns of S_n
+      if (__any_sync(0xffffffffu, need)) {
+        // O holds PV_0..PV_{n-1} once PV_{n-1} has completed.
+        if (!__all_sync(0xffffffffu,
+                        tc::mbar_wait(bar_pvdone((n - 1) & 1), ((n - 1) >> 1) & 1, abort_flag, kWaitLimit))) {
+          ok = false;
+          break;
+        }
+        tc::fence_after_sync();
+#pragma unroll
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t o[32];
+          tc::tmem_ld32_wait(tmem + lane_base + kColO + c0, o);
+#pragma unroll
+          for (int q = 0; q < 32; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * alpha);
+          tc::tmem_st32(tmem + lane_base + kColO + c0, o);
+        }
+      }
+      tc::tmem_wait_st();
+      tc::fence_before_sync();
+      tc::mbar_arrive(bar_pfull(n & 1));
+    }
+    if (!ok) record_timeout(abort_flag, P.err);
+    // ---------------------------------------------------------- epilogue
+    if (ok && L > 0) {
+      if (!__all_sync(0xffffffffu,
+                      tc::mbar_wait(bar_pvdone((L - 1) & 1), ((L - 1) >> 1) & 1, abort_flag, kWaitLimit))) {
+        record_timeout(abort_flag, P.err);
+        ok = false;
+      }
+      tc::fence_after_sync();
+    }
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    uint8_t* stage = smem + C::OFF_K + r * C::O_PITCH;
+#pragma unroll
+    for (int c0 = 0; c0 < D; c0 += 32) {
+      uint32_t o[32];
+      if (ok && L > 0) {
+        tc::tmem_ld32_wait(tmem + lane_base + kColO + c0, o);
+      } else {
+#pragma unroll
+        for (int q = 0; q < 32; ++q) o[q] = 0u;
+      }
+      uint32_t w[16];
+      float dummy = 0.f;
+#pragma unroll
+      for (int q = 0; q < 16; ++q)
+        w[q] = pack_bf16x2(__uint_as_float(o[2 * q]) * inv, __uint_as_float(o[2 * q + 1]) * inv, dummy);
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        reinterpret_cast<uint4*>(stage + c0 * 2)[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+    }
+    if (P.lse && row_exists)
+      P.lse[(bh * g.N + i0) * 64 + r] = l > 0.f ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    constexpr int CPR = D / 8;  // 16-byte chunks per row
+    const int rows = has1 ? 128 : 64;
+    uint4* og = reinterpret_cast<uint4*>(P.o + (bh * g.N + i0) * 64 * (size_t)D);
+    for (int e2 = r; e2 < rows * CPR; e2 += 128) {
+      const int rr = e2 / CPR, cc = e2 % CPR;
+      og[e2] = *reinterpret_cast<const uint4*>(smem + C::OFF_K + rr * C::O_PITCH + cc * 16);
+    }
+  }
+
+  // ------------------------------------------------------------ teardown
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 5) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return (PFN_cuTensorMapEncodeTiled_v12000) nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }();
+  return fn;
+}
+
+bool make_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int esz, int inner,
+              uint64_t rows, int box_inner, int box_rows, CUtensorMapSwizzle sw) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)inner * esz};
+  cuuint32_t box[2] = {(cuuint32_t)box_inner, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int D, bool FP8>
+bsattn_status run(const bsattn_plan* p, const void* q, const void* k, const __nv_bfloat16* v,
+                  TcParams prm, cudaStream_t st) {
+  using C = Cfg<D, FP8>;
+  const uint64_t rows = (uint64_t)p->desc.B * p->desc.heads * p->N * 64;
+  if (rows + 128 >= (1ull << 31)) return BSATTN_ERR_UNSUPPORTED;
+  CUtensorMap mq, mk, mv;
+  const CUtensorMapDataType dqk = FP8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const CUtensorMapSwizzle sw = C::SWB == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  if (!make_map(&mq, q, dqk, C::ESZ, D, rows, C::SWB / C::ESZ, 128, sw) ||
+      !make_map(&mk, k, dqk, C::ESZ, D, rows, C::SWB / C::ESZ, 64, sw) ||
+      !make_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, rows, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+    return BSATTN_ERR_CUDA;
+  size_t smem = 1024 + C::OFF_DYN + (size_t)prm.bm_words * 8 + (size_t)prm.umax * 4;
+  if (smem < 80 * 1024) smem = 80 * 1024;  // at most two CTAs (2 x 256 TMEM columns) per SM
+  if (smem > 227 * 1024) return BSATTN_ERR_UNSUPPORTED;
+  auto kern = attn_tc_kernel<D, FP8>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return BSATTN_ERR_CUDA;
+  dim3 grid((p->N + 1) / 2, p->desc.heads, p->desc.B);
+  kern<<<grid, kThreads, smem, st>>>(mq, mk, mv, prm);
+  return cudaGetLastError() == cudaSuccess ? BSATTN_OK : BSATTN_ERR_CUDA;
+}
+
+}  // namespace
+
+size_t attention_workspace_bytes(const bsattn_plan*) { return 0; }
+
+bsattn_status launch_attention(const bsattn_plan* p, const void* q, const void* k, const float* qs,
+                               const float* ks, const __nv_bfloat16* v, const int32_t* idx,
+                               const int32_t* cnt, __nv_bfloat16* o, float* lse, void*, size_t,
+                               cudaStream_t st) {
+  if (p->N > 32768) return BSATTN_ERR_UNSUPPORTED;
+  TcParams prm;
+  prm.g = make_geom(p);
+  prm.qs = qs;
+  prm.ks = ks;
+  prm.idx = idx;
+  prm.cnt = cnt;
+  prm.kmax = p->kmax;
+  prm.o = o;
+  prm.lse = lse;
+  prm.scale_log2 = p->scale * 1.4426950408889634f;
+  prm.err = p->d_err;
+  prm.umax = p->N < 2 * p->kmax ? p->N : 2 * p->kmax;
+  prm.bm_words = (p->N + 31) / 32;
+  const bool fp8 = p->desc.qk_fp8 != 0;
+  if (p->desc.head_dim == 128)
+    return fp8 ? run<128, true>(p, q, k, v, prm, st) : run<128, false>(p, q, k, v, prm, st);
+  return fp8 ? run<64, true>(p, q, k, v, prm, st) : run<64, false>(p, q, k, v, prm, st);
+}
