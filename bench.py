@@ -70,6 +70,24 @@ def pair_flops(head_dim: int) -> float:
     return 4.0 * 64 * 64 * head_dim
 
 
+def issued_pairs(idx: torch.Tensor, cnt: torch.Tensor, N: int) -> int:
+    """Tile pairs the attention kernel multiplies: it stacks query tiles
+    2p and 2p+1 into one 128-row block over the union of their lists, so
+    each union entry costs two tile pairs of MMA work."""
+    rows = cnt.numel()
+    kmax = idx.shape[-1]
+    ii = idx.reshape(rows, kmax).to(torch.int64)
+    valid = torch.arange(kmax, device=idx.device)[None, :] < cnt.reshape(rows, 1)
+    hit = torch.zeros((rows, N), dtype=torch.bool, device=idx.device)
+    r = torch.arange(rows, device=idx.device)[:, None].expand(rows, kmax)
+    hit[r[valid], ii[valid]] = True
+    hit = hit.reshape(-1, N, N)  # [B*heads, query tile, key tile]
+    if N % 2:
+        hit = torch.cat([hit, torch.zeros_like(hit[:, :1])], dim=1)
+    union = hit[:, 0::2] | hit[:, 1::2]
+    return int(union.sum().item()) * 2
+
+
 def launches_per_step(wl) -> int:
     pooled = wl.rule != "window"
     return 3 + (2 if pooled else 1) + 2  # reorder x3, [scores], select, attention, unreorder
@@ -260,6 +278,7 @@ def main():
         raise SystemExit("device error word set")
     kept = kept_pairs_from_counts(cnt)
     flops = kept * pair_flops(wl.head_dim)
+    issued = issued_pairs(idx, cnt, plan.N)
 
     sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
     for _ in range(args.warmup):
@@ -321,6 +340,8 @@ def main():
         "dtype": "bf16+e4m3" if wl.qk_fp8 else "bf16",
         "data": "synthetic",
         "config": workload_config(wl, {"kept_pairs": kept, "kept_tflop": flops / 1e12,
+                                        "mma_tile_pairs": issued,
+                                        "pair_efficiency": kept / issued if issued else None,
                                         "parallelism": f"independent layer per GPU x{world}"}),
         "ms_per_layer": ms_per_step,
         "kernels_ms": comp,
