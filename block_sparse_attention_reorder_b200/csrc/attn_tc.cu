@@ -16,8 +16,9 @@
 //              (the running max is only moved when it grows by more than
 //              2^8, which keeps O and l exact up to rounding), write P as
 //              bf16 into the TMEM columns S came from.
-//   warp 4     TMA producer: Q block once, then K_j / V_j per step into a
-//              two-stage ring.
+//   warp 4     TMA producer: Q block once, then K_j and V_j into two
+//              separate two-stage rings (K released by its S MMA, V by its
+//              PV MMA, so the next K loads while the current PV runs).
 //   warp 5     MMA issuer (one thread): S_{n+2} = Q K^T is issued right
 //              after PV_n so it overlaps softmax n+1; O += P_n V_n reads P
 //              from TMEM (A operand) and V from shared memory (MN-major B).
@@ -73,8 +74,8 @@ struct Cfg {
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
   static constexpr int OFF_V = OFF_K + kStages * K_BYTES;
   static constexpr int OFF_BAR = OFF_V + kStages * V_BYTES;
-  // barriers: q, full[2], empty[2], sfull[2], pfull[2], pvdone[2], final
-  static constexpr int NBAR = 1 + 2 * kStages + 7;
+  // barriers: q, kfull[S], kempty[S], vfull[S], vempty[S], sfull[2], pfull[2], pvdone[2], final
+  static constexpr int NBAR = 1 + 4 * kStages + 7;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base, abort, L, pad
   static constexpr int OFF_COL = OFF_MISC + 16;         // 64 packed column coords
   static constexpr int OFF_SCAN = OFF_COL + 256;        // block-scan scratch
@@ -106,12 +107,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const uint32_t sb = tc::smem_addr(smem);
   const uint32_t bar_q = sb + C::OFF_BAR;
-  auto bar_full = [&](int s) { return sb + C::OFF_BAR + 8u * (1 + s); };
-  auto bar_empty = [&](int s) { return sb + C::OFF_BAR + 8u * (1 + kStages + s); };
-  auto bar_sfull = [&](int b) { return sb + C::OFF_BAR + 8u * (1 + 2 * kStages + b); };
-  auto bar_pfull = [&](int b) { return sb + C::OFF_BAR + 8u * (3 + 2 * kStages + b); };
-  auto bar_pvdone = [&](int b) { return sb + C::OFF_BAR + 8u * (5 + 2 * kStages + b); };
-  const uint32_t bar_final = sb + C::OFF_BAR + 8u * (7 + 2 * kStages);
+  auto bar_kfull = [&](int s) { return sb + C::OFF_BAR + 8u * (1 + s); };
+  auto bar_kempty = [&](int s) { return sb + C::OFF_BAR + 8u * (1 + kStages + s); };
+  auto bar_vfull = [&](int s) { return sb + C::OFF_BAR + 8u * (1 + 2 * kStages + s); };
+  auto bar_vempty = [&](int s) { return sb + C::OFF_BAR + 8u * (1 + 3 * kStages + s); };
+  auto bar_sfull = [&](int b) { return sb + C::OFF_BAR + 8u * (1 + 4 * kStages + b); };
+  auto bar_pfull = [&](int b) { return sb + C::OFF_BAR + 8u * (3 + 4 * kStages + b); };
+  auto bar_pvdone = [&](int b) { return sb + C::OFF_BAR + 8u * (5 + 4 * kStages + b); };
+  const uint32_t bar_final = sb + C::OFF_BAR + 8u * (7 + 4 * kStages);
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
   volatile int* never = reinterpret_cast<volatile int*>(misc + 3);  // stays 0: waits that ignore abort
@@ -132,8 +135,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   if (tid == 0) {
     tc::mbar_init(bar_q, 1);
     for (int s = 0; s < kStages; ++s) {
-      tc::mbar_init(bar_full(s), 1);
-      tc::mbar_init(bar_empty(s), 1);
+      tc::mbar_init(bar_kfull(s), 1);
+      tc::mbar_init(bar_kempty(s), 1);
+      tc::mbar_init(bar_vfull(s), 1);
+      tc::mbar_init(bar_vempty(s), 1);
     }
     for (int x = 0; x < 2; ++x) {
       tc::mbar_init(bar_sfull(x), 1);
@@ -226,32 +231,50 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 #pragma unroll
       for (int cb = 0; cb < C::QBLK; ++cb)
         tc::tma_load_2d(sb + C::OFF_Q + cb * 128 * C::SWB, &tmQ, bar_q, cb * C::SWB / C::ESZ, qrow);
-      int last[kStages];
+      // K_m is issued as soon as S_{m-2} has released its slot, V_{m-1} once
+      // PV_{m-3} has: the two rings free up in MMA completion order, so K
+      // runs one step ahead of V and its load latency hides behind softmax.
+      int lastk[kStages], lastv[kStages];
 #pragma unroll
-      for (int s = 0; s < kStages; ++s) last[s] = -1;
-      for (int n = 0; n < L; ++n) {
-        const int s = n % kStages;
-        if (n >= kStages && !tc::mbar_wait(bar_empty(s), ((n / kStages) - 1) & 1, abort_flag, kWaitLimit)) {
-          record_timeout(abort_flag, P.err);
-          break;
+      for (int s = 0; s < kStages; ++s) lastk[s] = lastv[s] = -1;
+      for (int m = 0; m <= L; ++m) {
+        if (m < L) {
+          const int s = m % kStages;
+          if (m >= kStages &&
+              !tc::mbar_wait(bar_kempty(s), ((m / kStages) - 1) & 1, abort_flag, kWaitLimit)) {
+            record_timeout(abort_flag, P.err);
+            break;
+          }
+          const int krow = (int)((bh * g.N + (int)(ulist[m] & 0x3FFFFFFFu)) * 64);
+          tc::mbar_arrive_expect_tx(bar_kfull(s), C::K_BYTES);
+#pragma unroll
+          for (int cb = 0; cb < C::QBLK; ++cb)
+            tc::tma_load_2d(sb + C::OFF_K + s * C::K_BYTES + cb * 64 * C::SWB, &tmK, bar_kfull(s),
+                            cb * C::SWB / C::ESZ, krow);
+          lastk[s] = m;
         }
-        const int j = (int)(ulist[n] & 0x3FFFFFFFu);
-        const int krow = (int)((bh * g.N + j) * 64);
-        tc::mbar_arrive_expect_tx(bar_full(s), C::K_BYTES + C::V_BYTES);
+        if (m >= 1) {
+          const int v = m - 1, s = v % kStages;
+          if (v >= kStages &&
+              !tc::mbar_wait(bar_vempty(s), ((v / kStages) - 1) & 1, abort_flag, kWaitLimit)) {
+            record_timeout(abort_flag, P.err);
+            break;
+          }
+          const int vrow = (int)((bh * g.N + (int)(ulist[v] & 0x3FFFFFFFu)) * 64);
+          tc::mbar_arrive_expect_tx(bar_vfull(s), C::V_BYTES);
 #pragma unroll
-        for (int cb = 0; cb < C::QBLK; ++cb)
-          tc::tma_load_2d(sb + C::OFF_K + s * C::K_BYTES + cb * 64 * C::SWB, &tmK, bar_full(s),
-                          cb * C::SWB / C::ESZ, krow);
-#pragma unroll
-        for (int vb = 0; vb < C::VBLK; ++vb)
-          tc::tma_load_2d(sb + C::OFF_V + s * C::V_BYTES + vb * 8192, &tmV, bar_full(s), vb * 64, krow);
-        last[s] = n;
+          for (int vb = 0; vb < C::VBLK; ++vb)
+            tc::tma_load_2d(sb + C::OFF_V + s * C::V_BYTES + vb * 8192, &tmV, bar_vfull(s), vb * 64, vrow);
+          lastv[s] = v;
+        }
       }
       if (*abort_flag) {
         // Let copies already issued land before the CTA's memory goes away.
         tc::mbar_wait(bar_q, 0, never, kWaitLimit);
-        for (int s = 0; s < kStages; ++s)
-          if (last[s] >= 0) tc::mbar_wait(bar_full(s), (last[s] / kStages) & 1, never, kWaitLimit);
+        for (int s = 0; s < kStages; ++s) {
+          if (lastk[s] >= 0) tc::mbar_wait(bar_kfull(s), (lastk[s] / kStages) & 1, never, kWaitLimit);
+          if (lastv[s] >= 0) tc::mbar_wait(bar_vfull(s), (lastv[s] / kStages) & 1, never, kWaitLimit);
+        }
       }
     }
   } else if (warp == 5) {
@@ -262,7 +285,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       bool ok = tc::mbar_wait(bar_q, 0, abort_flag, kWaitLimit);
       auto issue_S = [&](int m) -> bool {
         const int s = m % kStages;
-        if (!tc::mbar_wait(bar_full(s), (m / kStages) & 1, abort_flag, kWaitLimit)) return false;
+        if (!tc::mbar_wait(bar_kfull(s), (m / kStages) & 1, abort_flag, kWaitLimit)) return false;
         tc::fence_after_sync();
         const uint32_t dS = tmem + ((m & 1) ? kColS1 : kColS0);
 #pragma unroll
@@ -278,13 +301,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             tc::mma_ss_f16(dS, da, db, idS, kk > 0 ? 1u : 0u);
         }
         tc::mma_commit(bar_sfull(m & 1));
+        tc::mma_commit(bar_kempty(s));
         return true;
       };
       if (ok) ok = issue_S(0);
       if (ok && L > 1) ok = issue_S(1);
       for (int n = 0; ok && n < L; ++n) {
         const int s = n % kStages;
-        if (!tc::mbar_wait(bar_pfull(n & 1), (n >> 1) & 1, abort_flag, kWaitLimit)) {
+        if (!tc::mbar_wait(bar_pfull(n & 1), (n >> 1) & 1, abort_flag, kWaitLimit) ||
+            !tc::mbar_wait(bar_vfull(s), (n / kStages) & 1, abort_flag, kWaitLimit)) {
           ok = false;
           break;
         }
@@ -297,7 +322,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           tc::mma_ts_f16(tmem + kColO, pA + kk * 8, dv, idPV, (n > 0 || kk > 0) ? 1u : 0u);
         }
         tc::mma_commit(bar_pvdone(n & 1));
-        tc::mma_commit(bar_empty(s));
+        tc::mma_commit(bar_vempty(s));
         if (n + 2 < L && !issue_S(n + 2)) {
           ok = false;
           break;
@@ -337,34 +362,43 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         const float c = P.scale_log2 * (FP8 ? qsc * __ldg(P.ks + bh * g.N + j) : 1.f);
         const int bt = j / (g.nH * g.nW), bhh = (j / g.nW) % g.nH, bw = j % g.nW;
         const int vt = g.T - bt * g.tt, vh = g.H - bhh * g.th, vw = g.W - bw * g.tw;
-        const bool partial = vt < g.tt || vh < g.th || vw < g.tw;
-        float mx = -INFINITY;
+        if (vt < g.tt || vh < g.th || vw < g.tw) {  // padded keys of an edge tile
 #pragma unroll
-        for (int q = 0; q < 64; ++q) {
-          float x = __uint_as_float(sr[q]) * c;
-          if (partial) {
+          for (int q = 0; q < 64; ++q) {
             const uint32_t cc = colc[q];
             if ((int)(cc & 0xffu) >= vt || (int)((cc >> 8) & 0xffu) >= vh || (int)((cc >> 16) & 0xffu) >= vw)
-              x = -INFINITY;
+              sr[q] = 0xff800000u;  // -inf
           }
-          sr[q] = __float_as_uint(x);
-          mx = fmaxf(mx, x);
         }
+        // Row max of the raw scores: eight independent chains. c > 0, so the
+        // max of the scaled logits is c times the raw max.
+        float mx8[8];
+#pragma unroll
+        for (int a = 0; a < 8; ++a) mx8[a] = __uint_as_float(sr[a]);
+#pragma unroll
+        for (int q = 8; q < 64; ++q) mx8[q & 7] = fmaxf(mx8[q & 7], __uint_as_float(sr[q]));
+        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * c;
         const float m_new = fmaxf(m, mx);
         if (m == -INFINITY) {
           m = m_new;  // first kept tile of this row: O row is still zero
         } else if (m_new - m > kRescaleThreshold) {
-          alpha = exp2f(m - m_new);
+          alpha = tc::ex2(m - m_new);
           m = m_new;
           l *= alpha;
           need = true;
         }
-        float ls = 0.f;
+        // p = 2^(s*c - m); the row sum uses the fp32 values, eight chains.
+        float ls8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int q = 0; q < 32; ++q)
-          pk[q] = pack_bf16x2(exp2f(__uint_as_float(sr[2 * q]) - m),
-                              exp2f(__uint_as_float(sr[2 * q + 1]) - m), ls);
-        l += ls;
+        for (int q = 0; q < 32; ++q) {
+          const float p0 = tc::ex2(fmaf(__uint_as_float(sr[2 * q]), c, -m));
+          const float p1 = tc::ex2(fmaf(__uint_as_float(sr[2 * q + 1]), c, -m));
+          ls8[q & 7] += p0 + p1;
+          __nv_bfloat162 hv = __floats2bfloat162_rn(p0, p1);
+          pk[q] = *reinterpret_cast<uint32_t*>(&hv);
+        }
+        l += ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
       } else {
 #pragma unroll
         for (int q = 0; q < 32; ++q) pk[q] = 0u;
