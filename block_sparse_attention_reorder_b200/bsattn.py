@@ -71,6 +71,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "attn_block_scores": [P, P, P, P, P],
         "attn_select_from_scores": [P, P, P, P, P],
         "attn_select": [P, P, P, P, P, P, Z, P],
+        "attn_select_static": [P, P, P, P, P, P],
         "attn_quantize_e4m3": [P, P, P, P, P],
         "attn_forward": [P, P, P, P, P, P, P, P, P, P, P, Z, P],
         "attn_layer": [P, P, P, P, P, P, P, P, P, Z, P],
@@ -87,7 +88,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
 _lib = load_library()
 EXPORTED = ("attn_plan_create", "attn_plan_destroy", "attn_plan_info", "attn_status_string",
             "attn_reorder", "attn_pool", "attn_unreorder", "attn_block_scores",
-            "attn_select_from_scores", "attn_select", "attn_quantize_e4m3", "attn_forward",
+            "attn_select_from_scores", "attn_select", "attn_select_static", "attn_quantize_e4m3",
+            "attn_forward",
             "attn_layer", "attn_check_device_status")
 
 
@@ -224,6 +226,21 @@ def attn_select(plan: Plan, q_nat, k_nat, idx, cnt, ws, stream=None):
     _want(cnt, torch.int32, sc, "cnt")
     _check(_lib.attn_select(plan.handle, _ptr(q_nat), _ptr(k_nat), _ptr(idx), _ptr(cnt), _ptr(ws),
                             ws.numel() * ws.element_size(), _stream(stream)), "attn_select")
+
+
+STATIC_SELECT_SCRATCH_BYTES = 16 << 20
+
+
+def attn_select_static(plan: Plan, q_nat, k_nat, idx, cnt, stream=None):
+    """attn_select for callers that cannot allocate: scratch is the library's
+    static device array (see include/bsattn.h for its limits)."""
+    _want(q_nat, torch.bfloat16, plan.natural_shape(), "q_nat")
+    _want(k_nat, torch.bfloat16, plan.natural_shape(), "k_nat")
+    si, sc = plan.list_shapes()
+    _want(idx, torch.int32, si, "idx")
+    _want(cnt, torch.int32, sc, "cnt")
+    _check(_lib.attn_select_static(plan.handle, _ptr(q_nat), _ptr(k_nat), _ptr(idx), _ptr(cnt),
+                                   _stream(stream)), "attn_select_static")
 
 
 def attn_quantize_e4m3(plan: Plan, x_tiled, codes, scales, stream=None):

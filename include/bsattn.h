@@ -154,6 +154,30 @@ bsattn_status attn_select(const bsattn_plan* plan, const void* q_nat, const void
                           int32_t* idx, int32_t* cnt, void* ws, size_t ws_bytes,
                           void* stream);
 
+/* Capacity of the library-owned scratch used by attn_select_static. */
+#define BSATTN_STATIC_SELECT_SCRATCH_BYTES (16u << 20)
+
+/* attn_select without a caller workspace (the paper has no counterpart; this
+ * is a convenience of this library). For callers that cannot allocate device
+ * memory themselves, e.g. code that runs where cudaMalloc is not allowed or
+ * whose allocator is owned by someone else. The pooled Q/K and the score
+ * matrix live in one static device array of
+ * BSATTN_STATIC_SELECT_SCRATCH_BYTES bytes that every GPU loading the library
+ * holds until the process exits. The call itself allocates nothing.
+ * - The first call on a device looks the array's device address up (once per
+ *   device, with that device current); make that first call before any
+ *   stream capture.
+ * - Problems whose select workspace (info.select_workspace_bytes) exceeds the
+ *   capacity are rejected with BSATTN_ERR_UNSUPPORTED; the window rule needs
+ *   no scratch.
+ * - All calls share the one array: calls that may overlap on the GPU (other
+ *   streams, other threads) race and must be serialised by the caller. No
+ *   part of the array needs to start at zero: each call writes every byte it
+ *   reads before reading it.
+ * Results equal attn_select's for the same inputs. */
+bsattn_status attn_select_static(const bsattn_plan* plan, const void* q_nat, const void* k_nat,
+                                 int32_t* idx, int32_t* cnt, void* stream);
+
 /* Per-tile e4m3 quantisation of a tiled bf16 tensor: per (b, head, tile)
  * scale = fp32(amax)/448 (amax 0 -> 1), code = e4m3(x/scale) rounded to
  * nearest even with finite saturation (OCP E4M3). */
