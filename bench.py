@@ -70,10 +70,21 @@ def pair_flops(head_dim: int) -> float:
     return 4.0 * 64 * 64 * head_dim
 
 
-def issued_pairs(idx: torch.Tensor, cnt: torch.Tensor, N: int) -> int:
-    """Tile pairs the attention kernel multiplies: it stacks query tiles
-    2p and 2p+1 into one 128-row block over the union of their lists, so
-    each union entry costs two tile pairs of MMA work."""
+def group_axes(wl):
+    """(pair axis, unused) of the attention kernel's query-tile pairs."""
+    if wl.rule == "window" and wl.win[2] == 0:
+        return 0, 1
+    return 2, 0
+
+
+def group_accounting(wl, plan, idx: torch.Tensor, cnt: torch.Tensor):
+    """Work the attention kernel does beyond the kept pairs.
+
+    Query tiles are stacked in pairs along one tile axis (one M = 128 block).
+    A pair loads each key tile in the union of its two lists once and
+    multiplies two tile pairs for it. Returns (MMA tile pairs, K/V tile loads).
+    """
+    N = plan.N
     rows = cnt.numel()
     kmax = idx.shape[-1]
     ii = idx.reshape(rows, kmax).to(torch.int64)
@@ -81,11 +92,21 @@ def issued_pairs(idx: torch.Tensor, cnt: torch.Tensor, N: int) -> int:
     hit = torch.zeros((rows, N), dtype=torch.bool, device=idx.device)
     r = torch.arange(rows, device=idx.device)[:, None].expand(rows, kmax)
     hit[r[valid], ii[valid]] = True
-    hit = hit.reshape(-1, N, N)  # [B*heads, query tile, key tile]
-    if N % 2:
-        hit = torch.cat([hit, torch.zeros_like(hit[:, :1])], dim=1)
-    union = hit[:, 0::2] | hit[:, 1::2]
-    return int(union.sum().item()) * 2
+    info = plan.info
+    hit = hit.reshape(-1, info.nT, info.nH, info.nW, N)
+    pa, ga = group_axes(wl)
+    for ax in (pa, ga):
+        if hit.shape[1 + ax] % 2:
+            pad = list(hit.shape)
+            pad[1 + ax] = 1
+            hit = torch.cat([hit, torch.zeros(pad, dtype=torch.bool, device=hit.device)], dim=1 + ax)
+
+    def fold(x, ax):
+        a = x.narrow(1 + ax, 0, x.shape[1 + ax])
+        return a.unfold(1 + ax, 2, 2).any(dim=-1)
+
+    pairs = fold(hit, pa)
+    return int(pairs.sum().item()) * 2, int(pairs.sum().item())
 
 
 def launches_per_step(wl) -> int:
@@ -278,7 +299,7 @@ def main():
         raise SystemExit("device error word set")
     kept = kept_pairs_from_counts(cnt)
     flops = kept * pair_flops(wl.head_dim)
-    issued = issued_pairs(idx, cnt, plan.N)
+    issued, loads = group_accounting(wl, plan, idx, cnt)
 
     sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
     for _ in range(args.warmup):
@@ -342,6 +363,8 @@ def main():
         "config": workload_config(wl, {"kept_pairs": kept, "kept_tflop": flops / 1e12,
                                         "mma_tile_pairs": issued,
                                         "pair_efficiency": kept / issued if issued else None,
+                                        "kv_tile_loads": loads,
+                                        "kv_loads_per_kept_pair": loads / kept if kept else None,
                                         "parallelism": f"independent layer per GPU x{world}"}),
         "ms_per_layer": ms_per_step,
         "kernels_ms": comp,

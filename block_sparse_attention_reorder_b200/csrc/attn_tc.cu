@@ -1,8 +1,10 @@
 // Block-sparse attention forward over kept tile pairs on the 5th-generation
 // tensor cores (tcgen05, TMEM accumulators, TMA-fed shared memory).
 //
-// Work unit: two adjacent query tiles i0 = 2p, i1 = 2p + 1 of one (batch,
-// head), stacked into one 128-row query block so that every QK^T and PV
+// Work unit: two adjacent query tiles i0, i1 of one (batch, head), next to
+// each other along one axis of the tile grid (w for top-k / top-p, t for a
+// window that does not reach along w), stacked into one 128-row query
+// block so that every QK^T and PV
 // product is an M = 128 tcgen05.mma. The block walks the union of the two
 // tiles' kept key-tile lists in ascending order; a key tile kept by only one
 // of the two query tiles gives zero probabilities to the other tile's rows.
@@ -55,6 +57,8 @@ struct TcParams {
   int* err;
   int umax;      // union list capacity (entries)
   int bm_words;  // bitmap words per list
+  int pair_axis; // 0 = t, 1 = h, 2 = w
+  int pdim[3];   // work items along t, h, w (pair axis halved)
 };
 
 template <int D, bool FP8>
@@ -125,10 +129,24 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   uint32_t* ulist = bmB + P.bm_words;
 
   const Geom& g = P.g;
-  const int i0 = 2 * blockIdx.x, i1 = i0 + 1;
+  // Work item -> its two member tiles along the pair axis (i1 = -1 at an
+  // odd grid edge).
+  int i0, i1;
+  {
+    const int nd[3] = {g.nT, g.nH, g.nW};
+    int c[3], rem = blockIdx.x;
+    c[2] = rem % P.pdim[2];
+    rem /= P.pdim[2];
+    c[1] = rem % P.pdim[1];
+    c[0] = rem / P.pdim[1];
+    c[P.pair_axis] *= 2;
+    i0 = (c[0] * g.nH + c[1]) * g.nW + c[2];
+    c[P.pair_axis] += 1;
+    i1 = c[P.pair_axis] < nd[P.pair_axis] ? (c[0] * g.nH + c[1]) * g.nW + c[2] : -1;
+  }
   const int head = blockIdx.y, b = blockIdx.z;
   const size_t bh = (size_t)b * g.Hh + head;
-  const bool has1 = i1 < g.N;
+  const bool has1 = i1 >= 0;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   // ------------------------------------------------------------ setup
@@ -159,6 +177,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     colc[tid] = (uint32_t)dt | ((uint32_t)dh << 8) | ((uint32_t)dw << 16);
   }
   for (int w = tid; w < 2 * P.bm_words; w += kThreads) bmA[w] = 0u;
+  if (!has1) {
+    // Rows 64..127 of the query block have no tile: zero them so no stale
+    // bit pattern reaches the tensor cores.
+    for (int x = tid; x < C::QBLK * 64 * C::SWB / 16; x += kThreads) {
+      const int cb = x / (64 * C::SWB / 16), off = x % (64 * C::SWB / 16);
+      reinterpret_cast<uint4*>(smem + C::OFF_Q + cb * 128 * C::SWB + 64 * C::SWB)[off] = make_uint4(0, 0, 0, 0);
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
   __syncthreads();
 
   // Union of the two kept lists as a bitmap pair, then compacted ascending.
@@ -171,7 +198,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   }
   {
     const int32_t* lA = P.idx + (bh * g.N + i0) * (size_t)P.kmax;
-    const int32_t* lB = lA + P.kmax;
+    const int32_t* lB = has1 ? P.idx + (bh * g.N + i1) * (size_t)P.kmax : lA;
     for (int e = tid; e < nA + nB; e += kThreads) {
       int j = e < nA ? __ldg(lA + e) : __ldg(lB + (e - nA));
       if (j < 0 || j >= g.N) {
@@ -226,11 +253,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       tc::tma_prefetch_desc(&tmQ);
       tc::tma_prefetch_desc(&tmK);
       tc::tma_prefetch_desc(&tmV);
-      const int qrow = (int)((bh * g.N + i0) * 64);
-      tc::mbar_arrive_expect_tx(bar_q, C::Q_BYTES);
+      tc::mbar_arrive_expect_tx(bar_q, (has1 ? 2 : 1) * 64 * C::QRB);
+      for (int x = 0; x < (has1 ? 2 : 1); ++x) {
+        const int qrow = (int)((bh * g.N + (x ? i1 : i0)) * 64);
 #pragma unroll
-      for (int cb = 0; cb < C::QBLK; ++cb)
-        tc::tma_load_2d(sb + C::OFF_Q + cb * 128 * C::SWB, &tmQ, bar_q, cb * C::SWB / C::ESZ, qrow);
+        for (int cb = 0; cb < C::QBLK; ++cb)
+          tc::tma_load_2d(sb + C::OFF_Q + cb * 128 * C::SWB + x * 64 * C::SWB, &tmQ, bar_q, cb * C::SWB / C::ESZ,
+                          qrow);
+      }
       // K_m is issued as soon as S_{m-2} has released its slot, V_{m-1} once
       // PV_{m-3} has: the two rings free up in MMA completion order, so K
       // runs one step ahead of V and its load latency hides behind softmax.
@@ -456,14 +486,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         reinterpret_cast<uint4*>(stage + c0 * 2)[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
     }
     if (P.lse && row_exists)
-      P.lse[(bh * g.N + i0) * 64 + r] = l > 0.f ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
+      P.lse[(bh * g.N + (half ? i1 : i0)) * 64 + (r & 63)] =
+          l > 0.f ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
     asm volatile("bar.sync 1, 128;" ::: "memory");
     constexpr int CPR = D / 8;  // 16-byte chunks per row
     const int rows = has1 ? 128 : 64;
-    uint4* og = reinterpret_cast<uint4*>(P.o + (bh * g.N + i0) * 64 * (size_t)D);
     for (int e2 = r; e2 < rows * CPR; e2 += 128) {
       const int rr = e2 / CPR, cc = e2 % CPR;
-      og[e2] = *reinterpret_cast<const uint4*>(smem + C::OFF_K + rr * C::O_PITCH + cc * 16);
+      uint4* og = reinterpret_cast<uint4*>(P.o + (bh * g.N + (rr >> 6 ? i1 : i0)) * 64 * (size_t)D);
+      og[(rr & 63) * CPR + cc] = *reinterpret_cast<const uint4*>(smem + C::OFF_K + rr * C::O_PITCH + cc * 16);
     }
   }
 
@@ -512,7 +543,7 @@ bsattn_status run(const bsattn_plan* p, const void* q, const void* k, const __nv
   CUtensorMap mq, mk, mv;
   const CUtensorMapDataType dqk = FP8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const CUtensorMapSwizzle sw = C::SWB == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
-  if (!make_map(&mq, q, dqk, C::ESZ, D, rows, C::SWB / C::ESZ, 128, sw) ||
+  if (!make_map(&mq, q, dqk, C::ESZ, D, rows, C::SWB / C::ESZ, 64, sw) ||
       !make_map(&mk, k, dqk, C::ESZ, D, rows, C::SWB / C::ESZ, 64, sw) ||
       !make_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, rows, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B))
     return BSATTN_ERR_CUDA;
@@ -522,7 +553,7 @@ bsattn_status run(const bsattn_plan* p, const void* q, const void* k, const __nv
   auto kern = attn_tc_kernel<D, FP8>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return BSATTN_ERR_CUDA;
-  dim3 grid((p->N + 1) / 2, p->desc.heads, p->desc.B);
+  dim3 grid(prm.pdim[0] * prm.pdim[1] * prm.pdim[2], p->desc.heads, p->desc.B);
   kern<<<grid, kThreads, smem, st>>>(mq, mk, mv, prm);
   return cudaGetLastError() == cudaSuccess ? BSATTN_OK : BSATTN_ERR_CUDA;
 }
@@ -549,6 +580,12 @@ bsattn_status launch_attention(const bsattn_plan* p, const void* q, const void* 
   prm.err = p->d_err;
   prm.umax = p->N < 2 * p->kmax ? p->N : 2 * p->kmax;
   prm.bm_words = (p->N + 31) / 32;
+  // Pairs along w for top-k / top-p (neighbouring query tiles keep similar
+  // key tiles); along t for a window that does not reach along w, whose
+  // w-neighbours share no key tile.
+  prm.pair_axis = (p->rule.kind == BSATTN_RULE_WINDOW && p->rule.win_w == 0) ? 0 : 2;
+  const int nd[3] = {p->nT, p->nH, p->nW};
+  for (int a = 0; a < 3; ++a) prm.pdim[a] = a == prm.pair_axis ? (nd[a] + 1) / 2 : nd[a];
   const bool fp8 = p->desc.qk_fp8 != 0;
   if (p->desc.head_dim == 128)
     return fp8 ? run<128, true>(p, q, k, v, prm, st) : run<128, false>(p, q, k, v, prm, st);
