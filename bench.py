@@ -61,6 +61,22 @@ def peaks():
                 "source": "fallback"}
 
 
+def measured_traffic(workload: str):
+    """DRAM bytes per attention launch from the committed ncu capture, or None
+    when the kernel source has changed since the counters were taken."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "attn_tc_traffic.json")) as f:
+            rec = json.load(f)
+        with open(os.path.join(ROOT, rec["kernel_source"]), "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()[:16]
+        if sha != rec["sha256_prefix"]:
+            return None
+        return rec["per_launch_dram_bytes"].get(workload)
+    except Exception:
+        return None
+
+
 def kept_pairs_from_counts(cnt: torch.Tensor) -> int:
     return int(cnt.to(torch.int64).sum().item())
 
@@ -372,7 +388,7 @@ def main():
                      "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": achieved / pk["bf16_tflops"],
                      "peak_note": f"{pk['source']} bf16 burst (kernel timed alone)",
-                     "traffic": None},
+                     "traffic": measured_traffic(wl.name)},
         "memory_kernels": memory_kernel_rates(wl, plan, comp, pk),
         "e2e": e2e,
         "gpu_launches": launches_per_step(wl) * args.steps,
