@@ -1,12 +1,36 @@
 // Key-tile selection on a block-score matrix: exact top-k, top-p with a
 // top-k floor, and the broadcast of the fixed window lists.
 //
-// Ordering: a score maps to a 32-bit unsigned key that orders like the
-// float (-0.0 is folded into +0.0 first, so they tie); ties are broken by
-// the lower tile index. Lists are written ascending.
+// Ordering: tiles run by score descending, equal scores (-0.0 and +0.0 are
+// equal) by tile index ascending. A 64-bit composite key (an order-preserving
+// integer image of the score << 32 | ~index) is unique per tile and orders
+// tiles that way. Both rules come down to one search: walking the row in that
+// order with a non-negative weight per tile (1 for a count, the softmax mass
+// for top-p), find the first tile at which the running weight reaches a target
+// R. Every tile up to and including it is kept; lists are written ascending.
+//
+// One warp per row; the row is staged in the warp's slice of shared memory
+// (lane l's i-th value is tile l + 32 i). The search never sorts the row: the
+// scores of the current range are binned into 256 equal-width bins with one
+// FMA (monotone in the score, so bins keep the order), a per-warp weight
+// histogram locates the bin where the running weight reaches R, and that bin
+// becomes the next range. A bin of at most 32 tiles is ranked exactly across
+// the warp's lanes; a range of one score value (a run of tied tiles) is
+// resolved by index order. A bounded number of levels, then a bit-by-bit
+// search over the composite keys, covers whatever is left (infinite scores,
+// ranges too narrow to split).
+//
+// Top-p mass: e_j = exp(s_j - max_j s) in fp64, held as an integer in units of
+// 2^-52 (so e_max = 2^52). Integer sums are exact in any order, so the result
+// does not depend on atomics or reduction order. With at most 2048 tiles the
+// rounding moves a normalised prefix mass by at most 2048 * 2^-53 < 2.3e-13.
 #include "internal.h"
 
 namespace {
+
+constexpr int kBins = 256;
+constexpr int kCand = 32;   // bin size ranked directly
+constexpr int kLevels = 4;  // histogram refinements before the bitwise search
 
 __device__ __forceinline__ uint32_t order_key(float x) {
   uint32_t u = __float_as_uint(x);
@@ -15,189 +39,398 @@ __device__ __forceinline__ uint32_t order_key(float x) {
 }
 
 __device__ __forceinline__ float key_to_float(uint32_t k) {
-  uint32_t u = (k & 0x80000000u) ? (k & 0x7fffffffu) : ~k;
+  const uint32_t u = (k & 0x80000000u) ? (k & 0x7fffffffu) : ~k;
   return __uint_as_float(u);
 }
 
-// ---------------------------------------------------------------------------
-// Top-k: one warp per row, the row's keys in registers (lane l holds columns
-// l, l+32, ...). The k-th largest key v is found by a bitwise search from the
-// most significant bit (count of keys >= candidate, warp-reduced). Keys > v
-// are kept, and of the keys == v the lowest-index (k - #{> v}) ones.
-// ---------------------------------------------------------------------------
-template <int VPT>
-__global__ void __launch_bounds__(256)
-topk_kernel(int rows, int N, int k, const float* __restrict__ S, int32_t* __restrict__ idx,
-            int32_t* __restrict__ cnt, int kmax) {
-  const int lane = threadIdx.x & 31;
-  const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (row >= rows) return;
-  const float* s = S + (size_t)row * N;
-  uint32_t key[VPT];
-#pragma unroll
-  for (int i = 0; i < VPT; ++i) {
-    int j = lane + 32 * i;
-    key[i] = j < N ? order_key(__ldg(s + j)) : 0u;  // 0 is below every real key
-  }
-  uint32_t v = 0;
-  for (int bit = 31; bit >= 0; --bit) {
-    uint32_t c = v | (1u << bit);
-    uint32_t n = 0;
-#pragma unroll
-    for (int i = 0; i < VPT; ++i) n += key[i] >= c;
-    if (__reduce_add_sync(0xffffffffu, n) >= (uint32_t)k) v = c;
-  }
-  uint32_t gt = 0;
-#pragma unroll
-  for (int i = 0; i < VPT; ++i) gt += key[i] > v;
-  const int need_eq = k - (int)__reduce_add_sync(0xffffffffu, gt);
-  const uint32_t lt_mask = (1u << lane) - 1u;
-  int base = 0, eq_seen = 0;
-  int32_t* out = idx + (size_t)row * kmax;
-#pragma unroll
-  for (int i = 0; i < VPT; ++i) {
-    int j = lane + 32 * i;
-    bool eq = (j < N) && key[i] == v;
-    uint32_t eqm = __ballot_sync(0xffffffffu, eq);
-    bool keep = key[i] > v || (eq && eq_seen + __popc(eqm & lt_mask) < need_eq);
-    eq_seen += __popc(eqm);
-    uint32_t km = __ballot_sync(0xffffffffu, keep);
-    if (keep) out[base + __popc(km & lt_mask)] = j;
-    base += __popc(km);
-  }
-  if (lane == 0) cnt[row] = base;
+__device__ __forceinline__ uint64_t comp_key(float x, int j) {
+  return ((uint64_t)order_key(x) << 32) | (uint64_t)(0xffffffffu - (uint32_t)j);
 }
 
-// ---------------------------------------------------------------------------
-// Top-p with a top-k floor: one CTA per row. The row's 64-bit keys
-// (order key << 32 | ~index) are bitonic-sorted descending in shared memory,
-// which orders by (score desc, index asc). Then, in fp64: pi_m =
-// exp(s_m - s_max) / sum, inclusive prefix sums c_m, m* = first m with
-// c_m >= p, kept = min(N, max(m*, k)). The kept indices are flagged and
-// compacted in ascending order.
-// ---------------------------------------------------------------------------
-constexpr int kTopPThreads = 256;
+__device__ __forceinline__ uint64_t shfl_idx_u64(uint64_t v, int src) {
+  return ((uint64_t)__shfl_sync(0xffffffffu, (uint32_t)(v >> 32), src) << 32) |
+         __shfl_sync(0xffffffffu, (uint32_t)v, src);
+}
+__device__ __forceinline__ uint64_t shfl_xor_u64(uint64_t v, int o) {
+  return ((uint64_t)__shfl_xor_sync(0xffffffffu, (uint32_t)(v >> 32), o) << 32) |
+         __shfl_xor_sync(0xffffffffu, (uint32_t)v, o);
+}
+__device__ __forceinline__ uint64_t shfl_up_u64(uint64_t v, int o) {
+  return ((uint64_t)__shfl_up_sync(0xffffffffu, (uint32_t)(v >> 32), o) << 32) |
+         __shfl_up_sync(0xffffffffu, (uint32_t)v, o);
+}
+__device__ __forceinline__ uint64_t shfl_down_u64(uint64_t v, int o) {
+  return ((uint64_t)__shfl_down_sync(0xffffffffu, (uint32_t)(v >> 32), o) << 32) |
+         __shfl_down_sync(0xffffffffu, (uint32_t)v, o);
+}
+__device__ __forceinline__ uint64_t warp_sum_u64(uint64_t v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += shfl_xor_u64(v, o);
+  return v;
+}
 
-__device__ __forceinline__ double block_sum_f64(double v, double* red) {
+// Softmax mass of score x relative to the row max, in units of 2^-52.
+__device__ __forceinline__ uint64_t mass_q(float x, double smax) {
+  return __double2ull_rn(exp((double)x - smax) * 4503599627370496.0);
+}
+
+// Tile weight: 1 for a count, the fixed-point mass otherwise.
+template <bool MASS>
+__device__ __forceinline__ uint64_t weight_of(float x, double smax) {
+  if constexpr (MASS)
+    return mass_q(x, smax);
+  else
+    return 1ull;
+}
+
+// Equal-width binning of the range [lo, hi] (lo < hi): one rounding of
+// x * sc + off, so monotone in x; the clamp absorbs rounding at the edges and
+// saturated or NaN conversions (a range that overflows puts every tile in bin
+// 0, and the search moves on to the bitwise step).
+struct Binning {
+  float sc, off;
+  __device__ __forceinline__ Binning(float lo, float hi) {
+    sc = (float)kBins / (hi - lo);
+    off = -lo * sc;
+  }
+  __device__ __forceinline__ int operator()(float x) const {
+    return min(max(__float2int_rz(fmaf(x, sc, off)), 0), kBins - 1);
+  }
+};
+
+// The warp's staged row: lane l's i-th value is tile l + 32 i.
+struct Row {
+  const float* p;  // &slice[lane]
+  int N, lane;
+  __device__ __forceinline__ float operator[](int i) const { return p[32 * i]; }
+  __device__ __forceinline__ bool valid(int i) const { return lane + 32 * i < N; }
+};
+
+struct Hist {
+  uint32_t* cnt;  // [kBins] tile count per bin
+  uint64_t* wt;   // [kBins] weight per bin (mass only)
+};
+
+__device__ __forceinline__ bool in_range(float x, float lo, float hi) { return x >= lo && x <= hi; }
+
+template <int VPT, bool MASS>
+__device__ __forceinline__ void build_hist(const Row& row, bool whole, float lo, float hi, const Binning& bin,
+                                           double smax, Hist h) {
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
-  __syncthreads();
-  double t = 0.0;
+  for (int q = 0; q < kBins / 32; ++q) {
+    h.cnt[row.lane + 32 * q] = 0;
+    if constexpr (MASS) h.wt[row.lane + 32 * q] = 0;
+  }
+  __syncwarp();
+#pragma unroll 8
+  for (int i = 0; i < VPT; ++i) {
+    const float x = row[i];
+    if (row.valid(i) && (whole || in_range(x, lo, hi))) {
+      const int b = bin(x);
+      atomicAdd(&h.cnt[b], 1u);
+      if constexpr (MASS) atomicAdd((unsigned long long*)&h.wt[b], (unsigned long long)mass_q(x, smax));
+    }
+  }
+  __syncwarp();
+}
+
+// Bin b (higher bins hold higher scores) in which the running weight, taken
+// from the top bin down, reaches R > 0; *above gets the weight of all higher
+// bins. Lane l owns bins [8l, 8l+8). Returns -1 if the total is below R.
+template <bool MASS>
+__device__ __forceinline__ int find_bin(Hist h, uint64_t R, int lane, uint64_t* above) {
+  uint64_t c[8], s = 0;
 #pragma unroll
-  for (int w = 0; w < kTopPThreads / 32; ++w) t += red[w];
-  __syncthreads();
+  for (int q = 0; q < 8; ++q) {
+    c[q] = MASS ? h.wt[8 * lane + q] : (uint64_t)h.cnt[8 * lane + q];
+    s += c[q];
+  }
+  uint64_t x = s;  // inclusive suffix sum over lanes
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint64_t y = shfl_down_u64(x, o);
+    if (lane + o < 32) x += y;
+  }
+  uint64_t run = x - s;
+  int hit = -1;
+  uint64_t hit_above = 0;
+#pragma unroll
+  for (int q = 7; q >= 0; --q) {
+    if (hit < 0 && run < R && R - run <= c[q]) {
+      hit = 8 * lane + q;
+      hit_above = run;
+    }
+    run += c[q];
+  }
+  const uint32_t m = __ballot_sync(0xffffffffu, hit >= 0);
+  if (!m) return -1;
+  const int src = __ffs(m) - 1;  // at most one bin crosses R
+  *above = shfl_idx_u64(hit_above, src);
+  return __shfl_sync(0xffffffffu, hit, src);
+}
+
+// Largest composite key t whose upper set {keys >= t} weighs at least R: the
+// key of the tile at which the running weight reaches R.
+template <int VPT, bool MASS>
+__device__ uint64_t bisect_key(const Row& row, uint64_t R, double smax) {
+  uint64_t t = 0;
+  for (int bit = 63; bit >= 0; --bit) {
+    const uint64_t c = t | (1ull << bit);
+    uint64_t w = 0;
+    for (int i = 0; i < VPT; ++i)
+      if (row.valid(i) && comp_key(row[i], row.lane + 32 * i) >= c) w += weight_of<MASS>(row[i], smax);
+    if (warp_sum_u64(w) >= R) t = c;
+  }
   return t;
 }
 
-// Exclusive prefix over threads of a per-thread value (fp64 or int), in
-// thread order; also returns the total.
-template <typename T>
-__device__ __forceinline__ T block_exclusive_scan(T v, T* red, T* total) {
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  T x = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    T y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
-  }
-  if (lane == 31) red[w] = x;
-  __syncthreads();
-  T off = 0, tot = 0;
-#pragma unroll
-  for (int i = 0; i < kTopPThreads / 32; ++i) {
-    if (i < w) off += red[i];
-    tot += red[i];
-  }
-  __syncthreads();
-  *total = tot;
-  return off + x - v;
-}
-
-template <int NP>
-__global__ void __launch_bounds__(kTopPThreads)
-topp_kernel(int N, int k, double p, const float* __restrict__ S, int32_t* __restrict__ idx,
-            int32_t* __restrict__ cnt, int kmax) {
-  constexpr int PER = NP / kTopPThreads > 0 ? NP / kTopPThreads : 1;
-  __shared__ unsigned long long keys[NP];
-  __shared__ unsigned char flag[NP];
-  __shared__ double redd[kTopPThreads / 32];
-  __shared__ int redi[kTopPThreads / 32];
-  __shared__ int mstar_s;
-  const size_t row = blockIdx.x;
-  const float* s = S + row * N;
-  for (int j = threadIdx.x; j < NP; j += kTopPThreads) {
-    keys[j] = j < N ? ((unsigned long long)order_key(__ldg(s + j)) << 32) |
-                          (unsigned long long)(0xffffffffu - (uint32_t)j)
-                    : 0ull;
-    flag[j] = 0;
-  }
-  if (threadIdx.x == 0) mstar_s = N;
-  __syncthreads();
-  // Bitonic sort, descending.
-  for (int size = 2; size <= NP; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int t = threadIdx.x; t < NP / 2; t += kTopPThreads) {
-        int a = 2 * t - (t & (stride - 1));
-        int b = a + stride;
-        bool desc = (a & size) == 0;
-        unsigned long long x = keys[a], y = keys[b];
-        if (desc ? (x < y) : (x > y)) {
-          keys[a] = y;
-          keys[b] = x;
+// The search described at the top of the file. On entry `h` holds the
+// histogram of the whole row under Binning(lo, hi), [lo, hi] being the row's
+// finite-or-not extent. Requires 1 <= R <= the row's total weight.
+template <int VPT, bool MASS>
+__device__ uint64_t crossing_key(const Row& row, uint64_t R, double smax, float lo, float hi, Hist h,
+                                 uint64_t* cand) {
+  const int lane = row.lane;
+  const uint32_t lt = (1u << lane) - 1u;
+  uint64_t A = 0;  // weight of the tiles above the current range
+  bool whole = true;
+  for (int level = 0; level < kLevels; ++level) {
+    if (!(lo < hi)) {
+      if (!(lo == hi)) break;  // NaN extent
+      // One score value: its tiles run in ascending index order, each with
+      // the same weight w; the crossing is the ceil((R - A) / w)-th of them.
+      const uint64_t w = weight_of<MASS>(lo, smax);
+      if (w == 0 || R <= A) break;
+      const uint64_t need = (R - A + w - 1) / w;
+      uint64_t base = 0;
+      for (int i = 0; i < VPT; ++i) {
+        const uint32_t m = __ballot_sync(0xffffffffu, row.valid(i) && row[i] == lo);
+        const uint64_t pc = (uint64_t)__popc(m);
+        if (base < need && need <= base + pc) {
+          uint32_t mm = m;  // drop the lowest (need - base - 1) set lanes
+          for (uint64_t s = 1; s < need - base; ++s) mm &= mm - 1;
+          return comp_key(lo, 32 * i + __ffs(mm) - 1);
         }
+        base += pc;
       }
-      __syncthreads();
-    }
-  }
-  const double smax = (double)key_to_float((uint32_t)(keys[0] >> 32));
-  // Thread t owns sorted positions [t*PER, (t+1)*PER).
-  double e[PER];
-  double local = 0.0;
-#pragma unroll
-  for (int i = 0; i < PER; ++i) {
-    int m = threadIdx.x * PER + i;
-    e[i] = m < N ? exp((double)key_to_float((uint32_t)(keys[m] >> 32)) - smax) : 0.0;
-    local += e[i];
-  }
-  // Total mass: sum of the per-thread sums (fixed order), then pi = e / total.
-  const double total = block_sum_f64(local, redd);
-  double run = 0.0;
-#pragma unroll
-  for (int i = 0; i < PER; ++i) {
-    e[i] = e[i] / total;
-    run += e[i];
-  }
-  double all;
-  double c = block_exclusive_scan<double>(run, redd, &all);
-#pragma unroll
-  for (int i = 0; i < PER; ++i) {
-    int m = threadIdx.x * PER + i;
-    c += e[i];
-    if (m < N && c >= p) {
-      atomicMin(&mstar_s, m + 1);
       break;
     }
-  }
-  __syncthreads();
-  int kept = max(mstar_s, k);
-  kept = min(kept, N);
-  for (int m = threadIdx.x; m < kept; m += kTopPThreads)
-    flag[0xffffffffu - (uint32_t)(keys[m] & 0xffffffffull)] = 1;
-  __syncthreads();
-  // Ascending compaction: thread t owns indices [t*PER, (t+1)*PER).
-  int mine = 0;
+    const Binning bin(lo, hi);
+    if (!whole) build_hist<VPT, MASS>(row, false, lo, hi, bin, smax, h);
+    uint64_t above = 0;
+    const int b = find_bin<MASS>(h, R - A, lane, &above);
+    if (b < 0) break;
+    A += above;
+    const uint32_t nb = h.cnt[b];
+    if (nb <= (uint32_t)kCand) {
+      // Rank the bin's tiles exactly: gather one per lane, sort descending.
+      int base = 0;
+#pragma unroll 8
+      for (int i = 0; i < VPT; ++i) {
+        const float x = row[i];
+        const bool in = row.valid(i) && (whole || in_range(x, lo, hi)) && bin(x) == b;
+        const uint32_t m = __ballot_sync(0xffffffffu, in);
+        const int pos = base + __popc(m & lt);
+        if (in && pos < kCand) cand[pos] = comp_key(x, lane + 32 * i);
+        base += __popc(m);
+      }
+      __syncwarp();
+      uint64_t ck = lane < (int)nb ? cand[lane] : 0ull;
+      __syncwarp();
 #pragma unroll
-  for (int i = 0; i < PER; ++i) mine += flag[threadIdx.x * PER + i];
-  int tot;
-  int pos = block_exclusive_scan<int>(mine, redi, &tot);
-  int32_t* out = idx + row * kmax;
+      for (int size = 2; size <= 32; size <<= 1)
 #pragma unroll
-  for (int i = 0; i < PER; ++i) {
-    int j = threadIdx.x * PER + i;
-    if (flag[j]) out[pos++] = j;
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+          const uint64_t ok = shfl_xor_u64(ck, stride);
+          const bool take_max = ((lane & stride) == 0) == ((lane & size) == 0);
+          if (take_max ? ok > ck : ok < ck) ck = ok;
+        }
+      uint64_t c;  // inclusive prefix of the sorted weights
+      if constexpr (MASS) {
+        c = ck ? mass_q(key_to_float((uint32_t)(ck >> 32)), smax) : 0ull;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint64_t y = shfl_up_u64(c, o);
+          if (lane >= o) c += y;
+        }
+      } else {
+        c = (uint64_t)(lane + 1);
+      }
+      const uint32_t m = __ballot_sync(0xffffffffu, ck != 0 && A + c >= R);
+      if (m) return shfl_idx_u64(ck, __ffs(m) - 1);
+      break;
+    }
+    // Next range: the extent of bin b's scores.
+    uint32_t klo = 0xffffffffu, khi = 0u;
+#pragma unroll 8
+    for (int i = 0; i < VPT; ++i) {
+      const float x = row[i];
+      if (row.valid(i) && (whole || in_range(x, lo, hi)) && bin(x) == b) {
+        const uint32_t k = order_key(x);
+        klo = min(klo, k);
+        khi = max(khi, k);
+      }
+    }
+    klo = __reduce_min_sync(0xffffffffu, klo);
+    khi = __reduce_max_sync(0xffffffffu, khi);
+    if (klo > khi) break;
+    lo = key_to_float(klo);
+    hi = key_to_float(khi);
+    whole = false;
   }
-  if (threadIdx.x == 0) cnt[row] = kept;
+  return bisect_key<VPT, MASS>(row, R, smax);
+}
+
+// Keep every tile at or above the crossing tile, ascending; returns the count.
+template <int VPT>
+__device__ __forceinline__ int write_kept(const Row& row, uint64_t kth, int32_t* out, int kmax) {
+  const float xth = key_to_float((uint32_t)(kth >> 32));  // NaN for ~0: keeps nothing
+  const int jth = (int)(0xffffffffu - (uint32_t)kth);
+  const uint32_t lt = (1u << row.lane) - 1u;
+  int base = 0;
+#pragma unroll 8
+  for (int i = 0; i < VPT; ++i) {
+    const float x = row[i];
+    const int j = row.lane + 32 * i;
+    const bool keep = row.valid(i) && (x > xth || (x == xth && j <= jth));
+    const uint32_t m = __ballot_sync(0xffffffffu, keep);
+    const int pos = base + __popc(m & lt);
+    if (keep && pos < kmax) out[pos] = j;
+    base += __popc(m);
+  }
+  return min(base, kmax);
+}
+
+// Stages one score row into the warp's slice; returns its extent (NaN-free
+// min and max; NaN if the row has no other value).
+template <int VPT>
+__device__ __forceinline__ void stage_row(const float* __restrict__ s, int N, int lane, float* slice, float* lo,
+                                          float* hi) {
+  float mn = __int_as_float(0x7fc00000), mx = mn;
+#pragma unroll 16
+  for (int i = 0; i < VPT; ++i) {
+    const int j = lane + 32 * i;
+    const float x = j < N ? __ldg(s + j) : 0.f;
+    slice[j] = x;
+    if (j < N) {
+      mn = fminf(mn, x);
+      mx = fmaxf(mx, x);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  }
+  *lo = mn;
+  *hi = mx;
+  __syncwarp();
+}
+
+// Rows per CTA: every warp's slice of staged scores and histograms must fit
+// the 48 KB of static shared memory.
+template <int VPT, bool MASS>
+struct Shape {
+  static constexpr int per_warp = 32 * VPT * 4 + kBins * 4 + (MASS ? kBins * 8 : 0) + kCand * 8;
+  static constexpr int warps = (8 * per_warp <= 48 * 1024) ? 8 : 4;
+  static_assert(warps * per_warp <= 48 * 1024, "selection shared memory");
+};
+
+template <int VPT>
+__global__ void __launch_bounds__(32 * Shape<VPT, false>::warps)
+topk_kernel(int rows, int N, int k, const float* __restrict__ S, int32_t* __restrict__ idx,
+            int32_t* __restrict__ cnt, int kmax) {
+  constexpr int W = Shape<VPT, false>::warps;
+  __shared__ float vals_s[W][32 * VPT];
+  __shared__ uint32_t hcnt_s[W][kBins];
+  __shared__ uint64_t cand_s[W][kCand];
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r0 = blockIdx.x * W + w;
+  if (r0 >= rows) return;
+  float lo, hi;
+  stage_row<VPT>(S + (size_t)r0 * N, N, lane, vals_s[w], &lo, &hi);
+  const Row row{&vals_s[w][lane], N, lane};
+  const Hist h{hcnt_s[w], nullptr};
+  const int r = min(k, N);
+  uint64_t kth = ~0ull;  // keeps nothing
+  if (r >= 1) {
+    if (lo < hi) build_hist<VPT, false>(row, true, lo, hi, Binning(lo, hi), 0.0, h);
+    kth = crossing_key<VPT, false>(row, (uint64_t)r, 0.0, lo, hi, h, cand_s[w]);
+  }
+  const int n = write_kept<VPT>(row, kth, idx + (size_t)r0 * kmax, kmax);
+  if (lane == 0) cnt[r0] = n;
+}
+
+// Top-p with a top-k floor: in descending order keep the shortest prefix
+// whose softmax mass reaches p of the row's total, then at least k and at
+// most N tiles.
+template <int VPT>
+__global__ void __launch_bounds__(32 * Shape<VPT, true>::warps)
+topp_kernel(int rows, int N, int k, double p, const float* __restrict__ S, int32_t* __restrict__ idx,
+            int32_t* __restrict__ cnt, int kmax) {
+  constexpr int W = Shape<VPT, true>::warps;
+  __shared__ float vals_s[W][32 * VPT];
+  __shared__ uint32_t hcnt_s[W][kBins];
+  __shared__ uint64_t hwt_s[W][kBins];
+  __shared__ uint64_t cand_s[W][kCand];
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r0 = blockIdx.x * W + w;
+  if (r0 >= rows) return;
+  float lo, hi;
+  stage_row<VPT>(S + (size_t)r0 * N, N, lane, vals_s[w], &lo, &hi);
+  const Row row{&vals_s[w][lane], N, lane};
+  const double smax = (double)hi;
+  const Hist hm{hcnt_s[w], hwt_s[w]};
+  // Level-0 histogram and the total mass in one pass.
+#pragma unroll
+  for (int q = 0; q < kBins / 32; ++q) {
+    hm.cnt[lane + 32 * q] = 0;
+    hm.wt[lane + 32 * q] = 0;
+  }
+  __syncwarp();
+  const Binning bin0(lo, hi);
+  uint64_t local = 0;
+#pragma unroll 4
+  for (int i = 0; i < VPT; ++i) {
+    if (row.valid(i)) {
+      const float x = row[i];
+      const uint64_t q = mass_q(x, smax);
+      const int b = bin0(x);
+      local += q;
+      atomicAdd(&hm.cnt[b], 1u);
+      atomicAdd((unsigned long long*)&hm.wt[b], (unsigned long long)q);
+    }
+  }
+  __syncwarp();
+  const uint64_t total = warp_sum_u64(local);
+  // R = ceil(p * total), clamped to [1, total].
+  const double tgt = ceil(p * (double)total);
+  uint64_t R = tgt >= (double)total ? total : (tgt > 1.0 ? (uint64_t)tgt : 1ull);
+  if (R > total) R = total;
+  // A row without finite mass (an infinite score) keeps only the floor.
+  uint64_t kth_m = ~0ull;
+  int mstar = 0;
+  if (R >= 1) {
+    kth_m = crossing_key<VPT, true>(row, R, smax, lo, hi, hm, cand_s[w]);
+    const float xth = key_to_float((uint32_t)(kth_m >> 32));
+    const int jth = (int)(0xffffffffu - (uint32_t)kth_m);
+    uint32_t nm = 0;
+#pragma unroll 8
+    for (int i = 0; i < VPT; ++i) {
+      const float x = row[i];
+      nm += (row.valid(i) && (x > xth || (x == xth && lane + 32 * i <= jth))) ? 1u : 0u;
+    }
+    mstar = (int)__reduce_add_sync(0xffffffffu, nm);
+  }
+  const int r = min(N, max(mstar, k));
+  uint64_t kth = kth_m;
+  if (r > mstar) {
+    const Hist hc{hcnt_s[w], nullptr};
+    if (lo < hi) build_hist<VPT, false>(row, true, lo, hi, bin0, 0.0, hc);
+    kth = crossing_key<VPT, false>(row, (uint64_t)r, 0.0, lo, hi, hc, cand_s[w]);
+  }
+  const int n = write_kept<VPT>(row, kth, idx + (size_t)r0 * kmax, kmax);
+  if (lane == 0) cnt[r0] = n;
 }
 
 __global__ void broadcast_lists_kernel(int N, int kmax, const int32_t* __restrict__ src_idx,
@@ -212,48 +445,60 @@ __global__ void broadcast_lists_kernel(int N, int kmax, const int32_t* __restric
 }
 
 template <int VPT>
-bsattn_status run_topk(int rows, int N, int k, const float* S, int32_t* idx, int32_t* cnt,
-                       int kmax, cudaStream_t st) {
-  topk_kernel<VPT><<<(rows + 7) / 8, 256, 0, st>>>(rows, N, k, S, idx, cnt, kmax);
+bsattn_status run_topk(int rows, int N, int k, const float* S, int32_t* idx, int32_t* cnt, int kmax,
+                       cudaStream_t st) {
+  constexpr int W = Shape<VPT, false>::warps;
+  topk_kernel<VPT><<<(rows + W - 1) / W, 32 * W, 0, st>>>(rows, N, k, S, idx, cnt, kmax);
   return cudaGetLastError() == cudaSuccess ? BSATTN_OK : BSATTN_ERR_CUDA;
 }
 
-template <int NP>
-bsattn_status run_topp(int rows, int N, int k, double p, const float* S, int32_t* idx,
-                       int32_t* cnt, int kmax, cudaStream_t st) {
-  topp_kernel<NP><<<rows, kTopPThreads, 0, st>>>(N, k, p, S, idx, cnt, kmax);
+template <int VPT>
+bsattn_status run_topp(int rows, int N, int k, double p, const float* S, int32_t* idx, int32_t* cnt, int kmax,
+                       cudaStream_t st) {
+  constexpr int W = Shape<VPT, true>::warps;
+  topp_kernel<VPT><<<(rows + W - 1) / W, 32 * W, 0, st>>>(rows, N, k, p, S, idx, cnt, kmax);
   return cudaGetLastError() == cudaSuccess ? BSATTN_OK : BSATTN_ERR_CUDA;
 }
 
 }  // namespace
 
-bsattn_status launch_select_topk(int rows, int N, int k, const float* S, int32_t* idx,
-                                 int32_t* cnt, int kmax, cudaStream_t st) {
-  int vpt = (N + 31) / 32;
+bsattn_status launch_select_topk(int rows, int N, int k, const float* S, int32_t* idx, int32_t* cnt, int kmax,
+                                 cudaStream_t st) {
+  if (rows <= 0 || N <= 0) return BSATTN_OK;
+  const int vpt = (N + 31) / 32;
   if (vpt <= 1) return run_topk<1>(rows, N, k, S, idx, cnt, kmax, st);
   if (vpt <= 2) return run_topk<2>(rows, N, k, S, idx, cnt, kmax, st);
   if (vpt <= 4) return run_topk<4>(rows, N, k, S, idx, cnt, kmax, st);
   if (vpt <= 8) return run_topk<8>(rows, N, k, S, idx, cnt, kmax, st);
+  if (vpt <= 12) return run_topk<12>(rows, N, k, S, idx, cnt, kmax, st);
   if (vpt <= 16) return run_topk<16>(rows, N, k, S, idx, cnt, kmax, st);
+  if (vpt <= 24) return run_topk<24>(rows, N, k, S, idx, cnt, kmax, st);
   if (vpt <= 32) return run_topk<32>(rows, N, k, S, idx, cnt, kmax, st);
   if (vpt <= 48) return run_topk<48>(rows, N, k, S, idx, cnt, kmax, st);
   if (vpt <= 64) return run_topk<64>(rows, N, k, S, idx, cnt, kmax, st);
   return BSATTN_ERR_UNSUPPORTED;
 }
 
-bsattn_status launch_select_topp(int rows, int N, int k, double p, const float* S, int32_t* idx,
-                                 int32_t* cnt, int kmax, cudaStream_t st) {
-  if (N <= 256) return run_topp<256>(rows, N, k, p, S, idx, cnt, kmax, st);
-  if (N <= 512) return run_topp<512>(rows, N, k, p, S, idx, cnt, kmax, st);
-  if (N <= 1024) return run_topp<1024>(rows, N, k, p, S, idx, cnt, kmax, st);
-  if (N <= 2048) return run_topp<2048>(rows, N, k, p, S, idx, cnt, kmax, st);
+bsattn_status launch_select_topp(int rows, int N, int k, double p, const float* S, int32_t* idx, int32_t* cnt,
+                                 int kmax, cudaStream_t st) {
+  if (rows <= 0 || N <= 0) return BSATTN_OK;
+  const int vpt = (N + 31) / 32;
+  if (vpt <= 1) return run_topp<1>(rows, N, k, p, S, idx, cnt, kmax, st);
+  if (vpt <= 2) return run_topp<2>(rows, N, k, p, S, idx, cnt, kmax, st);
+  if (vpt <= 4) return run_topp<4>(rows, N, k, p, S, idx, cnt, kmax, st);
+  if (vpt <= 8) return run_topp<8>(rows, N, k, p, S, idx, cnt, kmax, st);
+  if (vpt <= 12) return run_topp<12>(rows, N, k, p, S, idx, cnt, kmax, st);
+  if (vpt <= 16) return run_topp<16>(rows, N, k, p, S, idx, cnt, kmax, st);
+  if (vpt <= 24) return run_topp<24>(rows, N, k, p, S, idx, cnt, kmax, st);
+  if (vpt <= 32) return run_topp<32>(rows, N, k, p, S, idx, cnt, kmax, st);
+  if (vpt <= 48) return run_topp<48>(rows, N, k, p, S, idx, cnt, kmax, st);
+  if (vpt <= 64) return run_topp<64>(rows, N, k, p, S, idx, cnt, kmax, st);
   return BSATTN_ERR_UNSUPPORTED;
 }
 
-bsattn_status launch_broadcast_lists(int bh, int N, int kmax, const int32_t* src_idx,
-                                     const int32_t* src_cnt, int32_t* idx, int32_t* cnt,
-                                     cudaStream_t st) {
-  int per = N * kmax;
+bsattn_status launch_broadcast_lists(int bh, int N, int kmax, const int32_t* src_idx, const int32_t* src_cnt,
+                                     int32_t* idx, int32_t* cnt, cudaStream_t st) {
+  const int per = N * kmax;
   dim3 grid((per + 255) / 256 < 64 ? (per + 255) / 256 : 64, bh);
   broadcast_lists_kernel<<<grid, 256, 0, st>>>(N, kmax, src_idx, src_cnt, idx, cnt);
   return cudaGetLastError() == cudaSuccess ? BSATTN_OK : BSATTN_ERR_CUDA;

@@ -44,15 +44,25 @@ def lists_to_device(lists, kmax: int, device="cuda"):
     return torch.from_numpy(idx).to(device), torch.from_numpy(cnt).to(device)
 
 
-def assert_topp_equal(got, S_row, p, k):
-    """GPU top-p list vs the oracle's on the same fp32 row; a count that differs
-    by one is accepted only at an fp64 rounding tie (|c_m - p| < 1e-12)."""
+def assert_topp_equal(got, S_row, p, k, tol=1e-12):
+    """GPU top-p list vs the oracle's on the same fp32 row.
+
+    The prefix masses c_m are rounded on both sides (the oracle in fp64, the
+    kernel in 2^-52 fixed point, < 2.3e-13 for N <= 2048), so any m* whose
+    c_m lies within `tol` of p is a rounding tie: the count may be any
+    min(N, max(m, k)) for m from the first c_m >= p - tol to the first
+    c_m >= p + tol. The kept set must still be that many top-ranked tiles."""
     want_cnt, c = select.topp_count(S_row, p, k)
     order = select.rank_order(S_row)
+    N = S_row.shape[0]
     n = len(got)
     if n != want_cnt:
-        lo = min(n, want_cnt)
-        assert abs(n - want_cnt) == 1 and lo >= k and abs(c[lo - 1] - p) < 1e-12, (n, want_cnt)
+        lo_hit = np.nonzero(c >= p - tol)[0]
+        hi_hit = np.nonzero(c >= p + tol)[0]
+        lo = int(lo_hit[0]) + 1 if lo_hit.size else N
+        hi = int(hi_hit[0]) + 1 if hi_hit.size else N
+        allowed = {min(N, max(m, k)) for m in range(lo, hi + 1)}
+        assert n in allowed, (n, want_cnt, sorted(allowed)[:4])
     np.testing.assert_array_equal(np.asarray(got), np.sort(order[:n]))
 
 

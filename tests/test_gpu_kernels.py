@@ -95,6 +95,43 @@ def test_select_topp_bit_exact(bs, N, k, p, sharp):
         assert_topp_equal(got[r], Sn[r], p, k)
 
 
+def _degenerate_rows(N, seed):
+    """Rows that defeat value binning: ties, outliers, ulp clusters, denormals."""
+    rng = np.random.default_rng(seed)
+    base = rng.standard_normal(N).astype(np.float32)
+    rows = [np.full(N, 0.5, np.float32),                                   # one value
+            np.where(rng.random(N) < 0.5, 0.0, -0.0).astype(np.float32),   # +0 / -0
+            np.where(rng.random(N) < 0.5, 1.0, 2.0).astype(np.float32),    # two values
+            np.where(np.arange(N) == N // 3, 1e30, base).astype(np.float32),
+            np.where(np.arange(N) == N // 2, -1e30, base).astype(np.float32),
+            (base * 1e-42).astype(np.float32),                              # denormals
+            1.0 + rng.integers(0, 40, N).astype(np.float32) * np.finfo(np.float32).eps,  # ulps
+            np.where(rng.random(N) < 0.1, -np.inf, base).astype(np.float32),
+            np.round(base, 1).astype(np.float32),                           # many ties
+            np.where(np.arange(N) < N // 4, base.max(), base).astype(np.float32)]
+    return np.stack([r.astype(np.float32) for r in rows])
+
+
+@pytest.mark.parametrize("N", [37, 300, 1440, 2048])
+@pytest.mark.parametrize("rule", ["topk", "topp"])
+def test_select_degenerate_rows(bs, N, rule):
+    S = _degenerate_rows(N, seed=N)
+    rows = S.shape[0]
+    k = max(1, N // 10)
+    pad = np.tile(S, (N // rows + 1, 1))[:N]  # one head: N rows
+    plan = bs.Plan(1, 1, 64, 4, 4, 4 * N, rule=rule, k=k, p=0.9)
+    si, sc = plan.list_shapes()
+    idx = torch.empty(si, dtype=torch.int32, device="cuda")
+    cnt = torch.empty(sc, dtype=torch.int32, device="cuda")
+    bs.attn_select_from_scores(plan, torch.from_numpy(pad).view(1, 1, N, N).cuda(), idx, cnt)
+    got = lists_from_device(idx, cnt)
+    for r in range(N):
+        if rule == "topk":
+            np.testing.assert_array_equal(got[r], select.topk_row(pad[r], k))
+        else:
+            assert_topp_equal(got[r], pad[r], 0.9, k)
+
+
 @pytest.mark.parametrize("name", ["ragged_window_fp8", "ragged_bf16_window"])
 def test_window_lists(bs, name):
     wl = SMALL[name]
