@@ -83,18 +83,23 @@ __device__ __forceinline__ uint64_t weight_of(float x, double smax) {
     return 1ull;
 }
 
-// Equal-width binning of the range [lo, hi] (lo < hi): one rounding of
-// x * sc + off, so monotone in x; the clamp absorbs rounding at the edges and
-// saturated or NaN conversions (a range that overflows puts every tile in bin
-// 0, and the search moves on to the bitwise step).
+// Equal-width binning of the range [lo, hi] (lo < hi) without a float-to-int
+// conversion: one FMA computes x * sc - lo * sc + 1.5 * 2^23, whose rounding
+// to float leaves the bin as an integer in the low mantissa bits once the
+// value is clamped to [1.5 * 2^23, 1.5 * 2^23 + 255] (that span has unit
+// spacing). Every step is monotone in x, so bins keep the score order; NaN and
+// a range that overflows land in bin 0 (the search then moves on to the
+// bitwise step).
 struct Binning {
-  float sc, off;
+  static constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+  float sc, offm;
   __device__ __forceinline__ Binning(float lo, float hi) {
     sc = (float)kBins / (hi - lo);
-    off = -lo * sc;
+    offm = fmaf(-lo, sc, kMagic);
   }
   __device__ __forceinline__ int operator()(float x) const {
-    return min(max(__float2int_rz(fmaf(x, sc, off)), 0), kBins - 1);
+    const float t = fminf(fmaxf(fmaf(x, sc, offm), kMagic), kMagic + (float)(kBins - 1));
+    return __float_as_int(t) - __float_as_int(kMagic);
   }
 };
 
@@ -301,22 +306,16 @@ __device__ __forceinline__ int write_kept(const Row& row, uint64_t kth, int32_t*
   return min(base, kmax);
 }
 
-// Stages one score row into the warp's slice; returns its extent (NaN-free
-// min and max; NaN if the row has no other value).
+// NaN-free min and max of the staged row (NaN if it has no other value).
 template <int VPT>
-__device__ __forceinline__ void stage_row(const float* __restrict__ s, int N, int lane, float* slice, float* lo,
-                                          float* hi) {
+__device__ __forceinline__ void row_extent(const Row& row, float* lo, float* hi) {
   float mn = __int_as_float(0x7fc00000), mx = mn;
-#pragma unroll 16
-  for (int i = 0; i < VPT; ++i) {
-    const int j = lane + 32 * i;
-    const float x = j < N ? __ldg(s + j) : 0.f;
-    slice[j] = x;
-    if (j < N) {
-      mn = fminf(mn, x);
-      mx = fmaxf(mx, x);
+#pragma unroll 8
+  for (int i = 0; i < VPT; ++i)
+    if (row.valid(i)) {
+      mn = fminf(mn, row[i]);
+      mx = fmaxf(mx, row[i]);
     }
-  }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
@@ -324,14 +323,98 @@ __device__ __forceinline__ void stage_row(const float* __restrict__ s, int N, in
   }
   *lo = mn;
   *hi = mx;
+}
+
+// One pass over the staged row against bin b: mask[i] gets the 32-tile word
+// of chunk i's tiles in bins above b, and the tiles of bin b go to cand (the
+// first kCand of them) as composite keys. Returns the number of bin-b tiles.
+__device__ __forceinline__ int mask_and_gather(const Row& row, const Binning& bin, int b, uint32_t* mask,
+                                               uint64_t* cand) {
+  const uint32_t lt = (1u << row.lane) - 1u;
+  const int nfull = row.N >> 5, nchunk = (row.N + 31) >> 5;
+  int base = 0;
+  auto chunk = [&](int i, bool valid) {
+    const float x = row[i];
+    const int bx = bin(x);
+    const uint32_t ma = __ballot_sync(0xffffffffu, valid && bx > b);
+    const uint32_t me = __ballot_sync(0xffffffffu, valid && bx == b);
+    if (row.lane == 0) mask[i] = ma;
+    if (me) {
+      const int pos = base + __popc(me & lt);
+      if (((me >> row.lane) & 1u) && pos < kCand) cand[pos] = comp_key(x, row.lane + 32 * i);
+      base += __popc(me);
+    }
+  };
+#pragma unroll 4
+  for (int i = 0; i < nfull; ++i) chunk(i, true);
+  if (nchunk > nfull) chunk(nfull, row.valid(nfull));
+  __syncwarp();
+  return base;
+}
+
+// Sorts the warp's candidates (one composite key per lane, 0 for none)
+// descending.
+__device__ __forceinline__ uint64_t sort_desc32(uint64_t ck, int lane) {
+#pragma unroll
+  for (int size = 2; size <= 32; size <<= 1)
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      const uint64_t ok = shfl_xor_u64(ck, stride);
+      const bool take_max = ((lane & stride) == 0) == ((lane & size) == 0);
+      if (take_max ? ok > ck : ok < ck) ck = ok;
+    }
+  return ck;
+}
+
+// Writes the tiles whose mask bit is set, ascending, and returns how many
+// were written (at most kmax). Lane l owns the words [l*WPL, (l+1)*WPL).
+template <int VPT>
+__device__ __forceinline__ int compact_mask(const uint32_t* mask, int N, int lane, int32_t* out, int kmax) {
+  constexpr int WPL = (VPT + 31) / 32;
+  const int nchunk = (N + 31) >> 5;
+  uint32_t wv[WPL];
+  int c = 0;
+#pragma unroll
+  for (int t = 0; t < WPL; ++t) {
+    const int wi = lane * WPL + t;
+    wv[t] = wi < nchunk ? mask[wi] : 0u;
+    c += __popc(wv[t]);
+  }
+  int x = c;  // inclusive prefix over lanes
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  const int total = __shfl_sync(0xffffffffu, x, 31);
+  int pos = x - c;
+#pragma unroll
+  for (int t = 0; t < WPL; ++t) {
+    uint32_t m = wv[t];
+    const int jb = 32 * (lane * WPL + t);
+    while (m) {
+      if (pos < kmax) out[pos] = jb + __ffs(m) - 1;
+      ++pos;
+      m &= m - 1;
+    }
+  }
+  return min(total, kmax);
+}
+
+// Marks the first `keep` sorted candidates in the mask.
+__device__ __forceinline__ void mark_kept(uint64_t ck, int lane, int keep, uint32_t* mask) {
+  if (lane < keep && ck) {
+    const uint32_t j = 0xffffffffu - (uint32_t)ck;
+    atomicOr(&mask[j >> 5], 1u << (j & 31));
+  }
   __syncwarp();
 }
 
-// Rows per CTA: every warp's slice of staged scores and histograms must fit
-// the 48 KB of static shared memory.
+// Rows per CTA: every warp's slice of staged scores, histograms and masks
+// must fit the 48 KB of static shared memory.
 template <int VPT, bool MASS>
 struct Shape {
-  static constexpr int per_warp = 32 * VPT * 4 + kBins * 4 + (MASS ? kBins * 8 : 0) + kCand * 8;
+  static constexpr int per_warp = 32 * VPT * 4 + VPT * 4 + kBins * 4 + (MASS ? kBins * 8 : 0) + kCand * 8;
   static constexpr int warps = (8 * per_warp <= 48 * 1024) ? 8 : 4;
   static_assert(warps * per_warp <= 48 * 1024, "selection shared memory");
 };
@@ -343,21 +426,75 @@ topk_kernel(int rows, int N, int k, const float* __restrict__ S, int32_t* __rest
   constexpr int W = Shape<VPT, false>::warps;
   __shared__ float vals_s[W][32 * VPT];
   __shared__ uint32_t hcnt_s[W][kBins];
+  __shared__ uint32_t mask_s[W][VPT];
   __shared__ uint64_t cand_s[W][kCand];
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r0 = blockIdx.x * W + w;
   if (r0 >= rows) return;
-  float lo, hi;
-  stage_row<VPT>(S + (size_t)r0 * N, N, lane, vals_s[w], &lo, &hi);
-  const Row row{&vals_s[w][lane], N, lane};
-  const Hist h{hcnt_s[w], nullptr};
-  const int r = min(k, N);
-  uint64_t kth = ~0ull;  // keeps nothing
-  if (r >= 1) {
-    if (lo < hi) build_hist<VPT, false>(row, true, lo, hi, Binning(lo, hi), 0.0, h);
-    kth = crossing_key<VPT, false>(row, (uint64_t)r, 0.0, lo, hi, h, cand_s[w]);
+  const float* s = S + (size_t)r0 * N;
+  float* slice = vals_s[w];
+  uint32_t* hist = hcnt_s[w];
+  const Row row{&slice[lane], N, lane};
+
+  // Pass 1: load the whole row into registers (all loads in flight at once),
+  // stage it, histogram it. The bins span the extent of an evenly strided
+  // sample of chunks; tiles outside it fall into the edge bins (binning stays
+  // monotone).
+  constexpr int B0 = VPT < 8 ? VPT : 8;
+  constexpr int STEP = VPT / B0;
+  float v[VPT];
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    const int j = lane + 32 * i;
+    v[i] = j < N ? __ldg(s + j) : __int_as_float(0x7fc00000);
   }
-  const int n = write_kept<VPT>(row, kth, idx + (size_t)r0 * kmax, kmax);
+  float mn = v[0], mx = v[0];
+#pragma unroll
+  for (int t = 1; t < B0; ++t) {
+    mn = fminf(mn, v[t * STEP]);
+    mx = fmaxf(mx, v[t * STEP]);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  }
+  const bool spread = mn < mx;
+  const Binning bin(spread ? mn : 0.f, spread ? mx : 1.f);
+#pragma unroll
+  for (int q = 0; q < kBins / 32; ++q) hist[lane + 32 * q] = 0;
+  __syncwarp();
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    const int j = lane + 32 * i;
+    if (j < N) {
+      slice[j] = v[i];
+      atomicAdd(&hist[bin(v[i])], 1u);
+    }
+  }
+  __syncwarp();
+
+  const int r = min(k, N);
+  int32_t* out = idx + (size_t)r0 * kmax;
+  int n = 0;
+  uint64_t above = 0;
+  const int b = (spread && r >= 1) ? find_bin<false>(Hist{hist, nullptr}, (uint64_t)r, lane, &above) : -1;
+  if (b >= 0 && hist[b] <= (uint32_t)kCand) {
+    // Pass 2: bins above b are kept whole; rank bin b's tiles exactly.
+    const int nb = mask_and_gather(row, bin, b, mask_s[w], cand_s[w]);
+    const uint64_t ck = sort_desc32(lane < nb ? cand_s[w][lane] : 0ull, lane);
+    mark_kept(ck, lane, r - (int)above, mask_s[w]);
+    n = compact_mask<VPT>(mask_s[w], N, lane, out, kmax);
+  } else if (r >= 1) {
+    // General search over the exact extent.
+    float lo, hi;
+    row_extent<VPT>(row, &lo, &hi);
+    const Hist h{hist, nullptr};
+    __syncwarp();
+    if (lo < hi) build_hist<VPT, false>(row, true, lo, hi, Binning(lo, hi), 0.0, h);
+    const uint64_t kth = crossing_key<VPT, false>(row, (uint64_t)r, 0.0, lo, hi, h, cand_s[w]);
+    n = write_kept<VPT>(row, kth, out, kmax);
+  }
   if (lane == 0) cnt[r0] = n;
 }
 
@@ -372,23 +509,45 @@ topp_kernel(int rows, int N, int k, double p, const float* __restrict__ S, int32
   __shared__ float vals_s[W][32 * VPT];
   __shared__ uint32_t hcnt_s[W][kBins];
   __shared__ uint64_t hwt_s[W][kBins];
+  __shared__ uint32_t mask_s[W][VPT];
   __shared__ uint64_t cand_s[W][kCand];
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r0 = blockIdx.x * W + w;
   if (r0 >= rows) return;
-  float lo, hi;
-  stage_row<VPT>(S + (size_t)r0 * N, N, lane, vals_s[w], &lo, &hi);
-  const Row row{&vals_s[w][lane], N, lane};
+  const float* s = S + (size_t)r0 * N;
+  float* slice = vals_s[w];
+  const Row row{&slice[lane], N, lane};
+  // Pass 1: stage the row; the exact max is needed before any mass.
+  float v[VPT];
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    const int j = lane + 32 * i;
+    v[i] = j < N ? __ldg(s + j) : __int_as_float(0x7fc00000);
+  }
+  float lo = v[0], hi = v[0];
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    const int j = lane + 32 * i;
+    lo = fminf(lo, v[i]);
+    hi = fmaxf(hi, v[i]);
+    if (j < N) slice[j] = v[i];
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+  }
   const double smax = (double)hi;
   const Hist hm{hcnt_s[w], hwt_s[w]};
-  // Level-0 histogram and the total mass in one pass.
+  const bool spread = lo < hi;
+  const Binning bin0(spread ? lo : 0.f, spread ? hi : 1.f);
+  // Pass 2: count and mass histograms and the total mass.
 #pragma unroll
   for (int q = 0; q < kBins / 32; ++q) {
     hm.cnt[lane + 32 * q] = 0;
     hm.wt[lane + 32 * q] = 0;
   }
   __syncwarp();
-  const Binning bin0(lo, hi);
   uint64_t local = 0;
 #pragma unroll 4
   for (int i = 0; i < VPT; ++i) {
@@ -403,33 +562,72 @@ topp_kernel(int rows, int N, int k, double p, const float* __restrict__ S, int32
   }
   __syncwarp();
   const uint64_t total = warp_sum_u64(local);
-  // R = ceil(p * total), clamped to [1, total].
+  // R = ceil(p * total), clamped to [1, total]; a row without finite mass
+  // (an infinite score) has total 0 and keeps only the floor.
   const double tgt = ceil(p * (double)total);
   uint64_t R = tgt >= (double)total ? total : (tgt > 1.0 ? (uint64_t)tgt : 1ull);
   if (R > total) R = total;
-  // A row without finite mass (an infinite score) keeps only the floor.
-  uint64_t kth_m = ~0ull;
-  int mstar = 0;
-  if (R >= 1) {
-    kth_m = crossing_key<VPT, true>(row, R, smax, lo, hi, hm, cand_s[w]);
-    const float xth = key_to_float((uint32_t)(kth_m >> 32));
-    const int jth = (int)(0xffffffffu - (uint32_t)kth_m);
-    uint32_t nm = 0;
-#pragma unroll 8
-    for (int i = 0; i < VPT; ++i) {
-      const float x = row[i];
-      nm += (row.valid(i) && (x > xth || (x == xth && lane + 32 * i <= jth))) ? 1u : 0u;
+  int32_t* out = idx + (size_t)r0 * kmax;
+  int n = -1;
+  uint64_t A = 0;
+  const int b = (spread && R >= 1) ? find_bin<true>(hm, R, lane, &A) : -1;
+  if (b >= 0 && hm.cnt[b] <= (uint32_t)kCand) {
+    // Pass 3: bins above b are kept whole; bin b's tiles in order decide m*.
+    int cab = 0;  // tiles in bins above b
+#pragma unroll
+    for (int q = 0; q < kBins / 32; ++q) {
+      const int bb = lane + 32 * q;
+      cab += bb > b ? (int)hm.cnt[bb] : 0;
     }
-    mstar = (int)__reduce_add_sync(0xffffffffu, nm);
+    cab = (int)__reduce_add_sync(0xffffffffu, (uint32_t)cab);
+    const int nb = mask_and_gather(row, bin0, b, mask_s[w], cand_s[w]);
+    const uint64_t ck = sort_desc32(lane < nb ? cand_s[w][lane] : 0ull, lane);
+    uint64_t c = ck ? mass_q(key_to_float((uint32_t)(ck >> 32)), smax) : 0ull;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint64_t y = shfl_up_u64(c, o);
+      if (lane >= o) c += y;
+    }
+    const uint32_t hit = __ballot_sync(0xffffffffu, ck != 0 && A + c >= R);
+    if (hit) {
+      const int mstar = cab + __ffs(hit);
+      const int r = min(N, max(mstar, k));
+      if (r - cab <= nb) {
+        mark_kept(ck, lane, r - cab, mask_s[w]);
+        n = compact_mask<VPT>(mask_s[w], N, lane, out, kmax);
+      } else {
+        // The floor reaches past bin b: count search for rank r.
+        const uint64_t kth = crossing_key<VPT, false>(row, (uint64_t)r, 0.0, lo, hi, Hist{hm.cnt, nullptr},
+                                                      cand_s[w]);
+        n = write_kept<VPT>(row, kth, out, kmax);
+      }
+    }
   }
-  const int r = min(N, max(mstar, k));
-  uint64_t kth = kth_m;
-  if (r > mstar) {
-    const Hist hc{hcnt_s[w], nullptr};
-    if (lo < hi) build_hist<VPT, false>(row, true, lo, hi, bin0, 0.0, hc);
-    kth = crossing_key<VPT, false>(row, (uint64_t)r, 0.0, lo, hi, hc, cand_s[w]);
+  if (n < 0) {
+    // General search over the exact extent.
+    uint64_t kth_m = ~0ull;
+    int mstar = 0;
+    if (R >= 1) {
+      kth_m = crossing_key<VPT, true>(row, R, smax, lo, hi, hm, cand_s[w]);
+      const float xth = key_to_float((uint32_t)(kth_m >> 32));
+      const int jth = (int)(0xffffffffu - (uint32_t)kth_m);
+      uint32_t nm = 0;
+#pragma unroll 8
+      for (int i = 0; i < VPT; ++i) {
+        const float x = row[i];
+        nm += (row.valid(i) && (x > xth || (x == xth && lane + 32 * i <= jth))) ? 1u : 0u;
+      }
+      mstar = (int)__reduce_add_sync(0xffffffffu, nm);
+    }
+    const int r = min(N, max(mstar, k));
+    uint64_t kth = kth_m;
+    if (r > mstar) {
+      const Hist hc{hcnt_s[w], nullptr};
+      if (lo < hi) build_hist<VPT, false>(row, true, lo, hi, bin0, 0.0, hc);
+      kth = crossing_key<VPT, false>(row, (uint64_t)r, 0.0, lo, hi, hc, cand_s[w]);
+    }
+    n = write_kept<VPT>(row, kth, out, kmax);
   }
-  const int n = write_kept<VPT>(row, kth, idx + (size_t)r0 * kmax, kmax);
   if (lane == 0) cnt[r0] = n;
 }
 
