@@ -392,7 +392,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         const float c = P.scale_log2 * (FP8 ? qsc * __ldg(P.ks + bh * g.N + j) : 1.f);
         const int bt = j / (g.nH * g.nW), bhh = (j / g.nW) % g.nH, bw = j % g.nW;
         const int vt = g.T - bt * g.tt, vh = g.H - bhh * g.th, vw = g.W - bw * g.tw;
-        if (vt < g.tt || vh < g.th || vw < g.tw) {  // padded keys of an edge tile
+        const bool edge = vt < g.tt || vh < g.th || vw < g.tw;
+        if (edge) {  // padded keys of an edge tile
 #pragma unroll
           for (int q = 0; q < 64; ++q) {
             const uint32_t cc = colc[q];
@@ -400,15 +401,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
               sr[q] = 0xff800000u;  // -inf
           }
         }
-        // Row max of the raw scores: eight independent chains. c > 0, so the
-        // max of the scaled logits is c times the raw max.
-        float mx8[8];
+        // Row max of the raw scores: three-input max, four chains. c > 0, so
+        // the max of the scaled logits is c times the raw max.
+        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int a = 0; a < 8; ++a) mx8[a] = __uint_as_float(sr[a]);
-#pragma unroll
-        for (int q = 8; q < 64; ++q) mx8[q & 7] = fmaxf(mx8[q & 7], __uint_as_float(sr[q]));
-        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * c;
+        for (int q = 0; q < 32; ++q)
+          mx4[q & 3] = tc::fmax3(mx4[q & 3], __uint_as_float(sr[2 * q]), __uint_as_float(sr[2 * q + 1]));
+        const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * c;
         const float m_new = fmaxf(m, mx);
         if (m == -INFINITY) {
           m = m_new;  // first kept tile of this row: O row is still zero
@@ -418,17 +417,34 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           l *= alpha;
           need = true;
         }
-        // p = 2^(s*c - m); the row sum uses the fp32 values, eight chains.
-        float ls8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int q = 0; q < 32; ++q) {
-          const float p0 = tc::ex2(fmaf(__uint_as_float(sr[2 * q]), c, -m));
-          const float p1 = tc::ex2(fmaf(__uint_as_float(sr[2 * q + 1]), c, -m));
-          ls8[q & 7] += p0 + p1;
-          __nv_bfloat162 hv = __floats2bfloat162_rn(p0, p1);
+        // p = 2^(s*c - m) on packed pairs. A quarter of the pairs of a full
+        // tile take the FMA-pipe exponential so that the SFU, shared by both
+        // CTAs' softmax warps, is not the bottleneck; edge tiles (with -inf
+        // for padded keys) use the SFU throughout. The row sum uses the fp32
+        // values, four packed chains.
+        const float2 c2 = make_float2(c, c), nm2 = make_float2(-m, -m);
+        float2 ls2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                         make_float2(0.f, 0.f)};
+        auto emit = [&](int q, float2 pv) {
+          ls2[q & 3] = __fadd2_rn(ls2[q & 3], pv);
+          __nv_bfloat162 hv = __floats2bfloat162_rn(pv.x, pv.y);
           pk[q] = *reinterpret_cast<uint32_t*>(&hv);
+        };
+        if (edge) {
+#pragma unroll
+          for (int q = 0; q < 32; ++q) {
+            const float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[2 * q]), __uint_as_float(sr[2 * q + 1])), c2, nm2);
+            emit(q, make_float2(tc::ex2(x.x), tc::ex2(x.y)));
+          }
+        } else {
+#pragma unroll
+          for (int q = 0; q < 32; ++q) {
+            const float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[2 * q]), __uint_as_float(sr[2 * q + 1])), c2, nm2);
+            emit(q, (q & 3) == 3 ? tc::ex2_poly2(x) : make_float2(tc::ex2(x.x), tc::ex2(x.y)));
+          }
         }
-        l += ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
+        const float2 lsa = __fadd2_rn(__fadd2_rn(ls2[0], ls2[1]), __fadd2_rn(ls2[2], ls2[3]));
+        l += lsa.x + lsa.y;
       } else {
 #pragma unroll
         for (int q = 0; q < 32; ++q) pk[q] = 0u;

@@ -163,6 +163,36 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// Three-input fp32 max (NaN inputs are ignored, like fmaxf).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^x for two values on the FMA pipe, leaving the SFU to other work. With
+// x = n + f, n = round(x) and f in [-1/2, 1/2]: 2^f comes from a cubic whose
+// coefficients were fitted to 2^f on [-1/2, 1/2] for minimum maximum relative
+// error (Lawson's iteratively reweighted least squares; 1.5e-4), and n is
+// added to the exponent field. Adding 1.5 * 2^23 rounds x to an integer in
+// the low mantissa bits, which also supplies n << 23. x is clamped below at
+// -125 so the result stays a normal number (2^-125 stands in for anything
+// smaller); valid for x <= 127.
+__device__ __forceinline__ float2 ex2_poly2(float2 x) {
+  constexpr float kM = 12582912.0f;  // 1.5 * 2^23
+  constexpr float c0 = 0.99992824f, c1 = 0.69326097f, c2 = 0.24260852f, c3 = 0.05517050f;
+  x.x = fmaxf(x.x, -125.f);
+  x.y = fmaxf(x.y, -125.f);
+  const float2 t = __fadd2_rn(x, make_float2(kM, kM));
+  const float2 n = __fadd2_rn(t, make_float2(-kM, -kM));
+  const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);
+  float2 p = __ffma2_rn(make_float2(c3, c3), f, make_float2(c2, c2));
+  p = __ffma2_rn(p, f, make_float2(c1, c1));
+  p = __ffma2_rn(p, f, make_float2(c0, c0));
+  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
+}
+
 // ---------------------------------------------------------------- descriptors
 enum : uint32_t { kLayoutSW128 = 2, kLayoutSW64 = 4 };
 
