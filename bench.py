@@ -1,8 +1,9 @@
 """Benchmark of the block-sparse attention layer on one or more B200s.
 
-A step is one whole layer through the C ABI (attn_layer): tile reorder with
-fused pooling (and e4m3 quantisation on the FP8 workload), block scores,
-key-tile selection, block-sparse attention, unreorder. Inputs are seeded
+A step is one whole layer through the C ABI (attn_layer): tile pooling of Q
+and K (e4m3 tile codes with fused pooling on the FP8 workload), block
+scores, key-tile selection, and the block-sparse attention, which reads Q, K,
+V tile by tile from the natural layout and writes natural O. Inputs are seeded
 synthetic video-latent Q/K/V already resident in HBM; L2 is flushed between
 timed steps. Prints one JSON line (rank 0).
 
@@ -127,7 +128,8 @@ def group_accounting(wl, plan, idx: torch.Tensor, cnt: torch.Tensor):
 
 def launches_per_step(wl) -> int:
     pooled = wl.rule != "window"
-    return 3 + (2 if pooled else 1) + 2  # reorder x3, [scores], select, attention, unreorder
+    quant = 2 if wl.qk_fp8 else 0  # e4m3 tile codes of Q and K
+    return quant + (2 if pooled else 0) + 1 + 1  # [pool Q+K, scores], select, attention
 
 
 class ClockSampler:
@@ -405,8 +407,11 @@ def main():
 
 
 def component_timing(bsattn, plan, wl, q, k, v, flush, stream, reps=20):
-    """Average device time of each step of the layer, launched one by one."""
-    tiled = [torch.empty(plan.tiled_shape(), dtype=torch.bfloat16, device="cuda") for _ in range(3)]
+    """Average device time of each step of the layer, launched one by one.
+
+    The layer pools Q and K (bf16) or turns them into e4m3 tile codes, scores,
+    selects, and runs the attention on the natural tensors; "attention_tiled"
+    is the same attention on pre-tiled inputs, for comparison."""
     pq = torch.empty((wl.B, wl.heads, plan.N, wl.head_dim), dtype=torch.float32, device="cuda")
     pk = torch.empty_like(pq)
     S = torch.empty((wl.B, wl.heads, plan.N, plan.N), dtype=torch.float32, device="cuda") \
@@ -414,14 +419,17 @@ def component_timing(bsattn, plan, wl, q, k, v, flush, stream, reps=20):
     si, sc = plan.list_shapes()
     idx = torch.empty(si, dtype=torch.int32, device="cuda")
     cnt = torch.empty(sc, dtype=torch.int32, device="cuda")
+    tiled = [torch.empty(plan.tiled_shape(), dtype=torch.bfloat16, device="cuda") for _ in range(3)]
+    for x, t in zip((q, k, v), tiled):
+        bsattn.attn_reorder(plan, x, t, None, stream)
     o_t = torch.empty(plan.tiled_shape(), dtype=torch.bfloat16, device="cuda")
     o = torch.empty_like(q)
     if wl.qk_fp8:
         codes = [torch.empty(plan.tiled_shape(), dtype=torch.uint8, device="cuda") for _ in range(2)]
         scales = [torch.empty((wl.B, wl.heads, plan.N), dtype=torch.float32, device="cuda")
                   for _ in range(2)]
-    names = ["reorder_qk", "reorder_v", "block_scores", "select", "quantize", "attention",
-             "unreorder"]
+    names = ["pool_qk", "reorder_qk", "quantize", "block_scores", "select", "attention",
+             "attention_tiled"]
     acc = {n: 0.0 for n in names}
 
     def timed(name, fn):
@@ -435,24 +443,30 @@ def component_timing(bsattn, plan, wl, q, k, v, flush, stream, reps=20):
         marks = []
         flush.fill_(1.0)
         pooled = wl.rule != "window"
-        marks.append(timed("reorder_qk", lambda: (
-            bsattn.attn_reorder(plan, q, tiled[0], pq if pooled else None, stream),
-            bsattn.attn_reorder(plan, k, tiled[1], pk if pooled else None, stream))))
-        marks.append(timed("reorder_v", lambda: bsattn.attn_reorder(plan, v, tiled[2], None, stream)))
-        if pooled:
-            marks.append(timed("block_scores", lambda: bsattn.attn_block_scores(plan, pq, pk, S, stream)))
-        marks.append(timed("select", lambda: bsattn.attn_select_from_scores(plan, S, idx, cnt, stream)))
         if wl.qk_fp8:
+            marks.append(timed("reorder_qk", lambda: (
+                bsattn.attn_reorder(plan, q, tiled[0], pq if pooled else None, stream),
+                bsattn.attn_reorder(plan, k, tiled[1], pk if pooled else None, stream))))
             marks.append(timed("quantize", lambda: (
                 bsattn.attn_quantize_e4m3(plan, tiled[0], codes[0], scales[0], stream),
                 bsattn.attn_quantize_e4m3(plan, tiled[1], codes[1], scales[1], stream))))
             qa, ka, qs, ks = codes[0], codes[1], scales[0], scales[1]
+            qn, kn = qa, ka
         else:
+            if pooled:
+                marks.append(timed("pool_qk", lambda: (bsattn.attn_pool(plan, q, pq, stream),
+                                                       bsattn.attn_pool(plan, k, pk, stream))))
             qa, ka, qs, ks = tiled[0], tiled[1], None, None
+            qn, kn = q, k
+        if pooled:
+            marks.append(timed("block_scores", lambda: bsattn.attn_block_scores(plan, pq, pk, S, stream)))
+        marks.append(timed("select", lambda: bsattn.attn_select_from_scores(plan, S, idx, cnt, stream)))
         flush.fill_(2.0)
-        marks.append(timed("attention", lambda: bsattn.attn_forward(
+        marks.append(timed("attention", lambda: bsattn.attn_forward_natural(
+            plan, qn, kn, v, idx, cnt, o, q_scale=qs, k_scale=ks, stream=stream)))
+        flush.fill_(3.0)
+        marks.append(timed("attention_tiled", lambda: bsattn.attn_forward(
             plan, qa, ka, tiled[2], idx, cnt, o_t, q_scale=qs, k_scale=ks, stream=stream)))
-        marks.append(timed("unreorder", lambda: bsattn.attn_unreorder(plan, o_t, o, stream)))
         torch.cuda.synchronize()
         if r >= 2:
             for n, a, b in marks:
@@ -467,17 +481,15 @@ def memory_kernel_rates(wl, plan, comp, pk):
     til = bh * plan.N * 64 * wl.head_dim * 2
     pooled = bh * plan.N * wl.head_dim * 4
     out = {}
+    if "pool_qk" in comp:
+        out["pool_qk"] = (2 * nat + 2 * pooled) / (comp["pool_qk"] * 1e-3) / 1e9
     if "reorder_qk" in comp:
         b = 2 * (nat + til) + (2 * pooled if wl.rule != "window" else 0)
         out["reorder_qk"] = b / (comp["reorder_qk"] * 1e-3) / 1e9
-    if "reorder_v" in comp:
-        out["reorder_v"] = (nat + til) / (comp["reorder_v"] * 1e-3) / 1e9
     if "select" in comp and wl.rule != "window":
         rows = bh * plan.N
         b = rows * plan.N * 4 + rows * 4 + rows * (wl.k if wl.rule == "topk" else plan.N / 4) * 4
         out["select"] = b / (comp["select"] * 1e-3) / 1e9
-    if "unreorder" in comp:
-        out["unreorder"] = (nat + til) / (comp["unreorder"] * 1e-3) / 1e9
     res = {n: {"GB/s": round(x, 1), "frac": round(x / pk["hbm_gbs"], 3)} for n, x in out.items()}
     res["peak_GBs"] = pk["hbm_gbs"]
     res["note"] = "algorithmic bytes / kernel time; of " + pk["source"] + " HBM copy bandwidth"

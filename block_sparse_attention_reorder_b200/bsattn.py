@@ -74,6 +74,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "attn_select_static": [P, P, P, P, P, P],
         "attn_quantize_e4m3": [P, P, P, P, P],
         "attn_forward": [P, P, P, P, P, P, P, P, P, P, P, Z, P],
+        "attn_forward_natural": [P, P, P, P, P, P, P, P, P, P, P, Z, P],
         "attn_layer": [P, P, P, P, P, P, P, P, P, Z, P],
         "attn_check_device_status": [P, P],
     }
@@ -89,7 +90,7 @@ _lib = load_library()
 EXPORTED = ("attn_plan_create", "attn_plan_destroy", "attn_plan_info", "attn_status_string",
             "attn_reorder", "attn_pool", "attn_unreorder", "attn_block_scores",
             "attn_select_from_scores", "attn_select", "attn_select_static", "attn_quantize_e4m3",
-            "attn_forward",
+            "attn_forward", "attn_forward_natural",
             "attn_layer", "attn_check_device_status")
 
 
@@ -267,6 +268,27 @@ def attn_forward(plan: Plan, q, k, v, idx, cnt, o_tiled, lse=None, q_scale=None,
     _check(_lib.attn_forward(plan.handle, _ptr(q), _ptr(k), _ptr(q_scale), _ptr(k_scale), _ptr(v),
                              _ptr(idx), _ptr(cnt), _ptr(o_tiled), _ptr(lse), _ptr(ws), wsb,
                              _stream(stream)), "attn_forward")
+
+
+def attn_forward_natural(plan: Plan, q, k, v_nat, idx, cnt, o_nat, lse_nat=None, q_scale=None,
+                         k_scale=None, ws=None, stream=None):
+    if plan.qk_fp8:
+        _want(q, torch.uint8, plan.tiled_shape(), "q")
+        _want(k, torch.uint8, plan.tiled_shape(), "k")
+    else:
+        _want(q, torch.bfloat16, plan.natural_shape(), "q")
+        _want(k, torch.bfloat16, plan.natural_shape(), "k")
+    _want(v_nat, torch.bfloat16, plan.natural_shape(), "v_nat")
+    _want(o_nat, torch.bfloat16, plan.natural_shape(), "o_nat")
+    si, sc = plan.list_shapes()
+    _want(idx, torch.int32, si, "idx")
+    _want(cnt, torch.int32, sc, "cnt")
+    if lse_nat is not None:
+        _want(lse_nat, torch.float32, (plan.B, plan.heads, plan.L), "lse_nat")
+    wsb = 0 if ws is None else ws.numel() * ws.element_size()
+    _check(_lib.attn_forward_natural(plan.handle, _ptr(q), _ptr(k), _ptr(q_scale), _ptr(k_scale),
+                                     _ptr(v_nat), _ptr(idx), _ptr(cnt), _ptr(o_nat), _ptr(lse_nat),
+                                     _ptr(ws), wsb, _stream(stream)), "attn_forward_natural")
 
 
 def attn_layer(plan: Plan, q_nat, k_nat, v_nat, o_nat, ws, lse_nat=None, idx=None, cnt=None,

@@ -101,7 +101,10 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi, float& sum) 
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-template <int D, bool FP8>
+// NAT: V is read from and O (and lse) written to the natural token layout
+// [B, L, Hh, D] directly, through five-dimensional tensor maps whose box is
+// one tile; Q and K too unless they are e4m3 tile codes (tiled layout).
+template <int D, bool FP8, bool NAT>
 __global__ void __launch_bounds__(kThreads, 2)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, TcParams P) {
@@ -147,6 +150,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   const int head = blockIdx.y, b = blockIdx.z;
   const size_t bh = (size_t)b * g.Hh + head;
   const bool has1 = i1 >= 0;
+  // One tile (64 tokens x 64 columns) of a natural-layout tensor: the box
+  // {64 columns, tw, th, tt, 1} at the tile's first token, rows in (t, h, w)
+  // order like the tiled layout; tokens past the grid's edge read as zero.
+  auto load_nat = [&](uint32_t dst, const CUtensorMap* map, uint32_t bar, int col, int tile) {
+    const int bt = tile / (g.nH * g.nW), bhh = (tile / g.nW) % g.nH, bw = tile % g.nW;
+    tc::tma_load_5d(dst, map, bar, col, bw * g.tw, bhh * g.th, bt * g.tt, b);
+  };
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   // ------------------------------------------------------------ setup
@@ -255,11 +265,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       tc::tma_prefetch_desc(&tmV);
       tc::mbar_arrive_expect_tx(bar_q, (has1 ? 2 : 1) * 64 * C::QRB);
       for (int x = 0; x < (has1 ? 2 : 1); ++x) {
-        const int qrow = (int)((bh * g.N + (x ? i1 : i0)) * 64);
+        const int tile = x ? i1 : i0;
 #pragma unroll
-        for (int cb = 0; cb < C::QBLK; ++cb)
-          tc::tma_load_2d(sb + C::OFF_Q + cb * 128 * C::SWB + x * 64 * C::SWB, &tmQ, bar_q, cb * C::SWB / C::ESZ,
-                          qrow);
+        for (int cb = 0; cb < C::QBLK; ++cb) {
+          const uint32_t dst = sb + C::OFF_Q + cb * 128 * C::SWB + x * 64 * C::SWB;
+          if (NAT && !FP8)
+            load_nat(dst, &tmQ, bar_q, head * D + cb * 64, tile);
+          else
+            tc::tma_load_2d(dst, &tmQ, bar_q, cb * C::SWB / C::ESZ, (int)((bh * g.N + tile) * 64));
+        }
       }
       // K_m is issued as soon as S_{m-2} has released its slot, V_{m-1} once
       // PV_{m-3} has: the two rings free up in MMA completion order, so K
@@ -275,12 +289,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             record_timeout(abort_flag, P.err);
             break;
           }
-          const int krow = (int)((bh * g.N + (int)(ulist[m] & 0x3FFFFFFFu)) * 64);
+          const int kt = (int)(ulist[m] & 0x3FFFFFFFu);
           tc::mbar_arrive_expect_tx(bar_kfull(s), C::K_BYTES);
 #pragma unroll
-          for (int cb = 0; cb < C::QBLK; ++cb)
-            tc::tma_load_2d(sb + C::OFF_K + s * C::K_BYTES + cb * 64 * C::SWB, &tmK, bar_kfull(s),
-                            cb * C::SWB / C::ESZ, krow);
+          for (int cb = 0; cb < C::QBLK; ++cb) {
+            const uint32_t dst = sb + C::OFF_K + s * C::K_BYTES + cb * 64 * C::SWB;
+            if (NAT && !FP8)
+              load_nat(dst, &tmK, bar_kfull(s), head * D + cb * 64, kt);
+            else
+              tc::tma_load_2d(dst, &tmK, bar_kfull(s), cb * C::SWB / C::ESZ, (int)((bh * g.N + kt) * 64));
+          }
           lastk[s] = m;
         }
         if (m >= 1) {
@@ -290,11 +308,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             record_timeout(abort_flag, P.err);
             break;
           }
-          const int vrow = (int)((bh * g.N + (int)(ulist[v] & 0x3FFFFFFFu)) * 64);
+          const int vt = (int)(ulist[v] & 0x3FFFFFFFu);
           tc::mbar_arrive_expect_tx(bar_vfull(s), C::V_BYTES);
 #pragma unroll
-          for (int vb = 0; vb < C::VBLK; ++vb)
-            tc::tma_load_2d(sb + C::OFF_V + s * C::V_BYTES + vb * 8192, &tmV, bar_vfull(s), vb * 64, vrow);
+          for (int vb = 0; vb < C::VBLK; ++vb) {
+            const uint32_t dst = sb + C::OFF_V + s * C::V_BYTES + vb * 8192;
+            if (NAT)
+              load_nat(dst, &tmV, bar_vfull(s), head * D + vb * 64, vt);
+            else
+              tc::tma_load_2d(dst, &tmV, bar_vfull(s), vb * 64, (int)((bh * g.N + vt) * 64));
+          }
           lastv[s] = v;
         }
       }
@@ -501,16 +524,37 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       for (int q = 0; q < 4; ++q)
         reinterpret_cast<uint4*>(stage + c0 * 2)[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
     }
-    if (P.lse && row_exists)
-      P.lse[(bh * g.N + (half ? i1 : i0)) * 64 + (r & 63)] =
-          l > 0.f ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
+    // Token of row rr of the block (natural layout), -1 for a padded slot.
+    auto token_of = [&](int rr) -> int {
+      const int tile = rr >> 6 ? i1 : i0, q = rr & 63;
+      const int t = (tile / (g.nH * g.nW)) * g.tt + q / (g.th * g.tw);
+      const int h = ((tile / g.nW) % g.nH) * g.th + (q / g.tw) % g.th;
+      const int w = (tile % g.nW) * g.tw + q % g.tw;
+      return (t < g.T && h < g.H && w < g.W) ? (t * g.H + h) * g.W + w : -1;
+    };
+    const float lse_r = l > 0.f ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
+    if (P.lse && row_exists) {
+      if (NAT) {
+        const int n = token_of(r);
+        if (n >= 0) P.lse[bh * (size_t)g.L + n] = lse_r;
+      } else {
+        P.lse[(bh * g.N + (half ? i1 : i0)) * 64 + (r & 63)] = lse_r;
+      }
+    }
     asm volatile("bar.sync 1, 128;" ::: "memory");
     constexpr int CPR = D / 8;  // 16-byte chunks per row
     const int rows = has1 ? 128 : 64;
     for (int e2 = r; e2 < rows * CPR; e2 += 128) {
       const int rr = e2 / CPR, cc = e2 % CPR;
-      uint4* og = reinterpret_cast<uint4*>(P.o + (bh * g.N + (rr >> 6 ? i1 : i0)) * 64 * (size_t)D);
-      og[(rr & 63) * CPR + cc] = *reinterpret_cast<const uint4*>(smem + C::OFF_K + rr * C::O_PITCH + cc * 16);
+      const uint4 val = *reinterpret_cast<const uint4*>(smem + C::OFF_K + rr * C::O_PITCH + cc * 16);
+      if (NAT) {
+        const int n = token_of(rr);
+        if (n >= 0)
+          reinterpret_cast<uint4*>(P.o + (((size_t)b * g.L + n) * g.Hh + head) * D)[cc] = val;
+      } else {
+        uint4* og = reinterpret_cast<uint4*>(P.o + (bh * g.N + (rr >> 6 ? i1 : i0)) * 64 * (size_t)D);
+        og[(rr & 63) * CPR + cc] = val;
+      }
     }
   }
 
@@ -550,7 +594,25 @@ bool make_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int es
   return r == CUDA_SUCCESS;
 }
 
-template <int D, bool FP8>
+// Natural-layout tensor [B, T, H, W, Hh * D] as five dimensions, innermost
+// first, with a one-tile box of 64 columns (128 bytes, one swizzle span).
+bool make_map_nat(CUtensorMap* map, const void* base, const bsattn_plan* p) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const bsattn_desc& d = p->desc;
+  const cuuint64_t row = (cuuint64_t)d.heads * d.head_dim * 2;  // bytes per token
+  cuuint64_t dims[5] = {(cuuint64_t)d.heads * d.head_dim, (cuuint64_t)d.W, (cuuint64_t)d.H, (cuuint64_t)d.T,
+                        (cuuint64_t)d.B};
+  cuuint64_t strides[4] = {row, row * d.W, row * d.W * d.H, row * d.W * d.H * d.T};
+  cuuint32_t box[5] = {64, (cuuint32_t)d.tile_w, (cuuint32_t)d.tile_h, (cuuint32_t)d.tile_t, 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int D, bool FP8, bool NAT>
 bsattn_status run(const bsattn_plan* p, const void* q, const void* k, const __nv_bfloat16* v,
                   TcParams prm, cudaStream_t st) {
   using C = Cfg<D, FP8>;
@@ -559,14 +621,19 @@ bsattn_status run(const bsattn_plan* p, const void* q, const void* k, const __nv
   CUtensorMap mq, mk, mv;
   const CUtensorMapDataType dqk = FP8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const CUtensorMapSwizzle sw = C::SWB == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
-  if (!make_map(&mq, q, dqk, C::ESZ, D, rows, C::SWB / C::ESZ, 64, sw) ||
-      !make_map(&mk, k, dqk, C::ESZ, D, rows, C::SWB / C::ESZ, 64, sw) ||
-      !make_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, rows, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+  if (NAT && !FP8) {
+    if (!make_map_nat(&mq, q, p) || !make_map_nat(&mk, k, p)) return BSATTN_ERR_CUDA;
+  } else if (!make_map(&mq, q, dqk, C::ESZ, D, rows, C::SWB / C::ESZ, 64, sw) ||
+             !make_map(&mk, k, dqk, C::ESZ, D, rows, C::SWB / C::ESZ, 64, sw)) {
+    return BSATTN_ERR_CUDA;
+  }
+  if (NAT ? !make_map_nat(&mv, v, p)
+          : !make_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, rows, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B))
     return BSATTN_ERR_CUDA;
   size_t smem = 1024 + C::OFF_DYN + (size_t)prm.bm_words * 8 + (size_t)prm.umax * 4;
   if (smem < 80 * 1024) smem = 80 * 1024;  // at most two CTAs (2 x 256 TMEM columns) per SM
   if (smem > 227 * 1024) return BSATTN_ERR_UNSUPPORTED;
-  auto kern = attn_tc_kernel<D, FP8>;
+  auto kern = attn_tc_kernel<D, FP8, NAT>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return BSATTN_ERR_CUDA;
   dim3 grid(prm.pdim[0] * prm.pdim[1] * prm.pdim[2], p->desc.heads, p->desc.B);
@@ -581,7 +648,7 @@ size_t attention_workspace_bytes(const bsattn_plan*) { return 0; }
 bsattn_status launch_attention(const bsattn_plan* p, const void* q, const void* k, const float* qs,
                                const float* ks, const __nv_bfloat16* v, const int32_t* idx,
                                const int32_t* cnt, __nv_bfloat16* o, float* lse, void*, size_t,
-                               cudaStream_t st) {
+                               cudaStream_t st, bool natural) {
   if (p->N > 32768) return BSATTN_ERR_UNSUPPORTED;
   TcParams prm;
   prm.g = make_geom(p);
@@ -603,7 +670,12 @@ bsattn_status launch_attention(const bsattn_plan* p, const void* q, const void* 
   const int nd[3] = {p->nT, p->nH, p->nW};
   for (int a = 0; a < 3; ++a) prm.pdim[a] = a == prm.pair_axis ? (nd[a] + 1) / 2 : nd[a];
   const bool fp8 = p->desc.qk_fp8 != 0;
+  if (natural) {
+    if (p->desc.head_dim == 128)
+      return fp8 ? run<128, true, true>(p, q, k, v, prm, st) : run<128, false, true>(p, q, k, v, prm, st);
+    return fp8 ? run<64, true, true>(p, q, k, v, prm, st) : run<64, false, true>(p, q, k, v, prm, st);
+  }
   if (p->desc.head_dim == 128)
-    return fp8 ? run<128, true>(p, q, k, v, prm, st) : run<128, false>(p, q, k, v, prm, st);
-  return fp8 ? run<64, true>(p, q, k, v, prm, st) : run<64, false>(p, q, k, v, prm, st);
+    return fp8 ? run<128, true, false>(p, q, k, v, prm, st) : run<128, false, false>(p, q, k, v, prm, st);
+  return fp8 ? run<64, true, false>(p, q, k, v, prm, st) : run<64, false, false>(p, q, k, v, prm, st);
 }

@@ -54,12 +54,13 @@ static inline bool aligned16(const void* ptr) { return (((uintptr_t)ptr) & 15u) 
 // flags for launch_reorder
 enum : int {
   RO_WRITE_TILED = 1,  // write the tiled bf16 copy
-  RO_POOL = 2,         // write fp32 tile means
-  RO_QUANT = 4,        // write e4m3 codes + tile scales instead of/in addition to bf16
+  RO_QUANT = 4,        // write e4m3 codes + tile scales
 };
 bsattn_status launch_reorder(const Geom& g, const __nv_bfloat16* x_nat, __nv_bfloat16* x_tiled,
-                             float* pooled, uint8_t* codes, float* scales, int flags,
-                             cudaStream_t st);
+                             uint8_t* codes, float* scales, int flags, cudaStream_t st);
+// fp32 tile means of one or two natural tensors (x1/p1 may be null).
+bsattn_status launch_pool(const Geom& g, const __nv_bfloat16* x0, float* p0, const __nv_bfloat16* x1,
+                          float* p1, cudaStream_t st);
 bsattn_status launch_unreorder(const Geom& g, const __nv_bfloat16* x_tiled, __nv_bfloat16* x_nat,
                                const float* lse_tiled, float* lse_nat, cudaStream_t st);
 bsattn_status launch_quant_tiled(const Geom& g, const __nv_bfloat16* x_tiled, uint8_t* codes,
@@ -73,8 +74,11 @@ bsattn_status launch_select_topp(int rows, int N, int k, double p, const float* 
 bsattn_status launch_broadcast_lists(int bh, int N, int kmax, const int32_t* src_idx,
                                      const int32_t* src_cnt, int32_t* idx, int32_t* cnt,
                                      cudaStream_t st);
+// natural: V, O and lse in the natural layout ([B, L, Hh, D], [B, Hh, L]);
+// Q and K too unless they are e4m3 tile codes. Otherwise all tiled.
 bsattn_status launch_attention(const bsattn_plan* p, const void* q, const void* k,
                                const float* qs, const float* ks, const __nv_bfloat16* v,
                                const int32_t* idx, const int32_t* cnt, __nv_bfloat16* o,
-                               float* lse, void* ws, size_t ws_bytes, cudaStream_t st);
+                               float* lse, void* ws, size_t ws_bytes, cudaStream_t st,
+                               bool natural);
 size_t attention_workspace_bytes(const bsattn_plan* p);

@@ -41,28 +41,25 @@ SelectWs carve_select(const bsattn_plan* p, Carve& c) {
   return w;
 }
 
+// The layer reads Q, K, V and writes O in the natural layout; only e4m3 Q/K
+// codes (with their tile scales) need a tiled copy.
 struct LayerWs {
-  void* qt;  // bf16 tiled or e4m3 codes
-  void* kt;
-  __nv_bfloat16* vt;
+  uint8_t* qt;  // e4m3 tile codes (qk_fp8 only)
+  uint8_t* kt;
   float* qs;
   float* ks;
   SelectWs sel;
   int32_t* idx;
   int32_t* cnt;
-  __nv_bfloat16* ot;
-  float* lse_t;
   void* attn_ws;
 };
 
 LayerWs carve_layer(const bsattn_plan* p, Carve& c) {
   size_t bh = (size_t)p->desc.B * p->desc.heads;
   size_t elems = bh * p->N * p->V * p->desc.head_dim;
-  size_t qk_elt = p->desc.qk_fp8 ? 1 : 2;
   LayerWs w;
-  w.qt = c.take(elems * qk_elt);
-  w.kt = c.take(elems * qk_elt);
-  w.vt = (__nv_bfloat16*)c.take(elems * 2);
+  w.qt = (uint8_t*)c.take(p->desc.qk_fp8 ? elems : 0);
+  w.kt = (uint8_t*)c.take(p->desc.qk_fp8 ? elems : 0);
   w.qs = (float*)c.take(p->desc.qk_fp8 ? bh * p->N * sizeof(float) : 0);
   w.ks = (float*)c.take(p->desc.qk_fp8 ? bh * p->N * sizeof(float) : 0);
   if (p->rule.kind == BSATTN_RULE_WINDOW) {
@@ -72,8 +69,6 @@ LayerWs carve_layer(const bsattn_plan* p, Carve& c) {
   }
   w.idx = (int32_t*)c.take(bh * p->N * p->kmax * sizeof(int32_t));
   w.cnt = (int32_t*)c.take(bh * p->N * sizeof(int32_t));
-  w.ot = (__nv_bfloat16*)c.take(elems * 2);
-  w.lse_t = (float*)c.take(bh * p->N * p->V * sizeof(float));
   w.attn_ws = c.take(attention_workspace_bytes(p));
   return w;
 }
@@ -223,17 +218,20 @@ bsattn_status attn_reorder(const bsattn_plan* p, const void* x_nat, void* x_tile
     return BSATTN_ERR_INVALID_ARG;
   bsattn_status s = set_device(p);
   if (s) return s;
-  return launch_reorder(make_geom(p), (const __nv_bfloat16*)x_nat, (__nv_bfloat16*)x_tiled, pooled,
-                        nullptr, nullptr, RO_WRITE_TILED | (pooled ? RO_POOL : 0),
-                        (cudaStream_t)stream);
+  Geom g = make_geom(p);
+  if ((s = launch_reorder(g, (const __nv_bfloat16*)x_nat, (__nv_bfloat16*)x_tiled, nullptr, nullptr,
+                          RO_WRITE_TILED, (cudaStream_t)stream)))
+    return s;
+  return pooled ? launch_pool(g, (const __nv_bfloat16*)x_nat, pooled, nullptr, nullptr, (cudaStream_t)stream)
+                : BSATTN_OK;
 }
 
 bsattn_status attn_pool(const bsattn_plan* p, const void* x_nat, float* pooled, void* stream) {
   if (!p || !ok_ptr(x_nat) || !ok_ptr(pooled)) return BSATTN_ERR_INVALID_ARG;
   bsattn_status s = set_device(p);
   if (s) return s;
-  return launch_reorder(make_geom(p), (const __nv_bfloat16*)x_nat, nullptr, pooled, nullptr,
-                        nullptr, RO_POOL, (cudaStream_t)stream);
+  return launch_pool(make_geom(p), (const __nv_bfloat16*)x_nat, pooled, nullptr, nullptr,
+                     (cudaStream_t)stream);
 }
 
 bsattn_status attn_unreorder(const bsattn_plan* p, const void* x_tiled, void* x_nat,
@@ -290,10 +288,7 @@ bsattn_status attn_select(const bsattn_plan* p, const void* q_nat, const void* k
   Carve c(ws);
   SelectWs w = carve_select(p, c);
   Geom g = make_geom(p);
-  if ((s = launch_reorder(g, (const __nv_bfloat16*)q_nat, nullptr, w.pq, nullptr, nullptr, RO_POOL, st)))
-    return s;
-  if ((s = launch_reorder(g, (const __nv_bfloat16*)k_nat, nullptr, w.pk, nullptr, nullptr, RO_POOL, st)))
-    return s;
+  if ((s = launch_pool(g, (const __nv_bfloat16*)q_nat, w.pq, (const __nv_bfloat16*)k_nat, w.pk, st))) return s;
   if ((s = launch_block_scores(g, w.pq, w.pk, p->scale, w.S, st))) return s;
   return select_core(p, w.S, idx, cnt, st);
 }
@@ -319,7 +314,23 @@ bsattn_status attn_forward(const bsattn_plan* p, const void* q, const void* k, c
   bsattn_status s = set_device(p);
   if (s) return s;
   return launch_attention(p, q, k, qs, ks, (const __nv_bfloat16*)v, idx, cnt, (__nv_bfloat16*)o,
-                          lse, ws, ws_bytes, (cudaStream_t)stream);
+                          lse, ws, ws_bytes, (cudaStream_t)stream, false);
+}
+
+bsattn_status attn_forward_natural(const bsattn_plan* p, const void* q, const void* k, const float* qs,
+                                   const float* ks, const void* v_nat, const int32_t* idx,
+                                   const int32_t* cnt, void* o_nat, float* lse_nat, void* ws,
+                                   size_t ws_bytes, void* stream) {
+  if (!p || !ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v_nat) || !ok_ptr(idx) || !ok_ptr(cnt) ||
+      !ok_ptr(o_nat) || (lse_nat && !aligned16(lse_nat)))
+    return BSATTN_ERR_INVALID_ARG;
+  if (p->desc.qk_fp8 && (!ok_ptr(qs) || !ok_ptr(ks))) return BSATTN_ERR_INVALID_ARG;
+  size_t need = attention_workspace_bytes(p);
+  if (need && (!ws || !aligned16(ws) || ws_bytes < need)) return BSATTN_ERR_WORKSPACE;
+  bsattn_status s = set_device(p);
+  if (s) return s;
+  return launch_attention(p, q, k, qs, ks, (const __nv_bfloat16*)v_nat, idx, cnt, (__nv_bfloat16*)o_nat,
+                          lse_nat, ws, ws_bytes, (cudaStream_t)stream, true);
 }
 
 bsattn_status attn_layer(const bsattn_plan* p, const void* q_nat, const void* k_nat,
@@ -341,28 +352,22 @@ bsattn_status attn_layer(const bsattn_plan* p, const void* q_nat, const void* k_
   int32_t* idx = idx_out ? idx_out : w.idx;
   int32_t* cnt = cnt_out ? cnt_out : w.cnt;
   bool pool = p->rule.kind != BSATTN_RULE_WINDOW;
+  const void* q = q_nat;
+  const void* k = k_nat;
   if (p->desc.qk_fp8) {
-    int f = RO_QUANT | (pool ? RO_POOL : 0);
-    if ((s = launch_reorder(g, (const __nv_bfloat16*)q_nat, nullptr, w.sel.pq, (uint8_t*)w.qt, w.qs, f, st)))
-      return s;
-    if ((s = launch_reorder(g, (const __nv_bfloat16*)k_nat, nullptr, w.sel.pk, (uint8_t*)w.kt, w.ks, f, st)))
-      return s;
-  } else {
-    int f = RO_WRITE_TILED | (pool ? RO_POOL : 0);
-    if ((s = launch_reorder(g, (const __nv_bfloat16*)q_nat, (__nv_bfloat16*)w.qt, w.sel.pq, nullptr, nullptr, f, st)))
-      return s;
-    if ((s = launch_reorder(g, (const __nv_bfloat16*)k_nat, (__nv_bfloat16*)w.kt, w.sel.pk, nullptr, nullptr, f, st)))
-      return s;
+    // e4m3 tile codes and scales.
+    if ((s = launch_reorder(g, (const __nv_bfloat16*)q_nat, nullptr, w.qt, w.qs, RO_QUANT, st))) return s;
+    if ((s = launch_reorder(g, (const __nv_bfloat16*)k_nat, nullptr, w.kt, w.ks, RO_QUANT, st))) return s;
+    q = w.qt;
+    k = w.kt;
   }
-  if ((s = launch_reorder(g, (const __nv_bfloat16*)v_nat, w.vt, nullptr, nullptr, nullptr, RO_WRITE_TILED, st)))
+  // Tile means for the scores; the attention reads natural tensors tile by tile.
+  if (pool && (s = launch_pool(g, (const __nv_bfloat16*)q_nat, w.sel.pq, (const __nv_bfloat16*)k_nat, w.sel.pk, st)))
     return s;
   if (pool && (s = launch_block_scores(g, w.sel.pq, w.sel.pk, p->scale, w.sel.S, st))) return s;
   if ((s = select_core(p, w.sel.S, idx, cnt, st))) return s;
-  if ((s = launch_attention(p, w.qt, w.kt, w.qs, w.ks, w.vt, idx, cnt, w.ot,
-                            lse_nat ? w.lse_t : nullptr, w.attn_ws,
-                            attention_workspace_bytes(p), st)))
-    return s;
-  return launch_unreorder(g, w.ot, (__nv_bfloat16*)o_nat, lse_nat ? w.lse_t : nullptr, lse_nat, st);
+  return launch_attention(p, q, k, w.qs, w.ks, (const __nv_bfloat16*)v_nat, idx, cnt, (__nv_bfloat16*)o_nat,
+                          lse_nat, w.attn_ws, attention_workspace_bytes(p), st, true);
 }
 
 bsattn_status attn_check_device_status(const bsattn_plan* p, void* stream) {

@@ -1,5 +1,5 @@
-// Tile reorder (natural -> tiled) with fused tile-mean pooling and per-tile
-// e4m3 quantisation, the inverse scatter, and standalone tile quantisation.
+// Tile reorder (natural -> tiled) with fused per-tile e4m3 quantisation, the
+// inverse scatter, standalone tile quantisation, and tile-mean pooling.
 //
 // These steps move bytes: one CTA per (batch, head, tile) moves the tile's
 // 64 rows of D bf16 with 16-byte vector accesses. Reads are 64 row segments
@@ -79,12 +79,10 @@ __device__ __forceinline__ float tile_scale_from_amax(float amax) {
 template <int D>
 __global__ void __launch_bounds__(kThreads)
 reorder_kernel(Geom g, const __nv_bfloat16* __restrict__ x_nat, __nv_bfloat16* __restrict__ x_tiled,
-               float* __restrict__ pooled, uint8_t* __restrict__ codes, float* __restrict__ scales,
-               int flags) {
+               uint8_t* __restrict__ codes, float* __restrict__ scales, int flags) {
   constexpr int CH = D / 8;                 // 16-byte chunks per row
   constexpr int ITER = 64 * CH / kThreads;  // chunks per thread
   constexpr int RSTEP = kThreads / CH;      // row stride between a thread's chunks
-  __shared__ float red[RSTEP][D + 1];
   __shared__ float wred[kThreads / 32];
 
   const int j = blockIdx.x, head = blockIdx.y, b = blockIdx.z;
@@ -110,26 +108,6 @@ reorder_kernel(Geom g, const __nv_bfloat16* __restrict__ x_nat, __nv_bfloat16* _
     for (int i = 0; i < ITER; ++i) {
       int r = r0 + RSTEP * i;
       reinterpret_cast<uint4*>(x_tiled + (tile_off + r) * D)[c] = v[i];
-    }
-  }
-  if (flags & RO_POOL) {
-    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-#pragma unroll
-    for (int i = 0; i < ITER; ++i) {
-      float f[8];
-      bf16x8_to_f32(v[i], f);  // padded slots hold zeros
-#pragma unroll
-      for (int e = 0; e < 8; ++e) acc[e] += f[e];
-    }
-#pragma unroll
-    for (int e = 0; e < 8; ++e) red[r0][c * 8 + e] = acc[e];
-    __syncthreads();
-    if (threadIdx.x < D) {
-      float s = 0.f;
-#pragma unroll
-      for (int q = 0; q < RSTEP; ++q) s += red[q][threadIdx.x];
-      float nvalid = (float)(tc.vt * tc.vh * tc.vw);
-      pooled[(((size_t)b * g.Hh + head) * g.N + j) * D + threadIdx.x] = __fdiv_rn(s, nvalid);
     }
   }
   if (flags & RO_QUANT) {
@@ -209,16 +187,80 @@ quant_tiled_kernel(Geom g, const __nv_bfloat16* __restrict__ x_tiled, uint8_t* _
   if (threadIdx.x == 0) scales[tile] = scale;
 }
 
+// Tile means of natural bf16 tokens. A token row holds all heads
+// (Hh*D*2 contiguous bytes); a CTA takes one tile of one batch and tensor and
+// a block of kPoolCols 16-byte column chunks of those rows, thread c owning
+// chunk c: it sums the chunk over the tile's rows in (t, h, w) order (padded
+// rows add zero), so rows are read coalesced, no cross-thread reduction is
+// needed and the sum order is fixed.
+constexpr int kPoolCols = 128;
+
+template <int D>
+__global__ void __launch_bounds__(kPoolCols)
+pool_kernel(Geom g, const __nv_bfloat16* __restrict__ x0, const __nv_bfloat16* __restrict__ x1,
+            float* __restrict__ p0, float* __restrict__ p1, int ncblk) {
+  constexpr int CH = D / 8;   // 16-byte chunks per head row
+  __shared__ int rowoff[64];  // token offset of each in-tile row from the tile's first token, -1 if padded
+  const int tensor = blockIdx.z / ncblk, cblk = blockIdx.z % ncblk;
+  const __nv_bfloat16* x = tensor ? x1 : x0;
+  float* pooled = tensor ? p1 : p0;
+  const int j = blockIdx.x, b = blockIdx.y;
+  const TileCoord tc = tile_coord(g, j);
+  const int n0 = (tc.t0 * g.H + tc.h0) * g.W + tc.w0;
+  if (threadIdx.x < 64) {
+    const int n = row_token(g, tc, threadIdx.x);
+    rowoff[threadIdx.x] = n >= 0 ? n - n0 : -1;
+  }
+  __syncthreads();
+  const int cpt = g.Hh * CH;  // chunks per token (all heads)
+  const int c = cblk * kPoolCols + threadIdx.x;
+  if (c >= cpt) return;
+  const float nvalid = (float)(tc.vt * tc.vh * tc.vw);
+  const uint4* src = reinterpret_cast<const uint4*>(x + ((size_t)b * g.L + n0) * g.Hh * D) + c;
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  for (int r0 = 0; r0 < 64; r0 += 16) {  // sixteen loads in flight
+    uint4 v[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int off = rowoff[r0 + i];
+      v[i] = off >= 0 ? __ldg(src + (size_t)off * cpt) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      float f[8];
+      bf16x8_to_f32(v[i], f);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] += f[e];
+    }
+  }
+  const int head = c / CH, d0 = (c % CH) * 8;
+  float4* out = reinterpret_cast<float4*>(pooled + (((size_t)b * g.Hh + head) * g.N + j) * D + d0);
+  out[0] = make_float4(__fdiv_rn(acc[0], nvalid), __fdiv_rn(acc[1], nvalid), __fdiv_rn(acc[2], nvalid),
+                       __fdiv_rn(acc[3], nvalid));
+  out[1] = make_float4(__fdiv_rn(acc[4], nvalid), __fdiv_rn(acc[5], nvalid), __fdiv_rn(acc[6], nvalid),
+                       __fdiv_rn(acc[7], nvalid));
+}
+
 }  // namespace
 
+bsattn_status launch_pool(const Geom& g, const __nv_bfloat16* x0, float* p0, const __nv_bfloat16* x1,
+                          float* p1, cudaStream_t st) {
+  const int cpt = g.Hh * g.D / 8, ncblk = (cpt + kPoolCols - 1) / kPoolCols;
+  dim3 grid(g.N, g.B, (x1 ? 2 : 1) * ncblk);
+  if (g.D == 128)
+    pool_kernel<128><<<grid, kPoolCols, 0, st>>>(g, x0, x1, p0, p1, ncblk);
+  else
+    pool_kernel<64><<<grid, kPoolCols, 0, st>>>(g, x0, x1, p0, p1, ncblk);
+  return cudaGetLastError() == cudaSuccess ? BSATTN_OK : BSATTN_ERR_CUDA;
+}
+
 bsattn_status launch_reorder(const Geom& g, const __nv_bfloat16* x_nat, __nv_bfloat16* x_tiled,
-                             float* pooled, uint8_t* codes, float* scales, int flags,
-                             cudaStream_t st) {
+                             uint8_t* codes, float* scales, int flags, cudaStream_t st) {
   dim3 grid(g.N, g.Hh, g.B);
   if (g.D == 128)
-    reorder_kernel<128><<<grid, kThreads, 0, st>>>(g, x_nat, x_tiled, pooled, codes, scales, flags);
+    reorder_kernel<128><<<grid, kThreads, 0, st>>>(g, x_nat, x_tiled, codes, scales, flags);
   else
-    reorder_kernel<64><<<grid, kThreads, 0, st>>>(g, x_nat, x_tiled, pooled, codes, scales, flags);
+    reorder_kernel<64><<<grid, kThreads, 0, st>>>(g, x_nat, x_tiled, codes, scales, flags);
   return cudaGetLastError() == cudaSuccess ? BSATTN_OK : BSATTN_ERR_CUDA;
 }
 

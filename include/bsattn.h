@@ -196,9 +196,25 @@ bsattn_status attn_forward(const bsattn_plan* plan, const void* q, const void* k
                            const int32_t* idx, const int32_t* cnt, void* o_tiled,
                            float* lse, void* ws, size_t ws_bytes, void* stream);
 
-/* The whole layer on natural tensors: reorder + pool (+ e4m3 quantisation),
- * block scores, selection, block-sparse attention, unreorder. Writes natural
- * bf16 O and, if non-NULL, natural fp32 lse [B, Hh, L]. If idx_out/cnt_out
+/* Step 4 on natural tensors: the same attention as attn_forward, reading
+ * each (t, h, w) tile straight from natural [B, L, Hh, D] bf16 v (and q, k,
+ * unless the plan has qk_fp8, in which case q/k are tiled e4m3 codes with
+ * their tile scales as for attn_forward); tokens past the grid's edge read
+ * as zero and are masked. Writes natural bf16 o_nat [B, L, Hh, D] and, if
+ * non-NULL, natural fp32 lse [B, Hh, L]; padded slots are not written.
+ * Pointers 16-byte aligned; `ws` as for attn_forward. */
+bsattn_status attn_forward_natural(const bsattn_plan* plan, const void* q, const void* k,
+                                   const float* q_scale, const float* k_scale, const void* v_nat,
+                                   const int32_t* idx, const int32_t* cnt, void* o_nat,
+                                   float* lse_nat, void* ws, size_t ws_bytes, void* stream);
+
+/* The whole layer on natural tensors: pool (+ e4m3 quantisation of Q and K
+ * into tile codes), block scores, selection, block-sparse attention. The
+ * attention reads each (t, h, w) tile of Q, K and V straight from the
+ * natural layout (the tile reorder happens in its loads; tokens past the
+ * grid's edge read as zero and are masked) and writes natural bf16 O and, if
+ * non-NULL, natural fp32 lse [B, Hh, L]. Results equal the step-by-step path
+ * (reorder, attn_forward, unreorder). If idx_out/cnt_out
  * are non-NULL the kept lists are also copied there. `ws` must hold
  * info.layer_workspace_bytes. */
 bsattn_status attn_layer(const bsattn_plan* plan, const void* q_nat, const void* k_nat,

@@ -246,3 +246,55 @@ def test_bad_list_entry_sets_error_word_and_is_skipped(bs):
     cnt_bad = torch.full(sc, plan.kmax + 1, dtype=torch.int32, device="cuda")
     bs.attn_forward(plan, *tiled, idx2, cnt_bad, o2)
     assert bs.attn_check_device_status(plan) == 5
+
+
+@pytest.mark.parametrize("name", ["tiny_d64", "ragged_topk", "ragged_topp", "ragged_bf16_window",
+                                  "ragged_window_fp8", "ragged_d64_fp8"])
+def test_forward_natural_equals_tiled_path(bs, name):
+    """Natural-layout attention (tile reorder folded into its loads) gives
+    bit-identical O and lse to reorder -> attn_forward -> unreorder."""
+    wl = SMALL[name]
+    plan = _plan(bs, wl)
+    q, k, v = make_qkv(wl, "cuda")
+    si, sc = plan.list_shapes()
+    idx = torch.empty(si, dtype=torch.int32, device="cuda")
+    cnt = torch.empty(sc, dtype=torch.int32, device="cuda")
+    ws = plan.workspace("select")
+    bs.attn_select(plan, q, k, idx, cnt, ws)
+    ts = plan.tiled_shape()
+    vt = torch.empty(ts, dtype=torch.bfloat16, device="cuda")
+    bs.attn_reorder(plan, v, vt)
+    qs = ks = None
+    if plan.qk_fp8:
+        qa, ka = (torch.empty(ts, dtype=torch.uint8, device="cuda") for _ in range(2))
+        qs, ks = (torch.empty((wl.B, wl.heads, plan.N), dtype=torch.float32, device="cuda") for _ in range(2))
+        for x, codes, scales in ((q, qa, qs), (k, ka, ks)):
+            xt = torch.empty(ts, dtype=torch.bfloat16, device="cuda")
+            bs.attn_reorder(plan, x, xt)
+            bs.attn_quantize_e4m3(plan, xt, codes, scales)
+        qn, kn = qa, ka
+    else:
+        qa, ka = (torch.empty(ts, dtype=torch.bfloat16, device="cuda") for _ in range(2))
+        bs.attn_reorder(plan, q, qa)
+        bs.attn_reorder(plan, k, ka)
+        qn, kn = q, k
+    ot = torch.empty(ts, dtype=torch.bfloat16, device="cuda")
+    lse_t = torch.empty((wl.B, wl.heads, plan.N, 64), dtype=torch.float32, device="cuda")
+    bs.attn_forward(plan, qa, ka, vt, idx, cnt, ot, lse_t, q_scale=qs, k_scale=ks)
+    o_ref = torch.empty_like(q)
+    bs.attn_unreorder(plan, ot, o_ref)
+    o_nat = torch.full_like(q, float("nan"))
+    lse_nat = torch.full((wl.B, wl.heads, plan.L), float("nan"), dtype=torch.float32, device="cuda")
+    bs.attn_forward_natural(plan, qn, kn, v, idx, cnt, o_nat, lse_nat, q_scale=qs, k_scale=ks)
+    assert bs.attn_check_device_status(plan) == 0
+    assert torch.equal(o_nat, o_ref)
+    lse_ref = tiling_lse_natural(lse_t, wl, plan)
+    assert torch.equal(lse_nat.cpu(), lse_ref)
+
+
+def tiling_lse_natural(lse_t, wl, plan):
+    """Tiled lse [B, Hh, N, 64] -> natural [B, Hh, L] (oracle's tile order)."""
+    x = to64(lse_t)
+    out = np.stack([tiling.unreorder(x[:, h:h + 1, :, :, None], wl.T, wl.H, wl.W)[..., 0, 0]
+                    for h in range(wl.heads)], axis=1)
+    return torch.from_numpy(out.astype(np.float32))
