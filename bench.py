@@ -126,10 +126,11 @@ def group_accounting(wl, plan, idx: torch.Tensor, cnt: torch.Tensor):
     return int(pairs.sum().item()) * 2, int(pairs.sum().item())
 
 
-def launches_per_step(wl) -> int:
+def launches_per_step(wl, plan) -> int:
     pooled = wl.rule != "window"
     quant = 2 if wl.qk_fp8 else 0  # e4m3 tile codes of Q and K
-    return quant + (2 if pooled else 0) + 1 + 1  # [pool Q+K, scores], select, attention
+    retile = 1 if wl.qk_fp8 else (2 if plan.kmax >= 64 else 0)  # K and V (or V) re-tiled once
+    return quant + (2 if pooled else 0) + retile + 1 + 1  # [pool Q+K, scores], select, attention
 
 
 class ClockSampler:
@@ -393,7 +394,7 @@ def main():
                      "traffic": measured_traffic(wl.name)},
         "memory_kernels": memory_kernel_rates(wl, plan, comp, pk),
         "e2e": e2e,
-        "gpu_launches": launches_per_step(wl) * args.steps,
+        "gpu_launches": launches_per_step(wl, plan) * args.steps,
         "clocks": clocks,
     }
     if not args.no_cpu_baseline and world == 1:
@@ -428,8 +429,12 @@ def component_timing(bsattn, plan, wl, q, k, v, flush, stream, reps=20):
         codes = [torch.empty(plan.tiled_shape(), dtype=torch.uint8, device="cuda") for _ in range(2)]
         scales = [torch.empty((wl.B, wl.heads, plan.N), dtype=torch.float32, device="cuda")
                   for _ in range(2)]
-    names = ["pool_qk", "reorder_qk", "quantize", "block_scores", "select", "attention",
-             "attention_tiled"]
+    # The layer re-tiles K and V once when kmax >= 64 (many loads per key tile)
+    # or Q/K are e4m3 codes; its attention then reads tiled K/V, timed here as
+    # attn_forward.
+    tiles_kv = wl.qk_fp8 or plan.kmax >= 64
+    names = ["pool_qk", "reorder_qk", "quantize", "reorder_kv", "block_scores", "select", "attention",
+             "attention_tiled", "attention_natural"]
     acc = {n: 0.0 for n in names}
 
     def timed(name, fn):
@@ -461,8 +466,12 @@ def component_timing(bsattn, plan, wl, q, k, v, flush, stream, reps=20):
         if pooled:
             marks.append(timed("block_scores", lambda: bsattn.attn_block_scores(plan, pq, pk, S, stream)))
         marks.append(timed("select", lambda: bsattn.attn_select_from_scores(plan, S, idx, cnt, stream)))
+        if tiles_kv:
+            marks.append(timed("reorder_kv", lambda: (
+                bsattn.attn_reorder(plan, k, tiled[1], None, stream) if not wl.qk_fp8 else None,
+                bsattn.attn_reorder(plan, v, tiled[2], None, stream))))
         flush.fill_(2.0)
-        marks.append(timed("attention", lambda: bsattn.attn_forward_natural(
+        marks.append(timed("attention_natural", lambda: bsattn.attn_forward_natural(
             plan, qn, kn, v, idx, cnt, o, q_scale=qs, k_scale=ks, stream=stream)))
         flush.fill_(3.0)
         marks.append(timed("attention_tiled", lambda: bsattn.attn_forward(
@@ -471,7 +480,9 @@ def component_timing(bsattn, plan, wl, q, k, v, flush, stream, reps=20):
         if r >= 2:
             for n, a, b in marks:
                 acc[n] += a.elapsed_time(b)
-    return {n: acc[n] / reps for n in names if acc[n] > 0}
+    out = {n: acc[n] / reps for n in names if acc[n] > 0}
+    out["attention"] = out["attention_tiled" if tiles_kv else "attention_natural"]
+    return out
 
 
 def memory_kernel_rates(wl, plan, comp, pk):

@@ -101,10 +101,11 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi, float& sum) 
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// NAT: V is read from and O (and lse) written to the natural token layout
-// [B, L, Hh, D] directly, through five-dimensional tensor maps whose box is
-// one tile; Q and K too unless they are e4m3 tile codes (tiled layout).
-template <int D, bool FP8, bool NAT>
+// NQO: Q is read from and O (and lse) written to the natural token layout
+// [B, L, Hh, D] directly; NKV: K and V are read from it. Natural reads go
+// through five-dimensional tensor maps whose box is one tile. e4m3 Q/K are
+// always tile codes (tiled layout).
+template <int D, bool FP8, bool NQO, bool NKV>
 __global__ void __launch_bounds__(kThreads, 2)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, TcParams P) {
@@ -269,7 +270,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 #pragma unroll
         for (int cb = 0; cb < C::QBLK; ++cb) {
           const uint32_t dst = sb + C::OFF_Q + cb * 128 * C::SWB + x * 64 * C::SWB;
-          if (NAT && !FP8)
+          if (NQO && !FP8)
             load_nat(dst, &tmQ, bar_q, head * D + cb * 64, tile);
           else
             tc::tma_load_2d(dst, &tmQ, bar_q, cb * C::SWB / C::ESZ, (int)((bh * g.N + tile) * 64));
@@ -294,7 +295,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 #pragma unroll
           for (int cb = 0; cb < C::QBLK; ++cb) {
             const uint32_t dst = sb + C::OFF_K + s * C::K_BYTES + cb * 64 * C::SWB;
-            if (NAT && !FP8)
+            if (NKV && !FP8)
               load_nat(dst, &tmK, bar_kfull(s), head * D + cb * 64, kt);
             else
               tc::tma_load_2d(dst, &tmK, bar_kfull(s), cb * C::SWB / C::ESZ, (int)((bh * g.N + kt) * 64));
@@ -313,7 +314,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 #pragma unroll
           for (int vb = 0; vb < C::VBLK; ++vb) {
             const uint32_t dst = sb + C::OFF_V + s * C::V_BYTES + vb * 8192;
-            if (NAT)
+            if (NKV)
               load_nat(dst, &tmV, bar_vfull(s), head * D + vb * 64, vt);
             else
               tc::tma_load_2d(dst, &tmV, bar_vfull(s), vb * 64, (int)((bh * g.N + vt) * 64));
@@ -534,7 +535,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     };
     const float lse_r = l > 0.f ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
     if (P.lse && row_exists) {
-      if (NAT) {
+      if (NQO) {
         const int n = token_of(r);
         if (n >= 0) P.lse[bh * (size_t)g.L + n] = lse_r;
       } else {
@@ -547,7 +548,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     for (int e2 = r; e2 < rows * CPR; e2 += 128) {
       const int rr = e2 / CPR, cc = e2 % CPR;
       const uint4 val = *reinterpret_cast<const uint4*>(smem + C::OFF_K + rr * C::O_PITCH + cc * 16);
-      if (NAT) {
+      if (NQO) {
         const int n = token_of(rr);
         if (n >= 0)
           reinterpret_cast<uint4*>(P.o + (((size_t)b * g.L + n) * g.Hh + head) * D)[cc] = val;
@@ -612,7 +613,7 @@ bool make_map_nat(CUtensorMap* map, const void* base, const bsattn_plan* p) {
   return r == CUDA_SUCCESS;
 }
 
-template <int D, bool FP8, bool NAT>
+template <int D, bool FP8, bool NQO, bool NKV>
 bsattn_status run(const bsattn_plan* p, const void* q, const void* k, const __nv_bfloat16* v,
                   TcParams prm, cudaStream_t st) {
   using C = Cfg<D, FP8>;
@@ -621,19 +622,17 @@ bsattn_status run(const bsattn_plan* p, const void* q, const void* k, const __nv
   CUtensorMap mq, mk, mv;
   const CUtensorMapDataType dqk = FP8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const CUtensorMapSwizzle sw = C::SWB == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
-  if (NAT && !FP8) {
-    if (!make_map_nat(&mq, q, p) || !make_map_nat(&mk, k, p)) return BSATTN_ERR_CUDA;
-  } else if (!make_map(&mq, q, dqk, C::ESZ, D, rows, C::SWB / C::ESZ, 64, sw) ||
-             !make_map(&mk, k, dqk, C::ESZ, D, rows, C::SWB / C::ESZ, 64, sw)) {
+  if (NQO && !FP8 ? !make_map_nat(&mq, q, p) : !make_map(&mq, q, dqk, C::ESZ, D, rows, C::SWB / C::ESZ, 64, sw))
     return BSATTN_ERR_CUDA;
-  }
-  if (NAT ? !make_map_nat(&mv, v, p)
+  if (NKV && !FP8 ? !make_map_nat(&mk, k, p) : !make_map(&mk, k, dqk, C::ESZ, D, rows, C::SWB / C::ESZ, 64, sw))
+    return BSATTN_ERR_CUDA;
+  if (NKV ? !make_map_nat(&mv, v, p)
           : !make_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, rows, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B))
     return BSATTN_ERR_CUDA;
   size_t smem = 1024 + C::OFF_DYN + (size_t)prm.bm_words * 8 + (size_t)prm.umax * 4;
   if (smem < 80 * 1024) smem = 80 * 1024;  // at most two CTAs (2 x 256 TMEM columns) per SM
   if (smem > 227 * 1024) return BSATTN_ERR_UNSUPPORTED;
-  auto kern = attn_tc_kernel<D, FP8, NAT>;
+  auto kern = attn_tc_kernel<D, FP8, NQO, NKV>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return BSATTN_ERR_CUDA;
   dim3 grid(prm.pdim[0] * prm.pdim[1] * prm.pdim[2], p->desc.heads, p->desc.B);
@@ -648,7 +647,7 @@ size_t attention_workspace_bytes(const bsattn_plan*) { return 0; }
 bsattn_status launch_attention(const bsattn_plan* p, const void* q, const void* k, const float* qs,
                                const float* ks, const __nv_bfloat16* v, const int32_t* idx,
                                const int32_t* cnt, __nv_bfloat16* o, float* lse, void*, size_t,
-                               cudaStream_t st, bool natural) {
+                               cudaStream_t st, AttnLayout lay) {
   if (p->N > 32768) return BSATTN_ERR_UNSUPPORTED;
   TcParams prm;
   prm.g = make_geom(p);
@@ -669,13 +668,17 @@ bsattn_status launch_attention(const bsattn_plan* p, const void* q, const void* 
   prm.pair_axis = (p->rule.kind == BSATTN_RULE_WINDOW && p->rule.win_w == 0) ? 0 : 2;
   const int nd[3] = {p->nT, p->nH, p->nW};
   for (int a = 0; a < 3; ++a) prm.pdim[a] = a == prm.pair_axis ? (nd[a] + 1) / 2 : nd[a];
-  const bool fp8 = p->desc.qk_fp8 != 0;
-  if (natural) {
-    if (p->desc.head_dim == 128)
-      return fp8 ? run<128, true, true>(p, q, k, v, prm, st) : run<128, false, true>(p, q, k, v, prm, st);
-    return fp8 ? run<64, true, true>(p, q, k, v, prm, st) : run<64, false, true>(p, q, k, v, prm, st);
+  const bool fp8 = p->desc.qk_fp8 != 0, d128 = p->desc.head_dim == 128;
+#define BSATTN_RUN(QO, KV)                                                                          \
+  return d128 ? (fp8 ? run<128, true, QO, KV>(p, q, k, v, prm, st) : run<128, false, QO, KV>(p, q, k, v, prm, st)) \
+              : (fp8 ? run<64, true, QO, KV>(p, q, k, v, prm, st) : run<64, false, QO, KV>(p, q, k, v, prm, st))
+  switch (lay) {
+    case AttnLayout::Natural:
+      BSATTN_RUN(true, true);
+    case AttnLayout::NaturalQO:
+      BSATTN_RUN(true, false);
+    default:
+      BSATTN_RUN(false, false);
   }
-  if (p->desc.head_dim == 128)
-    return fp8 ? run<128, true, false>(p, q, k, v, prm, st) : run<128, false, false>(p, q, k, v, prm, st);
-  return fp8 ? run<64, true, false>(p, q, k, v, prm, st) : run<64, false, false>(p, q, k, v, prm, st);
+#undef BSATTN_RUN
 }

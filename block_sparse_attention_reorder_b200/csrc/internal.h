@@ -74,11 +74,18 @@ bsattn_status launch_select_topp(int rows, int N, int k, double p, const float* 
 bsattn_status launch_broadcast_lists(int bh, int N, int kmax, const int32_t* src_idx,
                                      const int32_t* src_cnt, int32_t* idx, int32_t* cnt,
                                      cudaStream_t st);
-// natural: V, O and lse in the natural layout ([B, L, Hh, D], [B, Hh, L]);
-// Q and K too unless they are e4m3 tile codes. Otherwise all tiled.
+// Where the attention's tensors live. Tiled: all tiled. Natural: Q, K, V, O
+// and lse in the natural layout ([B, L, Hh, D], [B, Hh, L]). NaturalQO: Q, O
+// and lse natural, K and V tiled. e4m3 Q/K are tile codes in every layout.
+enum class AttnLayout { Tiled, Natural, NaturalQO };
 bsattn_status launch_attention(const bsattn_plan* p, const void* q, const void* k,
                                const float* qs, const float* ks, const __nv_bfloat16* v,
                                const int32_t* idx, const int32_t* cnt, __nv_bfloat16* o,
                                float* lse, void* ws, size_t ws_bytes, cudaStream_t st,
-                               bool natural);
+                               AttnLayout lay);
+// Whether attn_layer re-tiles K and V: natural tile loads cost more per load
+// than tiled ones, which outweighs the one-off reorder once a key tile is
+// loaded about 40+ times (kmax >= 64); the e4m3 path re-tiles Q and K anyway
+// and V's reorder is cheap next to it.
+static inline bool layer_tiles_kv(const bsattn_plan* p) { return p->desc.qk_fp8 || p->kmax >= 64; }
 size_t attention_workspace_bytes(const bsattn_plan* p);
