@@ -129,7 +129,7 @@ def group_accounting(wl, plan, idx: torch.Tensor, cnt: torch.Tensor):
 def launches_per_step(wl, plan) -> int:
     pooled = wl.rule != "window"
     quant = 2 if wl.qk_fp8 else 0  # e4m3 tile codes of Q and K
-    retile = 1 if wl.qk_fp8 else (2 if plan.kmax >= 64 else 0)  # K and V (or V) re-tiled once
+    retile = 0 if plan.kmax < 64 else (1 if wl.qk_fp8 else 2)  # K and V (or V) re-tiled once
     return quant + (2 if pooled else 0) + retile + 1 + 1  # [pool Q+K, scores], select, attention
 
 
@@ -429,10 +429,9 @@ def component_timing(bsattn, plan, wl, q, k, v, flush, stream, reps=20):
         codes = [torch.empty(plan.tiled_shape(), dtype=torch.uint8, device="cuda") for _ in range(2)]
         scales = [torch.empty((wl.B, wl.heads, plan.N), dtype=torch.float32, device="cuda")
                   for _ in range(2)]
-    # The layer re-tiles K and V once when kmax >= 64 (many loads per key tile)
-    # or Q/K are e4m3 codes; its attention then reads tiled K/V, timed here as
-    # attn_forward.
-    tiles_kv = wl.qk_fp8 or plan.kmax >= 64
+    # The layer re-tiles K and V once when kmax >= 64 (many loads per key
+    # tile); its attention then reads tiled K/V, timed here as attn_forward.
+    tiles_kv = plan.kmax >= 64
     names = ["pool_qk", "reorder_qk", "quantize", "reorder_kv", "block_scores", "select", "attention",
              "attention_tiled", "attention_natural"]
     acc = {n: 0.0 for n in names}

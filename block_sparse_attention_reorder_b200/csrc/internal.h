@@ -85,7 +85,6 @@ bsattn_status launch_attention(const bsattn_plan* p, const void* q, const void* 
                                AttnLayout lay);
 // Whether attn_layer re-tiles K and V: natural tile loads cost more per load
 // than tiled ones, which outweighs the one-off reorder once a key tile is
-// loaded about 40+ times (kmax >= 64); the e4m3 path re-tiles Q and K anyway
-// and V's reorder is cheap next to it.
-static inline bool layer_tiles_kv(const bsattn_plan* p) { return p->desc.qk_fp8 || p->kmax >= 64; }
+// loaded about 40+ times (kmax >= 64).
+static inline bool layer_tiles_kv(const bsattn_plan* p) { return p->kmax >= 64; }
 size_t attention_workspace_bytes(const bsattn_plan* p);
