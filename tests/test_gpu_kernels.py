@@ -62,6 +62,24 @@ def test_block_scores(bs, name):
     assert np.all(np.abs(to64(S) - ref) <= bound)
 
 
+@pytest.mark.parametrize("grid,heads,D", [((24, 48, 80), 5, 128), ((20, 44, 84), 6, 64)])
+def test_block_scores_large(bs, grid, heads, D):
+    """Large rows take the 128-wide block kernel (ragged N in the second case)."""
+    T, H, W = grid
+    plan = bs.Plan(1, heads, D, T, H, W, rule="topk", k=8)
+    N = plan.N
+    g = torch.Generator(device="cpu").manual_seed(N)
+    pq = torch.randn((1, heads, N, D), generator=g, dtype=torch.float32)
+    pk = torch.randn((1, heads, N, D), generator=g, dtype=torch.float32)
+    S = torch.empty((1, heads, N, N), dtype=torch.float32, device="cuda")
+    bs.attn_block_scores(plan, pq.cuda(), pk.cuda(), S)
+    scale = 1 / math.sqrt(D)
+    ref = select.block_scores(pq.numpy(), pk.numpy(), scale)
+    bound = 1e-5 * scale * np.matmul(np.abs(pq.numpy()).astype(np.float64),
+                                     np.swapaxes(np.abs(pk.numpy()).astype(np.float64), -1, -2)) + 1e-30
+    assert np.all(np.abs(to64(S) - ref) <= bound)
+
+
 @pytest.mark.parametrize("N,k", [(32, 8), (364, 46), (1440, 144), (37, 37), (2048, 1),
                                  (100, 99), (5, 2), (1000, 500)])
 def test_select_topk_bit_exact(bs, N, k):
