@@ -498,6 +498,209 @@ topk_kernel(int rows, int N, int k, const float* __restrict__ S, int32_t* __rest
   if (lane == 0) cnt[r0] = n;
 }
 
+// Top-k for rows of a multiple of 4 tiles and at least 128: the row moves as
+// float4 (lane l holds tiles 128c + 4l .. 4l+3 of 128-tile chunk c), binning
+// uses 128 bins so that four bin indices pack into one 32-bit word, and the
+// second pass compares four packed bins with the boundary bin per SWAR
+// subtraction instead of binning every score again. The general search
+// (lane-strided view of the same staged row) covers crowded boundary bins.
+constexpr int kBins7 = 128;
+
+struct Binning7 {  // Binning with 128 bins (indices fit 7 bits)
+  static constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+  float sc, offm;
+  __device__ __forceinline__ Binning7(float lo, float hi) {
+    sc = (float)kBins7 / (hi - lo);
+    offm = fmaf(-lo, sc, kMagic);
+  }
+  __device__ __forceinline__ uint32_t operator()(float x) const {
+    const float t = fminf(fmaxf(fmaf(x, sc, offm), kMagic), kMagic + (float)(kBins7 - 1));
+    return (uint32_t)(__float_as_int(t) - __float_as_int(kMagic));
+  }
+};
+
+// High bits (7, 15, 23, 31) of a SWAR compare -> 4-bit nibble (bit e = byte e).
+__device__ __forceinline__ uint32_t high_bits_nibble(uint32_t m) { return ((m >> 7) * 0x10204080u) >> 28; }
+
+// Bin (of 128) in which the running count, taken from the top bin down,
+// reaches r > 0; *above = count of higher bins. Lane l owns bins [4l, 4l+4).
+__device__ __forceinline__ int find_bin128(const uint32_t* h, int r, int lane, int* above) {
+  uint32_t c[4], s = 0;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    c[q] = h[4 * lane + q];
+    s += c[q];
+  }
+  uint32_t x = s;  // inclusive suffix sum over lanes
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_down_sync(0xffffffffu, x, o);
+    if (lane + o < 32) x += y;
+  }
+  uint32_t run = x - s;
+  int hit = -1, hit_above = 0;
+#pragma unroll
+  for (int q = 3; q >= 0; --q) {
+    if (hit < 0 && run < (uint32_t)r && (uint32_t)r - run <= c[q]) {
+      hit = 4 * lane + q;
+      hit_above = (int)run;
+    }
+    run += c[q];
+  }
+  const uint32_t m = __ballot_sync(0xffffffffu, hit >= 0);
+  if (!m) return -1;
+  const int src = __ffs(m) - 1;
+  *above = __shfl_sync(0xffffffffu, hit_above, src);
+  return __shfl_sync(0xffffffffu, hit, src);
+}
+
+template <int C4>
+struct Shape4 {
+  static constexpr int per_warp = 128 * C4 * 4 + 128 * C4 + 2 * 4 * C4 * 4 + kBins * 4 + kCand * 8;
+  static constexpr int warps = (8 * per_warp <= 48 * 1024) ? 8 : 4;
+  static_assert(warps * per_warp <= 48 * 1024, "selection shared memory");
+};
+
+template <int C4>
+__global__ void __launch_bounds__(32 * Shape4<C4>::warps)
+topk4_kernel(int rows, int N, int k, const float* __restrict__ S, int32_t* __restrict__ idx,
+             int32_t* __restrict__ cnt, int kmax) {
+  constexpr int W = Shape4<C4>::warps, VPT = 4 * C4;
+  __shared__ __align__(16) float vals_s[W][128 * C4];
+  __shared__ uint32_t bins_s[W][32 * C4];
+  __shared__ uint32_t gt_s[W][4 * C4];
+  __shared__ uint32_t eq_s[W][4 * C4];
+  __shared__ uint32_t hcnt_s[W][kBins];
+  __shared__ uint64_t cand_s[W][kCand];
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r0 = blockIdx.x * W + w;
+  if (r0 >= rows) return;
+  const float* s = S + (size_t)r0 * N;
+  float* slice = vals_s[w];
+  uint32_t* hist = hcnt_s[w];
+  const float qnan = __int_as_float(0x7fc00000);
+
+  // Pass 1: all float4 loads in flight; bins over the extent of an evenly
+  // strided sample of chunks (tiles outside it land in the edge bins).
+  constexpr int B0 = C4 < 4 ? C4 : 4;
+  constexpr int STEP = C4 / B0;
+  float4 v[C4];
+#pragma unroll
+  for (int c = 0; c < C4; ++c) {
+    const int j0 = 128 * c + 4 * lane;  // N % 4 == 0: a float4 is all in or all out
+    v[c] = j0 < N ? __ldg(reinterpret_cast<const float4*>(s + j0)) : make_float4(qnan, qnan, qnan, qnan);
+  }
+  float mn = qnan, mx = qnan;
+#pragma unroll
+  for (int t = 0; t < B0; ++t) {
+    const float4 u = v[t * STEP];
+    mn = fminf(fminf(mn, fminf(u.x, u.y)), fminf(u.z, u.w));
+    mx = fmaxf(fmaxf(mx, fmaxf(u.x, u.y)), fmaxf(u.z, u.w));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  }
+  const bool spread = mn < mx;
+  const Binning7 bin(spread ? mn : 0.f, spread ? mx : 1.f);
+#pragma unroll
+  for (int q = 0; q < kBins7 / 32; ++q) hist[lane + 32 * q] = 0;
+  __syncwarp();
+#pragma unroll
+  for (int c = 0; c < C4; ++c) {
+    const int j0 = 128 * c + 4 * lane;
+    uint32_t word = 0;
+    if (j0 < N) {
+      *reinterpret_cast<float4*>(slice + j0) = v[c];
+      const uint32_t b0 = bin(v[c].x), b1 = bin(v[c].y), b2 = bin(v[c].z), b3 = bin(v[c].w);
+      atomicAdd(&hist[b0], 1u);
+      atomicAdd(&hist[b1], 1u);
+      atomicAdd(&hist[b2], 1u);
+      atomicAdd(&hist[b3], 1u);
+      word = b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
+    }
+    bins_s[w][32 * c + lane] = word;
+  }
+  __syncwarp();
+
+  const int r = min(k, N);
+  int32_t* out = idx + (size_t)r0 * kmax;
+  int n = 0, above = 0;
+  const int b = (spread && r >= 1) ? find_bin128(hist, r, lane, &above) : -1;
+  if (b >= 0 && hist[b] <= (uint32_t)kCand) {
+    // Pass 2: packed bins vs the boundary bin b, four at a time: with every
+    // byte x in [0, 127], (x | 0x80) - c keeps its byte and has the high bit
+    // set exactly when x >= c (c <= 128).
+    const uint32_t cb = (uint32_t)b * 0x01010101u, cb1 = (uint32_t)(b + 1) * 0x01010101u;
+    const int nch = (N + 127) >> 7;
+    const int sh = 4 * (lane & 7);
+    for (int c = 0; c < nch; ++c) {
+      const uint32_t x = bins_s[w][32 * c + lane] | 0x80808080u;
+      const uint32_t ge1 = (x - cb1) & 0x80808080u, ge0 = (x - cb) & 0x80808080u;
+      const uint32_t vm = (128 * c + 4 * lane < N) ? 0xFu : 0u;
+      uint32_t gx = (high_bits_nibble(ge1) & vm) << sh;
+      uint32_t ex = (high_bits_nibble(ge0 & ~ge1) & vm) << sh;
+#pragma unroll
+      for (int o = 1; o < 8; o <<= 1) {  // lanes 8q..8q+7 hold the 32 tiles of word 4c + q
+        gx |= __shfl_xor_sync(0xffffffffu, gx, o);
+        ex |= __shfl_xor_sync(0xffffffffu, ex, o);
+      }
+      if ((lane & 7) == 0) {
+        gt_s[w][4 * c + (lane >> 3)] = gx;
+        eq_s[w][4 * c + (lane >> 3)] = ex;
+      }
+    }
+    __syncwarp();
+    // The boundary bin's tiles, one per lane (their order does not matter:
+    // they are sorted next).
+    const int nw = (N + 31) >> 5;  // <= 64
+    const uint32_t e0 = lane < nw ? eq_s[w][lane] : 0u, e1 = lane + 32 < nw ? eq_s[w][lane + 32] : 0u;
+    const int pc = __popc(e0) + __popc(e1);
+    int x = pc;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    int pos = x - pc;
+    for (int t = 0; t < 2; ++t) {
+      uint32_t m = t ? e1 : e0;
+      const int wbase = 32 * (lane + 32 * t);
+      while (m) {
+        const int j = wbase + __ffs(m) - 1;
+        if (pos < kCand) cand_s[w][pos] = comp_key(slice[j], j);
+        ++pos;
+        m &= m - 1;
+      }
+    }
+    const int nb = min(__shfl_sync(0xffffffffu, x, 31), kCand);
+    __syncwarp();
+    // Keep the candidates ranked above r - above (rank by composite key; the
+    // keys are unique), no full sort needed.
+    const uint64_t mine = lane < nb ? cand_s[w][lane] : 0ull;
+    int rank = 0;
+    for (int t = 0; t < nb; ++t) rank += shfl_idx_u64(mine, t) > mine ? 1 : 0;
+    if (lane < nb && rank < r - above) {
+      const uint32_t j = 0xffffffffu - (uint32_t)mine;
+      atomicOr(&gt_s[w][j >> 5], 1u << (j & 31));
+    }
+    __syncwarp();
+    n = compact_mask<VPT>(gt_s[w], N, lane, out, kmax);
+  } else if (r >= 1) {
+    // General search over the exact extent on the same staged row.
+    const Row row{&slice[lane], N, lane};
+    float lo, hi;
+    row_extent<VPT>(row, &lo, &hi);
+    const Hist h{hist, nullptr};
+    __syncwarp();
+    if (lo < hi) build_hist<VPT, false>(row, true, lo, hi, Binning(lo, hi), 0.0, h);
+    const uint64_t kth = crossing_key<VPT, false>(row, (uint64_t)r, 0.0, lo, hi, h, cand_s[w]);
+    n = write_kept<VPT>(row, kth, out, kmax);
+  }
+  if (lane == 0) cnt[r0] = n;
+}
+
 // Top-p with a top-k floor: in descending order keep the shortest prefix
 // whose softmax mass reaches p of the row's total, then at least k and at
 // most N tiles.
@@ -650,6 +853,14 @@ bsattn_status run_topk(int rows, int N, int k, const float* S, int32_t* idx, int
   return cudaGetLastError() == cudaSuccess ? BSATTN_OK : BSATTN_ERR_CUDA;
 }
 
+template <int C4>
+bsattn_status run_topk4(int rows, int N, int k, const float* S, int32_t* idx, int32_t* cnt, int kmax,
+                        cudaStream_t st) {
+  constexpr int W = Shape4<C4>::warps;
+  topk4_kernel<C4><<<(rows + W - 1) / W, 32 * W, 0, st>>>(rows, N, k, S, idx, cnt, kmax);
+  return cudaGetLastError() == cudaSuccess ? BSATTN_OK : BSATTN_ERR_CUDA;
+}
+
 template <int VPT>
 bsattn_status run_topp(int rows, int N, int k, double p, const float* S, int32_t* idx, int32_t* cnt, int kmax,
                        cudaStream_t st) {
@@ -663,6 +874,17 @@ bsattn_status run_topp(int rows, int N, int k, double p, const float* S, int32_t
 bsattn_status launch_select_topk(int rows, int N, int k, const float* S, int32_t* idx, int32_t* cnt, int kmax,
                                  cudaStream_t st) {
   if (rows <= 0 || N <= 0) return BSATTN_OK;
+  if (N % 4 == 0 && N >= 128 && ((uintptr_t)S & 15u) == 0) {
+    const int c4 = (N + 127) / 128;
+    if (c4 <= 1) return run_topk4<1>(rows, N, k, S, idx, cnt, kmax, st);
+    if (c4 <= 2) return run_topk4<2>(rows, N, k, S, idx, cnt, kmax, st);
+    if (c4 <= 3) return run_topk4<3>(rows, N, k, S, idx, cnt, kmax, st);
+    if (c4 <= 4) return run_topk4<4>(rows, N, k, S, idx, cnt, kmax, st);
+    if (c4 <= 6) return run_topk4<6>(rows, N, k, S, idx, cnt, kmax, st);
+    if (c4 <= 8) return run_topk4<8>(rows, N, k, S, idx, cnt, kmax, st);
+    if (c4 <= 12) return run_topk4<12>(rows, N, k, S, idx, cnt, kmax, st);
+    if (c4 <= 16) return run_topk4<16>(rows, N, k, S, idx, cnt, kmax, st);
+  }
   const int vpt = (N + 31) / 32;
   if (vpt <= 1) return run_topk<1>(rows, N, k, S, idx, cnt, kmax, st);
   if (vpt <= 2) return run_topk<2>(rows, N, k, S, idx, cnt, kmax, st);
