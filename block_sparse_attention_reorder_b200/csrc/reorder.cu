@@ -190,9 +190,11 @@ quant_tiled_kernel(Geom g, const __nv_bfloat16* __restrict__ x_tiled, uint8_t* _
 // Tile means of natural bf16 tokens. A token row holds all heads
 // (Hh*D*2 contiguous bytes); a CTA takes one tile of one batch and tensor and
 // a block of kPoolCols 16-byte column chunks of those rows, thread c owning
-// chunk c: it sums the chunk over the tile's rows in (t, h, w) order (padded
-// rows add zero), so rows are read coalesced, no cross-thread reduction is
-// needed and the sum order is fixed.
+// chunk c: it sums the chunk over the tile's rows in (t, h, w) order, so rows
+// are read coalesced, no cross-thread reduction is needed and the sum order
+// is fixed. Loads go out sixteen at a time and unconditionally (a padded row
+// reloads the tile's first row, which is cached, and adds zero), which keeps
+// all sixteen in flight.
 constexpr int kPoolCols = 128;
 
 template <int D>
@@ -215,24 +217,23 @@ pool_kernel(Geom g, const __nv_bfloat16* __restrict__ x0, const __nv_bfloat16* _
   const int cpt = g.Hh * CH;  // chunks per token (all heads)
   const int c = cblk * kPoolCols + threadIdx.x;
   if (c >= cpt) return;
-  const float nvalid = (float)(tc.vt * tc.vh * tc.vw);
   const uint4* src = reinterpret_cast<const uint4*>(x + ((size_t)b * g.L + n0) * g.Hh * D) + c;
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  for (int r0 = 0; r0 < 64; r0 += 16) {  // sixteen loads in flight
+#pragma unroll 1
+  for (int r0 = 0; r0 < 64; r0 += 16) {
     uint4 v[16];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const int off = rowoff[r0 + i];
-      v[i] = off >= 0 ? __ldg(src + (size_t)off * cpt) : make_uint4(0, 0, 0, 0);
-    }
+    for (int i = 0; i < 16; ++i) v[i] = __ldg(src + (size_t)max(rowoff[r0 + i], 0) * cpt);
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
+      if (rowoff[r0 + i] < 0) continue;
       float f[8];
       bf16x8_to_f32(v[i], f);
 #pragma unroll
       for (int e = 0; e < 8; ++e) acc[e] += f[e];
     }
   }
+  const float nvalid = (float)(tc.vt * tc.vh * tc.vw);
   const int head = c / CH, d0 = (c % CH) * 8;
   float4* out = reinterpret_cast<float4*>(pooled + (((size_t)b * g.Hh + head) * g.N + j) * D + d0);
   out[0] = make_float4(__fdiv_rn(acc[0], nvalid), __fdiv_rn(acc[1], nvalid), __fdiv_rn(acc[2], nvalid),
