@@ -82,9 +82,25 @@ def kept_pairs_from_counts(cnt: torch.Tensor) -> int:
     return int(cnt.to(torch.int64).sum().item())
 
 
-def pair_flops(head_dim: int) -> float:
-    # QK^T and PV on one 64x64 tile pair: 2 * (2 * 64 * 64 * D)
-    return 4.0 * 64 * 64 * head_dim
+def pair_flops(head_dim: int, volume: int = 64) -> float:
+    # QK^T and PV on one V x V tile pair: 2 * (2 * V * V * D)
+    return 4.0 * volume * volume * head_dim
+
+
+def chunk_real_table(wl, plan):
+    """[N, nchunk] bool: whether 64-row chunk c of tile j holds a real token
+    (its first row is inside the grid), as the attention kernel decides."""
+    import numpy as np
+
+    tt, th, tw = wl.tile
+    info = plan.info
+    nch = plan.V // 64
+    j = np.arange(plan.N)
+    t0, h0, w0 = (j // (info.nH * info.nW)) * tt, ((j // info.nW) % info.nH) * th, (j % info.nW) * tw
+    r = 64 * np.arange(nch)
+    dt, dh, dw = r // (th * tw), (r // tw) % th, r % tw
+    return ((t0[:, None] + dt[None, :] < wl.T) & (h0[:, None] + dh[None, :] < wl.H)
+            & (w0[:, None] + dw[None, :] < wl.W))
 
 
 def group_axes(wl):
@@ -95,13 +111,34 @@ def group_axes(wl):
 
 
 def group_accounting(wl, plan, idx: torch.Tensor, cnt: torch.Tensor):
-    """Work the attention kernel does beyond the kept pairs.
+    """Work the attention kernel does, in 64 x 64 chunk pairs.
 
-    Query tiles are stacked in pairs along one tile axis (one M = 128 block).
-    A pair loads each key tile in the union of its two lists once and
-    multiplies two tile pairs for it. Returns (MMA tile pairs, K/V tile loads).
+    64-token tiles: query tiles are stacked in pairs along one tile axis (one
+    M = 128 block); a pair loads each key tile in the union of its two lists
+    once and multiplies two tile pairs for it. Larger tiles: a block holds two
+    64-row chunks of one query tile (padding-only chunks left out, as the
+    layer's natural-layout kernel does) and loads every real chunk of each
+    kept key tile. Returns (MMA 64x64 chunk pairs, K/V chunk loads).
     """
     N = plan.N
+    if plan.V > 64:
+        import numpy as np
+
+        real = chunk_real_table(wl, plan)
+        nreal = real.sum(axis=1)
+        nq = real.reshape(N, -1)
+        blocks = np.zeros(N, dtype=np.int64)
+        for c in range(0, real.shape[1], 2):
+            pair = nq[:, c] | (nq[:, c + 1] if c + 1 < real.shape[1] else False)
+            blocks += pair
+        rows = cnt.numel()
+        kmax = idx.shape[-1]
+        ii = idx.reshape(rows, kmax).cpu().numpy()
+        cc = cnt.reshape(rows).cpu().numpy()
+        loads = 0
+        for r in range(rows):
+            loads += int(blocks[r % N]) * int(nreal[ii[r, :cc[r]]].sum())
+        return 2 * loads, loads
     rows = cnt.numel()
     kmax = idx.shape[-1]
     ii = idx.reshape(rows, kmax).to(torch.int64)
@@ -126,10 +163,16 @@ def group_accounting(wl, plan, idx: torch.Tensor, cnt: torch.Tensor):
     return int(pairs.sum().item()) * 2, int(pairs.sum().item())
 
 
+def layer_tiles_kv(plan) -> bool:
+    """Whether attn_layer re-tiles K and V (kept chunks loaded 64+ times)."""
+    nch = plan.V // 64
+    return plan.kmax * (1 if nch == 1 else (nch + 1) // 2) >= 64
+
+
 def launches_per_step(wl, plan) -> int:
     pooled = wl.rule != "window"
     quant = 2 if wl.qk_fp8 else 0  # e4m3 tile codes of Q and K
-    retile = 0 if plan.kmax < 64 else (1 if wl.qk_fp8 else 2)  # K and V (or V) re-tiled once
+    retile = 0 if not layer_tiles_kv(plan) else (1 if wl.qk_fp8 else 2)  # K and V (or V) re-tiled once
     return quant + (2 if pooled else 0) + retile + 1 + 1  # [pool Q+K, scores], select, attention
 
 
@@ -215,14 +258,14 @@ def oracle_sample(wl, seconds_target: float = 12.0):
     qn, kn, vn = cpu_inputs(wl)
     t0 = time.perf_counter()
     if wl.qk_fp8:
-        qn, kn, _, _ = attention.fp8_qk(qn, kn, wl.T, wl.H, wl.W)
+        qn, kn, _, _ = attention.fp8_qk(qn, kn, wl.T, wl.H, wl.W, wl.tile)
     _, _, _, lists = attention.route(qn, kn, wl.T, wl.H, wl.W, wl.rule, k=wl.k, p=wl.p,
-                                     half=wl.win)
+                                     half=wl.win, tile=wl.tile)
     N = len(lists)
     order = np.random.default_rng(0).permutation(N)
     pairs, done = 0, 0
     for i in order:
-        attention.attention_rows(qn, kn, vn, lists, wl.T, wl.H, wl.W, rows=[(0, 0, int(i))])
+        attention.attention_rows(qn, kn, vn, lists, wl.T, wl.H, wl.W, wl.tile, rows=[(0, 0, int(i))])
         pairs += len(lists[i])
         done += 1
         if time.perf_counter() - t0 > seconds_target:
@@ -230,7 +273,7 @@ def oracle_sample(wl, seconds_target: float = 12.0):
     secs = time.perf_counter() - t0
     text = (f"one head of {wl.heads}: routing over all {N} tiles, then attention of {done} of "
             f"{N} query tiles ({pairs} kept tile pairs), fp64 numpy")
-    return pairs * pair_flops(wl.head_dim), secs, text
+    return pairs * pair_flops(wl.head_dim, math.prod(wl.tile)), secs, text
 
 
 def run_reference(args):
@@ -317,7 +360,7 @@ def main():
     if bsattn.attn_check_device_status(plan) != 0:
         raise SystemExit("device error word set")
     kept = kept_pairs_from_counts(cnt)
-    flops = kept * pair_flops(wl.head_dim)
+    flops = kept * pair_flops(wl.head_dim, plan.V)
     issued, loads = group_accounting(wl, plan, idx, cnt)
 
     sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
@@ -366,6 +409,10 @@ def main():
     pk = peaks()
     attn_ms = comp["attention"]
     achieved = flops / (attn_ms * 1e-3) / 1e12
+    nch2 = (plan.V // 64) ** 2  # 64 x 64 chunk pairs per kept tile pair
+    # Tensor work the kernel issues (paired query tiles multiply some pairs
+    # nobody kept; tiles of several chunks skip chunks of padding only).
+    achieved_mma = issued * pair_flops(wl.head_dim) / (attn_ms * 1e-3) / 1e12
     line = {
         "metric": METRIC,
         "value": world * flops / (ms_per_step * 1e-3) / 1e12,
@@ -380,16 +427,18 @@ def main():
         "dtype": "bf16+e4m3" if wl.qk_fp8 else "bf16",
         "data": "synthetic",
         "config": workload_config(wl, {"kept_pairs": kept, "kept_tflop": flops / 1e12,
-                                        "mma_tile_pairs": issued,
-                                        "pair_efficiency": kept / issued if issued else None,
-                                        "kv_tile_loads": loads,
-                                        "kv_loads_per_kept_pair": loads / kept if kept else None,
+                                        "tile": list(wl.tile),
+                                        "mma_chunk_pairs": issued,
+                                        "pair_efficiency": kept * nch2 / issued if issued else None,
+                                        "kv_chunk_loads": loads,
+                                        "kv_loads_per_kept_chunk_pair": loads / (kept * nch2) if kept else None,
                                         "parallelism": f"independent layer per GPU x{world}"}),
         "ms_per_layer": ms_per_step,
         "kernels_ms": comp,
         "roofline": {"bound": "tensor", "kernel": "attention", "achieved": achieved,
                      "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": achieved / pk["bf16_tflops"],
+                     "achieved_mma": achieved_mma,
                      "peak_note": f"{pk['source']} bf16 burst (kernel timed alone)",
                      "traffic": measured_traffic(wl.name)},
         "memory_kernels": memory_kernel_rates(wl, plan, comp, pk),
@@ -429,9 +478,9 @@ def component_timing(bsattn, plan, wl, q, k, v, flush, stream, reps=20):
         codes = [torch.empty(plan.tiled_shape(), dtype=torch.uint8, device="cuda") for _ in range(2)]
         scales = [torch.empty((wl.B, wl.heads, plan.N), dtype=torch.float32, device="cuda")
                   for _ in range(2)]
-    # The layer re-tiles K and V once when kmax >= 64 (many loads per key
-    # tile); its attention then reads tiled K/V, timed here as attn_forward.
-    tiles_kv = plan.kmax >= 64
+    # The layer re-tiles K and V once a kept key chunk is loaded 64+ times;
+    # its attention then reads tiled K/V, timed here as attn_forward.
+    tiles_kv = layer_tiles_kv(plan)
     names = ["pool_qk", "reorder_qk", "quantize", "reorder_kv", "block_scores", "select", "attention",
              "attention_tiled", "attention_natural"]
     acc = {n: 0.0 for n in names}
@@ -488,7 +537,7 @@ def memory_kernel_rates(wl, plan, comp, pk):
     """Algorithmic bytes / time for the HBM-bound steps."""
     bh = wl.B * wl.heads
     nat = wl.B * wl.L * wl.heads * wl.head_dim * 2
-    til = bh * plan.N * 64 * wl.head_dim * 2
+    til = bh * plan.N * plan.V * wl.head_dim * 2
     pooled = bh * plan.N * wl.head_dim * 4
     out = {}
     if "pool_qk" in comp:
@@ -516,7 +565,7 @@ def e2e_timing(bsattn, plan, q, k, v, ws, idx, cnt, stream, steps=10, warmup=3, 
     ho = [torch.empty(q.shape, dtype=q.dtype, pin_memory=True) for _ in range(2)]
     dq = [[torch.empty_like(x) for x in (q, k, v)] for _ in range(2)]
     do = [torch.empty_like(q) for _ in range(2)]
-    flops_per = kept_pairs_from_counts(cnt) * pair_flops(plan.D)
+    flops_per = kept_pairs_from_counts(cnt) * pair_flops(plan.D, plan.V)
     s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
     s_comp = stream
 

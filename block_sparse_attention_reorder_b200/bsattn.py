@@ -142,6 +142,8 @@ class Plan:
         self.T, self.H, self.W = T, H, W
         self.L = T * H * W
         self.N = info.n_blocks
+        self.V = info.tile_volume
+        self.tile = tuple(tile)
         self.kmax = info.kmax
         self.qk_fp8 = bool(qk_fp8)
 
@@ -166,7 +168,7 @@ class Plan:
         return (self.B, self.L, self.heads, self.D)
 
     def tiled_shape(self):
-        return (self.B, self.heads, self.N, 64, self.D)
+        return (self.B, self.heads, self.N, self.V, self.D)
 
     def list_shapes(self):
         return (self.B, self.heads, self.N, self.kmax), (self.B, self.heads, self.N)
@@ -263,7 +265,7 @@ def attn_forward(plan: Plan, q, k, v, idx, cnt, o_tiled, lse=None, q_scale=None,
     _want(idx, torch.int32, si, "idx")
     _want(cnt, torch.int32, sc, "cnt")
     if lse is not None:
-        _want(lse, torch.float32, (plan.B, plan.heads, plan.N, 64), "lse")
+        _want(lse, torch.float32, (plan.B, plan.heads, plan.N, plan.V), "lse")
     wsb = 0 if ws is None else ws.numel() * ws.element_size()
     _check(_lib.attn_forward(plan.handle, _ptr(q), _ptr(k), _ptr(q_scale), _ptr(k_scale), _ptr(v),
                              _ptr(idx), _ptr(cnt), _ptr(o_tiled), _ptr(lse), _ptr(ws), wsb,

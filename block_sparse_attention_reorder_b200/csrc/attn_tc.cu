@@ -1,15 +1,18 @@
 // Block-sparse attention forward over kept tile pairs on the 5th-generation
 // tensor cores (tcgen05, TMEM accumulators, TMA-fed shared memory).
 //
-// Work unit: two adjacent query tiles i0, i1 of one (batch, head), next to
-// each other along one axis of the tile grid (w for top-k / top-p, t for a
-// window that does not reach along w), stacked into one 128-row query
-// block so that every QK^T and PV
-// product is an M = 128 tcgen05.mma. The block walks the union of the two
-// tiles' kept key-tile lists in ascending order; a key tile kept by only one
-// of the two query tiles gives zero probabilities to the other tile's rows.
-// Adjacent query tiles of a smooth video latent keep mostly the same key
-// tiles, so little work is wasted.
+// Work unit: a 128-row query block of two 64-row chunks, so that every QK^T
+// and PV product is an M = 128 tcgen05.mma, and a step is one 64-key chunk.
+// Tiles of 64 tokens (one chunk): the block stacks two adjacent query tiles
+// i0, i1 of one (batch, head), next to each other along one axis of the tile
+// grid (w for top-k / top-p, t for a window that does not reach along w),
+// and walks the union of their kept key-tile lists in ascending order; a key
+// tile kept by only one of the two gives zero probabilities to the other
+// tile's rows. Adjacent query tiles of a smooth video latent keep mostly the
+// same key tiles, so little work is wasted. Larger tiles (64 * c tokens):
+// the block holds chunks 2b and 2b + 1 of one query tile, which keep the
+// same key tiles, and walks every chunk of each kept key tile that holds a
+// real token; nothing is wasted.
 //
 // Roles (192 threads):
 //   warps 0-3  softmax: thread r owns query row r (TMEM lane r). Per key
@@ -131,12 +134,36 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   uint32_t* bmA = reinterpret_cast<uint32_t*>(smem + C::OFF_DYN);
   uint32_t* bmB = bmA + P.bm_words;
   uint32_t* ulist = bmB + P.bm_words;
+  uint32_t* uorg = ulist + P.umax;  // packed first-token offsets of the steps' key chunks
 
   const Geom& g = P.g;
-  // Work item -> its two member tiles along the pair axis (i1 = -1 at an
-  // odd grid edge).
-  int i0, i1;
-  {
+  const int nchunk = g.nchunk;
+  // Whether chunk c of tile j holds a real token (its first row, the box's
+  // lowest corner, is inside the grid).
+  auto chunk_real = [&](int j, int c) -> bool {
+    const ChunkOrigin o = chunk_origin(g, c);
+    const int bt = j / (g.nH * g.nW), bhh = (j / g.nW) % g.nH, bw = j % g.nW;
+    return bt * g.tt + o.dt < g.T && bhh * g.th + o.dh < g.H && bw * g.tw + o.dw < g.W;
+  };
+  // Work item -> its two member (tile, chunk) halves; i1 = -1 when the
+  // second half is absent (odd grid edge, odd chunk count; with natural
+  // output also a chunk of padded rows only, which that output never holds).
+  int i0, i1, c0 = 0, c1 = 0;
+  if (nchunk > 1) {
+    const int per = (nchunk + 1) / 2;
+    i0 = i1 = blockIdx.x / per;
+    c0 = 2 * (blockIdx.x % per);
+    c1 = c0 + 1;
+    if (c1 >= nchunk) i1 = -1;
+    if (NQO) {
+      if (i1 >= 0 && !chunk_real(i1, c1)) i1 = -1;
+      if (!chunk_real(i0, c0)) {
+        if (i1 < 0) return;  // uniform over the CTA, before any setup
+        c0 = c1;
+        i1 = -1;
+      }
+    }
+  } else {
     const int nd[3] = {g.nT, g.nH, g.nW};
     int c[3], rem = blockIdx.x;
     c[2] = rem % P.pdim[2];
@@ -151,13 +178,23 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   const int head = blockIdx.y, b = blockIdx.z;
   const size_t bh = (size_t)b * g.Hh + head;
   const bool has1 = i1 >= 0;
-  // One tile (64 tokens x 64 columns) of a natural-layout tensor: the box
-  // {64 columns, tw, th, tt, 1} at the tile's first token, rows in (t, h, w)
-  // order like the tiled layout; tokens past the grid's edge read as zero.
-  auto load_nat = [&](uint32_t dst, const CUtensorMap* map, uint32_t bar, int col, int tile) {
+  // One chunk (64 tokens x 64 columns) of a natural-layout tensor: the box
+  // {64 columns, cw, ch, ct, 1} at the chunk's first token (tile origin plus
+  // the chunk's in-tile offset o), rows in (t, h, w) order like the tiled
+  // layout; tokens past the grid's edge read as zero.
+  auto load_nat = [&](uint32_t dst, const CUtensorMap* map, uint32_t bar, int col, int tile, ChunkOrigin o) {
     const int bt = tile / (g.nH * g.nW), bhh = (tile / g.nW) % g.nH, bw = tile % g.nW;
-    tc::tma_load_5d(dst, map, bar, col, bw * g.tw, bhh * g.th, bt * g.tt, b);
+    tc::tma_load_5d(dst, map, bar, col, bw * g.tw + o.dw, bhh * g.th + o.dh, bt * g.tt + o.dt, b);
   };
+  // In-tile offset of a step's key chunk (packed 10 bits per axis; zero for
+  // one-chunk tiles).
+  auto step_origin = [&](int n) -> ChunkOrigin {
+    if (nchunk == 1) return ChunkOrigin{0, 0, 0};
+    const uint32_t v = uorg[n];
+    return ChunkOrigin{(int)(v & 0x3FFu), (int)((v >> 10) & 0x3FFu), (int)(v >> 20)};
+  };
+  // First tiled-layout row of chunk c of tile j.
+  auto tiled_row = [&](int j, int c) -> int { return (int)((bh * g.N + j) * g.V) + 64 * c; };
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   // ------------------------------------------------------------ setup
@@ -183,8 +220,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     tc::tmem_alloc(sb + C::OFF_MISC, kTmemCols);
     tc::tmem_relinquish();
   }
-  if (tid < 64) {
-    int dt = tid / (g.th * g.tw), dh = (tid / g.tw) % g.th, dw = tid % g.tw;
+  if (tid < 64) {  // in-chunk (t, h, w) offsets of each chunk row
+    int dt = tid / (g.ch * g.cw), dh = (tid / g.cw) % g.ch, dw = tid % g.cw;
     colc[tid] = (uint32_t)dt | ((uint32_t)dh << 8) | ((uint32_t)dw << 16);
   }
   for (int w = tid; w < 2 * P.bm_words; w += kThreads) bmA[w] = 0u;
@@ -199,7 +236,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   }
   __syncthreads();
 
-  // Union of the two kept lists as a bitmap pair, then compacted ascending.
+  // Union of the two kept lists as a bitmap pair, then compacted ascending
+  // into the step list: one entry per real 64-key chunk of each kept key
+  // tile, key tile in bits 0-20, chunk in bits 21-29, bit 30 (31) set when
+  // the first (second) query half keeps the tile.
   int nA = P.cnt[bh * g.N + i0];
   int nB = has1 ? P.cnt[bh * g.N + i1] : 0;
   if (nA < 0 || nA > P.kmax || nB < 0 || nB > P.kmax) {
@@ -223,8 +263,23 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   {
     const int wpt = (P.bm_words + kThreads - 1) / kThreads;
     const int w0 = min(tid * wpt, P.bm_words), w1 = min(w0 + wpt, P.bm_words);
+    auto real_chunks = [&](int j) -> int {
+      int n = 0;
+      for (int c = 0; c < nchunk; ++c) n += chunk_real(j, c) ? 1 : 0;
+      return n;
+    };
     int mine = 0;
-    for (int w = w0; w < w1; ++w) mine += __popc(bmA[w] | bmB[w]);
+    for (int w = w0; w < w1; ++w) {
+      uint32_t bits = bmA[w] | bmB[w];
+      if (nchunk == 1) {
+        mine += __popc(bits);
+      } else {
+        while (bits) {
+          mine += real_chunks(w * 32 + __ffs(bits) - 1);
+          bits &= bits - 1;
+        }
+      }
+    }
     int x = mine;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -245,9 +300,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       while (bits) {
         int bit = __ffs(bits) - 1;
         bits &= bits - 1;
-        uint32_t e = (uint32_t)(w * 32 + bit) | (((a >> bit) & 1u) << 30) | (((bb >> bit) & 1u) << 31);
-        if (pos < P.umax) ulist[pos] = e;
-        ++pos;
+        const int j = w * 32 + bit;
+        const uint32_t e = (uint32_t)j | (((a >> bit) & 1u) << 30) | (((bb >> bit) & 1u) << 31);
+        for (int c = 0; c < nchunk; ++c) {
+          if (nchunk > 1 && !chunk_real(j, c)) continue;
+          if (pos < P.umax) {
+            ulist[pos] = e | ((uint32_t)c << 21);
+            if (nchunk > 1) {
+              const ChunkOrigin o = chunk_origin(g, c);
+              uorg[pos] = (uint32_t)o.dt | ((uint32_t)o.dh << 10) | ((uint32_t)o.dw << 20);
+            }
+          }
+          ++pos;
+        }
       }
     }
     if (tid == 0) misc[2] = (uint32_t)min(tot, P.umax);
@@ -266,14 +331,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       tc::tma_prefetch_desc(&tmV);
       tc::mbar_arrive_expect_tx(bar_q, (has1 ? 2 : 1) * 64 * C::QRB);
       for (int x = 0; x < (has1 ? 2 : 1); ++x) {
-        const int tile = x ? i1 : i0;
+        const int tile = x ? i1 : i0, chunk = x ? c1 : c0;
 #pragma unroll
         for (int cb = 0; cb < C::QBLK; ++cb) {
           const uint32_t dst = sb + C::OFF_Q + cb * 128 * C::SWB + x * 64 * C::SWB;
           if (NQO && !FP8)
-            load_nat(dst, &tmQ, bar_q, head * D + cb * 64, tile);
+            load_nat(dst, &tmQ, bar_q, head * D + cb * 64, tile, chunk_origin(g, chunk));
           else
-            tc::tma_load_2d(dst, &tmQ, bar_q, cb * C::SWB / C::ESZ, (int)((bh * g.N + tile) * 64));
+            tc::tma_load_2d(dst, &tmQ, bar_q, cb * C::SWB / C::ESZ, tiled_row(tile, chunk));
         }
       }
       // K_m is issued as soon as S_{m-2} has released its slot, V_{m-1} once
@@ -290,15 +355,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             record_timeout(abort_flag, P.err);
             break;
           }
-          const int kt = (int)(ulist[m] & 0x3FFFFFFFu);
+          const int kt = (int)(ulist[m] & 0x1FFFFFu), kc = (int)((ulist[m] >> 21) & 0x1FFu);
           tc::mbar_arrive_expect_tx(bar_kfull(s), C::K_BYTES);
 #pragma unroll
           for (int cb = 0; cb < C::QBLK; ++cb) {
             const uint32_t dst = sb + C::OFF_K + s * C::K_BYTES + cb * 64 * C::SWB;
             if (NKV && !FP8)
-              load_nat(dst, &tmK, bar_kfull(s), head * D + cb * 64, kt);
+              load_nat(dst, &tmK, bar_kfull(s), head * D + cb * 64, kt, step_origin(m));
             else
-              tc::tma_load_2d(dst, &tmK, bar_kfull(s), cb * C::SWB / C::ESZ, (int)((bh * g.N + kt) * 64));
+              tc::tma_load_2d(dst, &tmK, bar_kfull(s), cb * C::SWB / C::ESZ, tiled_row(kt, kc));
           }
           lastk[s] = m;
         }
@@ -309,15 +374,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             record_timeout(abort_flag, P.err);
             break;
           }
-          const int vt = (int)(ulist[v] & 0x3FFFFFFFu);
+          const int vt = (int)(ulist[v] & 0x1FFFFFu), vc = (int)((ulist[v] >> 21) & 0x1FFu);
           tc::mbar_arrive_expect_tx(bar_vfull(s), C::V_BYTES);
 #pragma unroll
           for (int vb = 0; vb < C::VBLK; ++vb) {
             const uint32_t dst = sb + C::OFF_V + s * C::V_BYTES + vb * 8192;
             if (NKV)
-              load_nat(dst, &tmV, bar_vfull(s), head * D + vb * 64, vt);
+              load_nat(dst, &tmV, bar_vfull(s), head * D + vb * 64, vt, step_origin(v));
             else
-              tc::tma_load_2d(dst, &tmV, bar_vfull(s), vb * 64, (int)((bh * g.N + vt) * 64));
+              tc::tma_load_2d(dst, &tmV, bar_vfull(s), vb * 64, tiled_row(vt, vc));
           }
           lastv[s] = v;
         }
@@ -399,7 +464,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     bool ok = true;
     for (int n = 0; n < L; ++n) {
       const uint32_t e = ulist[n];
-      const int j = (int)(e & 0x3FFFFFFFu);
+      const int j = (int)(e & 0x1FFFFFu);
       const bool keep = ((e >> (30 + half)) & 1u) != 0;  // uniform within the warp
       if (!__all_sync(0xffffffffu, tc::mbar_wait(bar_sfull(n & 1), (n >> 1) & 1, abort_flag, kWaitLimit))) {
         ok = false;
@@ -415,9 +480,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         tc::tmem_ld64_wait(sbuf, sr);
         const float c = P.scale_log2 * (FP8 ? qsc * __ldg(P.ks + bh * g.N + j) : 1.f);
         const int bt = j / (g.nH * g.nW), bhh = (j / g.nW) % g.nH, bw = j % g.nW;
-        const int vt = g.T - bt * g.tt, vh = g.H - bhh * g.th, vw = g.W - bw * g.tw;
-        const bool edge = vt < g.tt || vh < g.th || vw < g.tw;
-        if (edge) {  // padded keys of an edge tile
+        const ChunkOrigin ko = step_origin(n);
+        // Real extent of the key chunk along each axis, from its first token.
+        const int vt = g.T - bt * g.tt - ko.dt, vh = g.H - bhh * g.th - ko.dh, vw = g.W - bw * g.tw - ko.dw;
+        const bool edge = vt < g.ct || vh < g.ch || vw < g.cw;
+        if (edge) {  // padded keys of an edge chunk
 #pragma unroll
           for (int q = 0; q < 64; ++q) {
             const uint32_t cc = colc[q];
@@ -483,12 +550,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         }
         tc::fence_after_sync();
 #pragma unroll
-        for (int c0 = 0; c0 < D; c0 += 32) {
+        for (int col = 0; col < D; col += 32) {
           uint32_t o[32];
-          tc::tmem_ld32_wait(tmem + lane_base + kColO + c0, o);
+          tc::tmem_ld32_wait(tmem + lane_base + kColO + col, o);
 #pragma unroll
           for (int q = 0; q < 32; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * alpha);
-          tc::tmem_st32(tmem + lane_base + kColO + c0, o);
+          tc::tmem_st32(tmem + lane_base + kColO + col, o);
         }
       }
       tc::tmem_wait_st();
@@ -508,10 +575,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const float inv = l > 0.f ? 1.f / l : 0.f;
     uint8_t* stage = smem + C::OFF_K + r * C::O_PITCH;
 #pragma unroll
-    for (int c0 = 0; c0 < D; c0 += 32) {
+    for (int col = 0; col < D; col += 32) {
       uint32_t o[32];
       if (ok && L > 0) {
-        tc::tmem_ld32_wait(tmem + lane_base + kColO + c0, o);
+        tc::tmem_ld32_wait(tmem + lane_base + kColO + col, o);
       } else {
 #pragma unroll
         for (int q = 0; q < 32; ++q) o[q] = 0u;
@@ -523,14 +590,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         w[q] = pack_bf16x2(__uint_as_float(o[2 * q]) * inv, __uint_as_float(o[2 * q + 1]) * inv, dummy);
 #pragma unroll
       for (int q = 0; q < 4; ++q)
-        reinterpret_cast<uint4*>(stage + c0 * 2)[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+        reinterpret_cast<uint4*>(stage + col * 2)[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
     }
     // Token of row rr of the block (natural layout), -1 for a padded slot.
+    const ChunkOrigin qo0 = chunk_origin(g, c0), qo1 = chunk_origin(g, c1);
     auto token_of = [&](int rr) -> int {
       const int tile = rr >> 6 ? i1 : i0, q = rr & 63;
-      const int t = (tile / (g.nH * g.nW)) * g.tt + q / (g.th * g.tw);
-      const int h = ((tile / g.nW) % g.nH) * g.th + (q / g.tw) % g.th;
-      const int w = (tile % g.nW) * g.tw + q % g.tw;
+      const ChunkOrigin o = rr >> 6 ? qo1 : qo0;
+      const int t = (tile / (g.nH * g.nW)) * g.tt + o.dt + q / (g.ch * g.cw);
+      const int h = ((tile / g.nW) % g.nH) * g.th + o.dh + (q / g.cw) % g.ch;
+      const int w = (tile % g.nW) * g.tw + o.dw + q % g.cw;
       return (t < g.T && h < g.H && w < g.W) ? (t * g.H + h) * g.W + w : -1;
     };
     const float lse_r = l > 0.f ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
@@ -539,7 +608,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         const int n = token_of(r);
         if (n >= 0) P.lse[bh * (size_t)g.L + n] = lse_r;
       } else {
-        P.lse[(bh * g.N + (half ? i1 : i0)) * 64 + (r & 63)] = lse_r;
+        P.lse[(size_t)tiled_row(half ? i1 : i0, half ? c1 : c0) + (r & 63)] = lse_r;
       }
     }
     asm volatile("bar.sync 1, 128;" ::: "memory");
@@ -553,7 +622,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         if (n >= 0)
           reinterpret_cast<uint4*>(P.o + (((size_t)b * g.L + n) * g.Hh + head) * D)[cc] = val;
       } else {
-        uint4* og = reinterpret_cast<uint4*>(P.o + (bh * g.N + (rr >> 6 ? i1 : i0)) * 64 * (size_t)D);
+        uint4* og = reinterpret_cast<uint4*>(P.o + (size_t)tiled_row(rr >> 6 ? i1 : i0, rr >> 6 ? c1 : c0) * D);
         og[(rr & 63) * CPR + cc] = val;
       }
     }
@@ -605,7 +674,7 @@ bool make_map_nat(CUtensorMap* map, const void* base, const bsattn_plan* p) {
   cuuint64_t dims[5] = {(cuuint64_t)d.heads * d.head_dim, (cuuint64_t)d.W, (cuuint64_t)d.H, (cuuint64_t)d.T,
                         (cuuint64_t)d.B};
   cuuint64_t strides[4] = {row, row * d.W, row * d.W * d.H, row * d.W * d.H * d.T};
-  cuuint32_t box[5] = {64, (cuuint32_t)d.tile_w, (cuuint32_t)d.tile_h, (cuuint32_t)d.tile_t, 1};
+  cuuint32_t box[5] = {64, (cuuint32_t)p->cw, (cuuint32_t)p->ch, (cuuint32_t)p->ct, 1};  // one chunk
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -617,7 +686,7 @@ template <int D, bool FP8, bool NQO, bool NKV>
 bsattn_status run(const bsattn_plan* p, const void* q, const void* k, const __nv_bfloat16* v,
                   TcParams prm, cudaStream_t st) {
   using C = Cfg<D, FP8>;
-  const uint64_t rows = (uint64_t)p->desc.B * p->desc.heads * p->N * 64;
+  const uint64_t rows = (uint64_t)p->desc.B * p->desc.heads * p->N * p->V;
   if (rows + 128 >= (1ull << 31)) return BSATTN_ERR_UNSUPPORTED;
   CUtensorMap mq, mk, mv;
   const CUtensorMapDataType dqk = FP8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
@@ -629,13 +698,14 @@ bsattn_status run(const bsattn_plan* p, const void* q, const void* k, const __nv
   if (NKV ? !make_map_nat(&mv, v, p)
           : !make_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, rows, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B))
     return BSATTN_ERR_CUDA;
-  size_t smem = 1024 + C::OFF_DYN + (size_t)prm.bm_words * 8 + (size_t)prm.umax * 4;
+  size_t smem = 1024 + C::OFF_DYN + (size_t)prm.bm_words * 8 + (size_t)prm.umax * (p->nchunk > 1 ? 8 : 4);
   if (smem < 80 * 1024) smem = 80 * 1024;  // at most two CTAs (2 x 256 TMEM columns) per SM
   if (smem > 227 * 1024) return BSATTN_ERR_UNSUPPORTED;
   auto kern = attn_tc_kernel<D, FP8, NQO, NKV>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return BSATTN_ERR_CUDA;
-  dim3 grid(prm.pdim[0] * prm.pdim[1] * prm.pdim[2], p->desc.heads, p->desc.B);
+  const int items = p->nchunk > 1 ? p->N * ((p->nchunk + 1) / 2) : prm.pdim[0] * prm.pdim[1] * prm.pdim[2];
+  dim3 grid(items, p->desc.heads, p->desc.B);
   kern<<<grid, kThreads, smem, st>>>(mq, mk, mv, prm);
   return cudaGetLastError() == cudaSuccess ? BSATTN_OK : BSATTN_ERR_CUDA;
 }
@@ -660,7 +730,10 @@ bsattn_status launch_attention(const bsattn_plan* p, const void* q, const void* 
   prm.lse = lse;
   prm.scale_log2 = p->scale * 1.4426950408889634f;
   prm.err = p->d_err;
-  prm.umax = p->N < 2 * p->kmax ? p->N : 2 * p->kmax;
+  // Step-list capacity: the union of two lists of one-chunk tiles, or one
+  // list of tiles times their chunks.
+  prm.umax = p->nchunk == 1 ? (p->N < 2 * p->kmax ? p->N : 2 * p->kmax)
+                            : (p->N < p->kmax ? p->N : p->kmax) * p->nchunk;
   prm.bm_words = (p->N + 31) / 32;
   // Pairs along w for top-k / top-p (neighbouring query tiles keep similar
   // key tiles); along t for a window that does not reach along w, whose

@@ -19,6 +19,8 @@ struct bsattn_plan {
   bsattn_rule rule;
   int device;
   int Tp, Hp, Wp, nT, nH, nW, N, V, L, kmax;
+  int nchunk;          // 64-row chunks per tile (V / 64)
+  int ct, ch, cw;      // box of one chunk (t, h, w): ct * ch * cw = 64
   float scale;
   int* d_err;        // device error word
   int32_t* d_win_idx;  // window rule: [N, kmax]
@@ -26,12 +28,27 @@ struct bsattn_plan {
 };
 
 // Geometry passed by value to kernels.
+// Largest supported tile: 512 chunks of 64 tokens.
+constexpr int kMaxChunks = 512;
+
+// A tile holds V = 64 * nchunk tokens in (dt, dh, dw) row-major order; its
+// rows [64c, 64c + 64) form chunk c, which is the box (ct, ch, cw) of the
+// tile starting at in-tile coordinates chunk_origin(c).
 struct Geom {
   int B, Hh, D;
   int T, H, W;
   int tt, th, tw;
   int nT, nH, nW, N, L;
+  int V, nchunk, ct, ch, cw;
 };
+
+struct ChunkOrigin {
+  int dt, dh, dw;
+};
+__host__ __device__ __forceinline__ ChunkOrigin chunk_origin(const Geom& g, int c) {
+  const int r = 64 * c;
+  return ChunkOrigin{r / (g.th * g.tw), (r / g.tw) % g.th, r % g.tw};
+}
 
 static inline Geom make_geom(const bsattn_plan* p) {
   Geom g;
@@ -39,6 +56,7 @@ static inline Geom make_geom(const bsattn_plan* p) {
   g.T = p->desc.T; g.H = p->desc.H; g.W = p->desc.W;
   g.tt = p->desc.tile_t; g.th = p->desc.tile_h; g.tw = p->desc.tile_w;
   g.nT = p->nT; g.nH = p->nH; g.nW = p->nW; g.N = p->N; g.L = p->L;
+  g.V = p->V; g.nchunk = p->nchunk; g.ct = p->ct; g.ch = p->ch; g.cw = p->cw;
   return g;
 }
 
@@ -83,8 +101,12 @@ bsattn_status launch_attention(const bsattn_plan* p, const void* q, const void* 
                                const int32_t* idx, const int32_t* cnt, __nv_bfloat16* o,
                                float* lse, void* ws, size_t ws_bytes, cudaStream_t st,
                                AttnLayout lay);
-// Whether attn_layer re-tiles K and V: natural tile loads cost more per load
-// than tiled ones, which outweighs the one-off reorder once a key tile is
-// loaded about 40+ times (kmax >= 64).
-static inline bool layer_tiles_kv(const bsattn_plan* p) { return p->kmax >= 64; }
+// Whether attn_layer re-tiles K and V: natural chunk loads cost more per load
+// than tiled ones, which outweighs the one-off reorder once a key chunk is
+// loaded about 40+ times: kmax >= 64 with one-chunk tiles (two query tiles
+// per block), kmax * ceil(nchunk / 2) >= 64 otherwise (every block of a query
+// tile loads each kept chunk).
+static inline bool layer_tiles_kv(const bsattn_plan* p) {
+  return (long long)p->kmax * (p->nchunk == 1 ? 1 : (p->nchunk + 1) / 2) >= 64;
+}
 size_t attention_workspace_bytes(const bsattn_plan* p);

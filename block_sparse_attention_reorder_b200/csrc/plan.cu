@@ -105,6 +105,25 @@ const char* attn_status_string(bsattn_status s) {
   return "unknown status";
 }
 
+// Box (ct, ch, cw) of 64 tokens covering in-tile rows [64c, 64c + 64) of a
+// (tt, th, tw) tile in (dt, dh, dw) row-major order, if those rows form a box
+// for every c: whole (dh, dw) planes, whole dw rows, or 64-wide dw runs.
+static bool chunk_box(int tt, int th, int tw, int* ct, int* ch, int* cw) {
+  if (th * tw <= 64) {
+    if (64 % (th * tw) != 0 || tt % (64 / (th * tw)) != 0) return false;
+    *ct = 64 / (th * tw); *ch = th; *cw = tw;
+    return true;
+  }
+  if (tw <= 64) {
+    if (64 % tw != 0 || th % (64 / tw) != 0) return false;
+    *ct = 1; *ch = 64 / tw; *cw = tw;
+    return true;
+  }
+  if (tw % 64 != 0) return false;
+  *ct = 1; *ch = 1; *cw = 64;
+  return true;
+}
+
 bsattn_status attn_plan_create(const bsattn_desc* d, const bsattn_rule* r, bsattn_plan** out) {
   if (!d || !r || !out) return BSATTN_ERR_INVALID_ARG;
   *out = nullptr;
@@ -112,7 +131,14 @@ bsattn_status attn_plan_create(const bsattn_desc* d, const bsattn_rule* r, bsatt
       d->tile_h < 1 || d->tile_w < 1 || d->head_dim < 1)
     return BSATTN_ERR_INVALID_ARG;
   if (d->head_dim != 64 && d->head_dim != 128) return BSATTN_ERR_UNSUPPORTED;
-  if (d->tile_t * d->tile_h * d->tile_w != 64) return BSATTN_ERR_UNSUPPORTED;
+  // Tiles of 64 * nchunk tokens whose 64-row chunks are boxes of the tile.
+  int ct, ch, cw;
+  {
+    const long long vol = (long long)d->tile_t * d->tile_h * d->tile_w;
+    if (vol % 64 != 0 || vol > 64LL * kMaxChunks) return BSATTN_ERR_UNSUPPORTED;
+    if (d->tile_t > 1024 || d->tile_h > 1024 || d->tile_w > 1024) return BSATTN_ERR_UNSUPPORTED;
+    if (!chunk_box(d->tile_t, d->tile_h, d->tile_w, &ct, &ch, &cw)) return BSATTN_ERR_UNSUPPORTED;
+  }
   if (d->qk_fp8 != 0 && d->qk_fp8 != 1) return BSATTN_ERR_INVALID_ARG;
   long long Tp = (d->T + d->tile_t - 1) / d->tile_t * (long long)d->tile_t;
   long long Hp = (d->H + d->tile_h - 1) / d->tile_h * (long long)d->tile_h;
@@ -120,6 +146,8 @@ bsattn_status attn_plan_create(const bsattn_desc* d, const bsattn_rule* r, bsatt
   long long N = (Tp / d->tile_t) * (Hp / d->tile_h) * (Wp / d->tile_w);
   long long L = (long long)d->T * d->H * d->W;
   if (N > (1 << 20) || L > (1LL << 30) / d->heads) return BSATTN_ERR_UNSUPPORTED;
+  // Tiled row coordinates (B * heads * Tp * Hp * Wp rows) stay within int32.
+  if ((long long)d->B * d->heads * Tp * Hp * Wp >= (1LL << 31)) return BSATTN_ERR_UNSUPPORTED;
 
   int kmax = 0;
   switch (r->kind) {
@@ -150,7 +178,10 @@ bsattn_status attn_plan_create(const bsattn_desc* d, const bsattn_rule* r, bsatt
   p->rule = *r;
   p->Tp = (int)Tp; p->Hp = (int)Hp; p->Wp = (int)Wp;
   p->nT = (int)(Tp / d->tile_t); p->nH = (int)(Hp / d->tile_h); p->nW = (int)(Wp / d->tile_w);
-  p->N = (int)N; p->V = 64; p->L = (int)L; p->kmax = kmax;
+  p->N = (int)N; p->L = (int)L; p->kmax = kmax;
+  p->V = d->tile_t * d->tile_h * d->tile_w;
+  p->nchunk = p->V / 64;
+  p->ct = ct; p->ch = ch; p->cw = cw;
   p->scale = d->softmax_scale > 0.f ? d->softmax_scale : (float)(1.0 / sqrt((double)d->head_dim));
   if (cudaGetDevice(&p->device) != cudaSuccess) { delete p; return BSATTN_ERR_CUDA; }
   if (cudaMalloc(&p->d_err, sizeof(int)) != cudaSuccess) { delete p; return BSATTN_ERR_CUDA; }

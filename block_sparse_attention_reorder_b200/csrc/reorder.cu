@@ -1,10 +1,13 @@
 // Tile reorder (natural -> tiled) with fused per-tile e4m3 quantisation, the
 // inverse scatter, standalone tile quantisation, and tile-mean pooling.
 //
-// These steps move bytes: one CTA per (batch, head, tile) moves the tile's
-// 64 rows of D bf16 with 16-byte vector accesses. Reads are 64 row segments
-// of 2*D bytes (the natural layout interleaves heads), writes are one
-// contiguous 64*D*2-byte block, so both sides use full 32-byte sectors.
+// These steps move bytes: one CTA per (batch, head, 64-row chunk of a tile)
+// moves the chunk's 64 rows of D bf16 with 16-byte vector accesses. Reads are
+// 64 row segments of 2*D bytes (the natural layout interleaves heads), writes
+// are one contiguous 64*D*2-byte block, so both sides use full 32-byte
+// sectors. e4m3 quantisation needs the whole tile's amax: with one chunk per
+// tile the values stay in registers, with several a CTA takes the tile and
+// reads it twice (the second time mostly from L2).
 #include <cuda_fp8.h>
 
 #include "internal.h"
@@ -85,17 +88,18 @@ reorder_kernel(Geom g, const __nv_bfloat16* __restrict__ x_nat, __nv_bfloat16* _
   constexpr int RSTEP = kThreads / CH;      // row stride between a thread's chunks
   __shared__ float wred[kThreads / 32];
 
-  const int j = blockIdx.x, head = blockIdx.y, b = blockIdx.z;
+  const int j = blockIdx.x / g.nchunk, head = blockIdx.y, b = blockIdx.z;
   const int c = threadIdx.x % CH;
   const int r0 = threadIdx.x / CH;
   const TileCoord tc = tile_coord(g, j);
-  const size_t tile_off = (((size_t)b * g.Hh + head) * g.N + j) * 64;
+  const int row0 = 64 * (blockIdx.x % g.nchunk);  // first in-tile row of the chunk
+  const size_t tile_off = (((size_t)b * g.Hh + head) * g.N + j) * g.V + row0;
 
   uint4 v[ITER];
 #pragma unroll
   for (int i = 0; i < ITER; ++i) {
     int r = r0 + RSTEP * i;
-    int n = row_token(g, tc, r);
+    int n = row_token(g, tc, row0 + r);
     if (n >= 0) {
       const uint4* src = reinterpret_cast<const uint4*>(x_nat + (((size_t)b * g.L + n) * g.Hh + head) * D) + c;
       v[i] = __ldg(src);
@@ -138,21 +142,22 @@ unreorder_kernel(Geom g, const __nv_bfloat16* __restrict__ x_tiled, __nv_bfloat1
   constexpr int CH = D / 8;
   constexpr int ITER = 64 * CH / kThreads;
   constexpr int RSTEP = kThreads / CH;
-  const int j = blockIdx.x, head = blockIdx.y, b = blockIdx.z;
+  const int j = blockIdx.x / g.nchunk, head = blockIdx.y, b = blockIdx.z;
   const int c = threadIdx.x % CH;
   const int r0 = threadIdx.x / CH;
   const TileCoord tc = tile_coord(g, j);
-  const size_t tile_off = (((size_t)b * g.Hh + head) * g.N + j) * 64;
+  const int row0 = 64 * (blockIdx.x % g.nchunk);
+  const size_t tile_off = (((size_t)b * g.Hh + head) * g.N + j) * g.V + row0;
 #pragma unroll
   for (int i = 0; i < ITER; ++i) {
     int r = r0 + RSTEP * i;
-    int n = row_token(g, tc, r);
+    int n = row_token(g, tc, row0 + r);
     if (n < 0) continue;
     uint4 v = __ldg(reinterpret_cast<const uint4*>(x_tiled + (tile_off + r) * D) + c);
     reinterpret_cast<uint4*>(x_nat + (((size_t)b * g.L + n) * g.Hh + head) * D)[c] = v;
   }
   if (lse_tiled && threadIdx.x < 64) {
-    int n = row_token(g, tc, threadIdx.x);
+    int n = row_token(g, tc, row0 + threadIdx.x);
     if (n >= 0) lse_nat[((size_t)b * g.Hh + head) * g.L + n] = lse_tiled[tile_off + threadIdx.x];
   }
 }
@@ -187,6 +192,61 @@ quant_tiled_kernel(Geom g, const __nv_bfloat16* __restrict__ x_tiled, uint8_t* _
   if (threadIdx.x == 0) scales[tile] = scale;
 }
 
+// e4m3 codes of tiles of several chunks: pass 1 takes the tile's amax, pass 2
+// reads the tile again and writes the codes (and, for NAT sources with
+// x_tiled set, the tiled bf16 copy). NAT: the source is the natural layout
+// (padded rows read as zero); else it is the tiled bf16 layout.
+template <int D, bool NAT>
+__global__ void __launch_bounds__(kThreads)
+quant_multi_kernel(Geom g, const __nv_bfloat16* __restrict__ src, __nv_bfloat16* __restrict__ x_tiled,
+                   uint8_t* __restrict__ codes, float* __restrict__ scales) {
+  constexpr int CH = D / 8;
+  constexpr int ITER = 64 * CH / kThreads;
+  constexpr int RSTEP = kThreads / CH;
+  __shared__ float wred[kThreads / 32];
+  const int j = blockIdx.x, head = blockIdx.y, b = blockIdx.z;
+  const int c = threadIdx.x % CH;
+  const int r0 = threadIdx.x / CH;
+  const TileCoord tc = tile_coord(g, j);
+  const size_t tile = ((size_t)b * g.Hh + head) * g.N + j;
+  auto load = [&](int r) -> uint4 {
+    if (NAT) {
+      const int n = row_token(g, tc, r);
+      if (n < 0) return make_uint4(0, 0, 0, 0);
+      return __ldg(reinterpret_cast<const uint4*>(src + (((size_t)b * g.L + n) * g.Hh + head) * D) + c);
+    }
+    return __ldg(reinterpret_cast<const uint4*>(src + (tile * g.V + r) * D) + c);
+  };
+  float m = 0.f;
+  for (int row0 = 0; row0 < g.V; row0 += 64) {
+    uint4 v[ITER];
+#pragma unroll
+    for (int i = 0; i < ITER; ++i) v[i] = load(row0 + r0 + RSTEP * i);
+#pragma unroll
+    for (int i = 0; i < ITER; ++i) {
+      float f[8];
+      bf16x8_to_f32(v[i], f);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(f[e]));
+    }
+  }
+  const float scale = tile_scale_from_amax(block_max(m, wred));
+  for (int row0 = 0; row0 < g.V; row0 += 64) {
+    uint4 v[ITER];
+#pragma unroll
+    for (int i = 0; i < ITER; ++i) v[i] = load(row0 + r0 + RSTEP * i);
+#pragma unroll
+    for (int i = 0; i < ITER; ++i) {
+      const size_t row = tile * g.V + row0 + r0 + RSTEP * i;
+      if (NAT && x_tiled) reinterpret_cast<uint4*>(x_tiled + row * D)[c] = v[i];
+      float f[8];
+      bf16x8_to_f32(v[i], f);
+      reinterpret_cast<uint2*>(codes + row * D)[c] = quant8(f, scale);
+    }
+  }
+  if (threadIdx.x == 0) scales[tile] = scale;
+}
+
 // Tile means of natural bf16 tokens. A token row holds all heads
 // (Hh*D*2 contiguous bytes); a CTA takes one tile of one batch and tensor and
 // a block of kPoolCols 16-byte column chunks of those rows, thread c owning
@@ -202,37 +262,42 @@ __global__ void __launch_bounds__(kPoolCols)
 pool_kernel(Geom g, const __nv_bfloat16* __restrict__ x0, const __nv_bfloat16* __restrict__ x1,
             float* __restrict__ p0, float* __restrict__ p1, int ncblk) {
   constexpr int CH = D / 8;   // 16-byte chunks per head row
-  __shared__ int rowoff[64];  // token offset of each in-tile row from the tile's first token, -1 if padded
+  __shared__ int rowoff[64];  // token offset of each row of a 64-row chunk from the tile's first token, -1 if padded
   const int tensor = blockIdx.z / ncblk, cblk = blockIdx.z % ncblk;
   const __nv_bfloat16* x = tensor ? x1 : x0;
   float* pooled = tensor ? p1 : p0;
   const int j = blockIdx.x, b = blockIdx.y;
   const TileCoord tc = tile_coord(g, j);
   const int n0 = (tc.t0 * g.H + tc.h0) * g.W + tc.w0;
-  if (threadIdx.x < 64) {
-    const int n = row_token(g, tc, threadIdx.x);
-    rowoff[threadIdx.x] = n >= 0 ? n - n0 : -1;
-  }
-  __syncthreads();
   const int cpt = g.Hh * CH;  // chunks per token (all heads)
   const int c = cblk * kPoolCols + threadIdx.x;
-  if (c >= cpt) return;
+  const bool active = c < cpt;
   const uint4* src = reinterpret_cast<const uint4*>(x + ((size_t)b * g.L + n0) * g.Hh * D) + c;
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  for (int row0 = 0; row0 < g.V; row0 += 64) {
+    if (row0 > 0) __syncthreads();  // every thread is done with the previous offsets
+    if (threadIdx.x < 64) {
+      const int n = row_token(g, tc, row0 + threadIdx.x);
+      rowoff[threadIdx.x] = n >= 0 ? n - n0 : -1;
+    }
+    __syncthreads();
+    if (!active) continue;
 #pragma unroll 1
-  for (int r0 = 0; r0 < 64; r0 += 16) {
-    uint4 v[16];
+    for (int r0 = 0; r0 < 64; r0 += 16) {
+      uint4 v[16];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = __ldg(src + (size_t)max(rowoff[r0 + i], 0) * cpt);
+      for (int i = 0; i < 16; ++i) v[i] = __ldg(src + (size_t)max(rowoff[r0 + i], 0) * cpt);
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      if (rowoff[r0 + i] < 0) continue;
-      float f[8];
-      bf16x8_to_f32(v[i], f);
+      for (int i = 0; i < 16; ++i) {
+        if (rowoff[r0 + i] < 0) continue;
+        float f[8];
+        bf16x8_to_f32(v[i], f);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) acc[e] += f[e];
+        for (int e = 0; e < 8; ++e) acc[e] += f[e];
+      }
     }
   }
+  if (!active) return;
   const float nvalid = (float)(tc.vt * tc.vh * tc.vw);
   const int head = c / CH, d0 = (c % CH) * 8;
   float4* out = reinterpret_cast<float4*>(pooled + (((size_t)b * g.Hh + head) * g.N + j) * D + d0);
@@ -257,7 +322,16 @@ bsattn_status launch_pool(const Geom& g, const __nv_bfloat16* x0, float* p0, con
 
 bsattn_status launch_reorder(const Geom& g, const __nv_bfloat16* x_nat, __nv_bfloat16* x_tiled,
                              uint8_t* codes, float* scales, int flags, cudaStream_t st) {
-  dim3 grid(g.N, g.Hh, g.B);
+  if ((flags & RO_QUANT) && g.nchunk > 1) {
+    __nv_bfloat16* xt = (flags & RO_WRITE_TILED) ? x_tiled : nullptr;
+    dim3 grid(g.N, g.Hh, g.B);
+    if (g.D == 128)
+      quant_multi_kernel<128, true><<<grid, kThreads, 0, st>>>(g, x_nat, xt, codes, scales);
+    else
+      quant_multi_kernel<64, true><<<grid, kThreads, 0, st>>>(g, x_nat, xt, codes, scales);
+    return cudaGetLastError() == cudaSuccess ? BSATTN_OK : BSATTN_ERR_CUDA;
+  }
+  dim3 grid(g.N * g.nchunk, g.Hh, g.B);
   if (g.D == 128)
     reorder_kernel<128><<<grid, kThreads, 0, st>>>(g, x_nat, x_tiled, codes, scales, flags);
   else
@@ -267,7 +341,7 @@ bsattn_status launch_reorder(const Geom& g, const __nv_bfloat16* x_nat, __nv_bfl
 
 bsattn_status launch_unreorder(const Geom& g, const __nv_bfloat16* x_tiled, __nv_bfloat16* x_nat,
                                const float* lse_tiled, float* lse_nat, cudaStream_t st) {
-  dim3 grid(g.N, g.Hh, g.B);
+  dim3 grid(g.N * g.nchunk, g.Hh, g.B);
   if (g.D == 128)
     unreorder_kernel<128><<<grid, kThreads, 0, st>>>(g, x_tiled, x_nat, lse_tiled, lse_nat);
   else
@@ -278,6 +352,13 @@ bsattn_status launch_unreorder(const Geom& g, const __nv_bfloat16* x_tiled, __nv
 bsattn_status launch_quant_tiled(const Geom& g, const __nv_bfloat16* x_tiled, uint8_t* codes,
                                  float* scales, cudaStream_t st) {
   dim3 grid(g.N, g.Hh, g.B);
+  if (g.nchunk > 1) {
+    if (g.D == 128)
+      quant_multi_kernel<128, false><<<grid, kThreads, 0, st>>>(g, x_tiled, nullptr, codes, scales);
+    else
+      quant_multi_kernel<64, false><<<grid, kThreads, 0, st>>>(g, x_tiled, nullptr, codes, scales);
+    return cudaGetLastError() == cudaSuccess ? BSATTN_OK : BSATTN_ERR_CUDA;
+  }
   if (g.D == 128)
     quant_tiled_kernel<128><<<grid, kThreads, 0, st>>>(g, x_tiled, codes, scales);
   else

@@ -67,6 +67,12 @@ WORKLOADS = {
                            win=(1, 1, 0), qk_fp8=True, seed=3),
     "topp": Workload("topp", 1, 40, 128, 21, 45, 80, "topp", k=16, p=0.9, seed=4,
                      temperature=(0.3, 3.0)),
+    # The hardware-friendly (6, 8, 8) tile of 384 tokens: the Wan-14B layer at
+    # the same 10% density (24 of 240 tiles), and the e4m3 tile window.
+    "wan14b_t688": Workload("wan14b_t688", 1, 40, 128, 21, 45, 80, "topk", k=24, seed=2,
+                            tile=(6, 8, 8)),
+    "window_fp8_t688": Workload("window_fp8_t688", 1, 12, 128, 21, 30, 52, "window",
+                                win=(1, 1, 0), qk_fp8=True, seed=3, tile=(6, 8, 8)),
 }
 
 

@@ -36,7 +36,7 @@
  *   - Block scores containing NaN give unspecified (but in-bounds) lists.
  *
  * Layouts (B batch, Hh heads, D head_dim, L = T*H*W, N = number of tiles,
- * V = tile volume = tile_t*tile_h*tile_w = 64):
+ * V = tile volume = tile_t*tile_h*tile_w, a multiple of 64):
  *   natural   [B, L, Hh, D] bf16, token n = (t*H + h)*W + w
  *   tiled     [B, Hh, N, V, D] (bf16, or u8 e4m3 codes), tile id
  *             j = ((t/tile_t)*nH + h/tile_h)*nW + w/tile_w, in-tile row
@@ -87,7 +87,7 @@ typedef struct {
 typedef struct {
   int B, heads, head_dim;       /* head_dim in {64, 128}                      */
   int T, H, W;                  /* latent grid, each >= 1                     */
-  int tile_t, tile_h, tile_w;   /* tile shape; volume must be 64              */
+  int tile_t, tile_h, tile_w;   /* tile shape; see attn_plan_create           */
   float softmax_scale;          /* <= 0 selects 1/sqrt(head_dim)              */
   int qk_fp8;                   /* 1: attn_forward takes per-tile e4m3 Q/K    */
 } bsattn_desc;
@@ -96,7 +96,7 @@ typedef struct {
   int Tp, Hp, Wp;               /* padded grid                                */
   int nT, nH, nW;               /* tiles per axis                             */
   int n_blocks;                 /* N = nT*nH*nW                               */
-  int tile_volume;              /* V = 64                                     */
+  int tile_volume;              /* V = tile_t * tile_h * tile_w               */
   int kmax;                     /* idx row capacity                           */
   float softmax_scale;          /* resolved scale                             */
   size_t select_workspace_bytes;  /* attn_select                              */
@@ -111,7 +111,20 @@ typedef struct bsattn_plan bsattn_plan;
  * a 4-byte device error word). The current CUDA device is bound to the plan.
  * Errors: INVALID_ARG (null, non-positive sizes, k outside its range,
  * p outside (0,1], negative half-widths), UNSUPPORTED (head_dim not 64/128,
- * tile volume != 64, N above 2048 for top-k/top-p), CUDA. */
+ * unsupported tile shape, N above 2048 for top-k/top-p, more than 2^31
+ * padded token rows over all batches and heads), CUDA.
+ *
+ * Tile shapes (the pages' "3D tile granularity"; FPSAttention's tile ablation
+ * compares (3,4,4) with the hardware-friendly (6,8,8)): the volume V must be
+ * 64 * c with 1 <= c <= 512, each side at most 1024, and each run of 64 in-tile rows [64i, 64i + 64)
+ * must be a box of the tile: 64 / (tile_h * tile_w) whole (h, w) frames when
+ * tile_h * tile_w divides 64, else 64 / tile_w whole w rows when tile_w
+ * divides 64 (and 64 / tile_w divides tile_h), else a 64-long run along w
+ * when 64 divides tile_w.
+ * (4,4,4), (2,4,8), (6,8,8), (4,8,8) and (8,8,8) qualify; (3,4,4) (V = 48)
+ * does not. The attention works on these 64-row chunks: with V = 64 two
+ * adjacent query tiles share a 128-row block, with V > 64 a block holds two
+ * chunks of one query tile, which keep the same key tiles. */
 bsattn_status attn_plan_create(const bsattn_desc* desc, const bsattn_rule* rule,
                                bsattn_plan** out);
 void attn_plan_destroy(bsattn_plan* plan);

@@ -21,6 +21,18 @@ SMALL = {
                                seed=14),
     "ragged_bf16_window": Workload("ragged_bf16_window", 1, 2, 128, 6, 6, 9, "window",
                                    win=(1, 0, 1), seed=15),
+    # Other tile shapes: a 64-token tile that is not a cube, and tiles of
+    # several 64-row chunks, some of them padding only at the grid's edge.
+    "tile248_window_fp8": Workload("tile248_window_fp8", 1, 2, 128, 5, 9, 13, "window",
+                                   win=(1, 1, 0), qk_fp8=True, seed=16, tile=(2, 4, 8)),
+    "tile688_topk": Workload("tile688_topk", 2, 2, 128, 9, 12, 13, "topk", k=3, seed=17,
+                             tile=(6, 8, 8)),
+    "tile488_topp": Workload("tile488_topp", 1, 3, 128, 6, 11, 17, "topp", k=2, p=0.9, seed=18,
+                             temperature=(0.3, 3.0), tile=(4, 8, 8)),
+    "tile688_window_fp8": Workload("tile688_window_fp8", 1, 2, 128, 9, 12, 13, "window",
+                                   win=(1, 1, 1), qk_fp8=True, seed=19, tile=(6, 8, 8)),
+    "tile11x128_d64": Workload("tile11x128_d64", 1, 2, 64, 3, 5, 70, "topk", k=2, seed=20,
+                               tile=(1, 1, 128)),
 }
 
 

@@ -150,7 +150,8 @@ def test_select_degenerate_rows(bs, N, rule):
             assert_topp_equal(got[r], pad[r], 0.9, k)
 
 
-@pytest.mark.parametrize("name", ["ragged_window_fp8", "ragged_bf16_window"])
+@pytest.mark.parametrize("name", ["ragged_window_fp8", "ragged_bf16_window", "tile248_window_fp8",
+                                  "tile688_window_fp8"])
 def test_window_lists(bs, name):
     wl = SMALL[name]
     plan = _plan(bs, wl)
@@ -159,12 +160,13 @@ def test_window_lists(bs, name):
     cnt = torch.empty(sc, dtype=torch.int32, device="cuda")
     bs.attn_select_from_scores(plan, None, idx, cnt)
     got = lists_from_device(idx, cnt)
-    grid = tiling.tile_grid(wl.T, wl.H, wl.W)
+    grid = tiling.tile_grid(wl.T, wl.H, wl.W, wl.tile)
     for r, l in enumerate(got):
         np.testing.assert_array_equal(l, select.window_row(r % plan.N, grid, wl.win))
 
 
-@pytest.mark.parametrize("name", ["ragged_window_fp8", "ragged_d64_fp8", "tiny_d64"])
+@pytest.mark.parametrize("name", ["ragged_window_fp8", "ragged_d64_fp8", "tiny_d64", "tile688_window_fp8",
+                                  "tile11x128_d64"])
 def test_quantize_e4m3_bytes(bs, name):
     wl = SMALL[name]
     plan = _plan(bs, wl)
@@ -176,7 +178,7 @@ def test_quantize_e4m3_bytes(bs, name):
     codes = torch.empty(plan.tiled_shape(), dtype=torch.uint8, device="cuda")
     scales = torch.empty((wl.B, wl.heads, plan.N), dtype=torch.float32, device="cuda")
     bs.attn_quantize_e4m3(plan, xt, codes, scales)
-    rc, rs = e4m3.quantize_tiled(tiling.reorder(to64(q).astype(np.float32), wl.T, wl.H, wl.W))
+    rc, rs = e4m3.quantize_tiled(tiling.reorder(to64(q).astype(np.float32), wl.T, wl.H, wl.W, wl.tile))
     np.testing.assert_array_equal(scales.cpu().numpy(), rs)
     np.testing.assert_array_equal(codes.cpu().numpy(), rc)
 
@@ -186,12 +188,13 @@ def _oracle_inputs(wl):
     return q, k, v, to64(q), to64(k), to64(v)
 
 
-@pytest.mark.parametrize("name", ["tiny_d64", "ragged_topk", "ragged_topp", "ragged_bf16_window"])
+@pytest.mark.parametrize("name", ["tiny_d64", "ragged_topk", "ragged_topp", "ragged_bf16_window",
+                                  "tile688_topk", "tile488_topp", "tile11x128_d64"])
 def test_forward_bf16_against_oracle(bs, name):
     wl = SMALL[name]
     plan = _plan(bs, wl, qk_fp8=False)
     q, k, v, qn, kn, vn = _oracle_inputs(wl)
-    _, _, _, lists = attention.route(qn, kn, wl.T, wl.H, wl.W, wl.rule, k=wl.k, p=wl.p,
+    _, _, _, lists = attention.route(qn, kn, wl.T, wl.H, wl.W, wl.rule, tile=wl.tile, k=wl.k, p=wl.p,
                                      half=wl.win, score_dtype=np.float32)
     idx, cnt = lists_to_device(lists, plan.kmax)
     tiled = []
@@ -200,26 +203,27 @@ def test_forward_bf16_against_oracle(bs, name):
         bs.attn_reorder(plan, x.cuda(), t)
         tiled.append(t)
     o = torch.empty(plan.tiled_shape(), dtype=torch.bfloat16, device="cuda")
-    lse = torch.empty((wl.B, wl.heads, plan.N, 64), dtype=torch.float32, device="cuda")
+    lse = torch.empty((wl.B, wl.heads, plan.N, plan.V), dtype=torch.float32, device="cuda")
     si, sc = plan.list_shapes()
     bs.attn_forward(plan, tiled[0], tiled[1], tiled[2], idx.view(si), cnt.view(sc), o, lse)
     assert bs.attn_check_device_status(plan) == 0
-    o_ref, lse_ref = attention.attention_full(qn, kn, vn, lists, wl.T, wl.H, wl.W)
-    o_nat = tiling.unreorder(to64(o), wl.T, wl.H, wl.W)
+    o_ref, lse_ref = attention.attention_full(qn, kn, vn, lists, wl.T, wl.H, wl.W, wl.tile)
+    o_nat = tiling.unreorder(to64(o), wl.T, wl.H, wl.W, wl.tile)
     err = np.abs(o_nat - o_ref)
     assert err.max() <= 2e-2 and err.mean() <= 2e-3, (err.max(), err.mean())
-    lse_nat = np.stack([tiling.unreorder(to64(lse)[:, h:h + 1, :, :, None], wl.T, wl.H, wl.W)[..., 0, 0]
+    lse_nat = np.stack([tiling.unreorder(to64(lse)[:, h:h + 1, :, :, None], wl.T, wl.H, wl.W, wl.tile)[..., 0, 0]
                         for h in range(wl.heads)], axis=1)
     np.testing.assert_allclose(lse_nat, lse_ref, rtol=0, atol=2e-2)
 
 
-@pytest.mark.parametrize("name", ["ragged_window_fp8", "ragged_d64_fp8"])
+@pytest.mark.parametrize("name", ["ragged_window_fp8", "ragged_d64_fp8", "tile248_window_fp8",
+                                  "tile688_window_fp8"])
 def test_forward_fp8_against_oracle(bs, name):
     wl = SMALL[name]
     plan = _plan(bs, wl)
     q, k, v, qn, kn, vn = _oracle_inputs(wl)
-    qd, kd, (qc, qs), (kc, ks) = attention.fp8_qk(qn, kn, wl.T, wl.H, wl.W)
-    _, _, _, lists = attention.route(qn, kn, wl.T, wl.H, wl.W, wl.rule, k=wl.k, p=wl.p,
+    qd, kd, (qc, qs), (kc, ks) = attention.fp8_qk(qn, kn, wl.T, wl.H, wl.W, wl.tile)
+    _, _, _, lists = attention.route(qn, kn, wl.T, wl.H, wl.W, wl.rule, tile=wl.tile, k=wl.k, p=wl.p,
                                      half=wl.win, score_dtype=np.float32)
     idx, cnt = lists_to_device(lists, plan.kmax)
     vt = torch.empty(plan.tiled_shape(), dtype=torch.bfloat16, device="cuda")
@@ -230,8 +234,8 @@ def test_forward_fp8_against_oracle(bs, name):
                     idx.view(si), cnt.view(sc), o, q_scale=torch.from_numpy(qs).cuda(),
                     k_scale=torch.from_numpy(ks).cuda())
     assert bs.attn_check_device_status(plan) == 0
-    o_ref, _ = attention.attention_full(qd, kd, vn, lists, wl.T, wl.H, wl.W)
-    o_nat = tiling.unreorder(to64(o), wl.T, wl.H, wl.W)
+    o_ref, _ = attention.attention_full(qd, kd, vn, lists, wl.T, wl.H, wl.W, wl.tile)
+    o_nat = tiling.unreorder(to64(o), wl.T, wl.H, wl.W, wl.tile)
     rel = np.linalg.norm(o_nat - o_ref) / np.linalg.norm(o_ref)
     assert rel <= 1e-2, rel
 
@@ -267,7 +271,9 @@ def test_bad_list_entry_sets_error_word_and_is_skipped(bs):
 
 
 @pytest.mark.parametrize("name", ["tiny_d64", "ragged_topk", "ragged_topp", "ragged_bf16_window",
-                                  "ragged_window_fp8", "ragged_d64_fp8"])
+                                  "ragged_window_fp8", "ragged_d64_fp8", "tile248_window_fp8",
+                                  "tile688_topk", "tile488_topp", "tile688_window_fp8",
+                                  "tile11x128_d64"])
 def test_forward_natural_equals_tiled_path(bs, name):
     """Natural-layout attention (tile reorder folded into its loads) gives
     bit-identical O and lse to reorder -> attn_forward -> unreorder."""
@@ -297,7 +303,7 @@ def test_forward_natural_equals_tiled_path(bs, name):
         bs.attn_reorder(plan, k, ka)
         qn, kn = q, k
     ot = torch.empty(ts, dtype=torch.bfloat16, device="cuda")
-    lse_t = torch.empty((wl.B, wl.heads, plan.N, 64), dtype=torch.float32, device="cuda")
+    lse_t = torch.empty((wl.B, wl.heads, plan.N, plan.V), dtype=torch.float32, device="cuda")
     bs.attn_forward(plan, qa, ka, vt, idx, cnt, ot, lse_t, q_scale=qs, k_scale=ks)
     o_ref = torch.empty_like(q)
     bs.attn_unreorder(plan, ot, o_ref)
@@ -311,8 +317,8 @@ def test_forward_natural_equals_tiled_path(bs, name):
 
 
 def tiling_lse_natural(lse_t, wl, plan):
-    """Tiled lse [B, Hh, N, 64] -> natural [B, Hh, L] (oracle's tile order)."""
+    """Tiled lse [B, Hh, N, V] -> natural [B, Hh, L] (oracle's tile order)."""
     x = to64(lse_t)
-    out = np.stack([tiling.unreorder(x[:, h:h + 1, :, :, None], wl.T, wl.H, wl.W)[..., 0, 0]
+    out = np.stack([tiling.unreorder(x[:, h:h + 1, :, :, None], wl.T, wl.H, wl.W, wl.tile)[..., 0, 0]
                     for h in range(wl.heads)], axis=1)
     return torch.from_numpy(out.astype(np.float32))

@@ -40,7 +40,7 @@ def run_layer(bs, wl, q, k, v, want_lse=True):
 def _reference_inputs(wl, q, k, v):
     qn, kn, vn = to64(q), to64(k), to64(v)
     if wl.qk_fp8:
-        qd, kd, _, _ = attention.fp8_qk(qn, kn, wl.T, wl.H, wl.W)
+        qd, kd, _, _ = attention.fp8_qk(qn, kn, wl.T, wl.H, wl.W, wl.tile)
         return qn, kn, qd, kd, vn
     return qn, kn, qn, kn, vn
 
@@ -62,7 +62,7 @@ def test_layer_small(bs, name):
     q, k, v = make_qkv(wl, "cuda")
     plan, o, lse, idx, cnt = run_layer(bs, wl, q, k, v)
     qn, kn, qa, ka, vn = _reference_inputs(wl, q, k, v)
-    _, _, S, lists = attention.route(qn, kn, wl.T, wl.H, wl.W, wl.rule, k=wl.k, p=wl.p,
+    _, _, S, lists = attention.route(qn, kn, wl.T, wl.H, wl.W, wl.rule, tile=wl.tile, k=wl.k, p=wl.p,
                                      half=wl.win)
     got = lists_from_device(idx, cnt)
     same = [np.array_equal(a, b) for a, b in zip(got, lists)]
@@ -73,11 +73,11 @@ def test_layer_small(bs, name):
             assert_valid_selection(g, Sf[r], wl.rule, k=wl.k, p=wl.p)
     assert np.mean(same) >= 0.9
     o_ref, lse_ref = attention.attention_full(qa, ka, vn, lists,
-                                              wl.T, wl.H, wl.W)
+                                              wl.T, wl.H, wl.W, wl.tile)
     if all(same):
         _check_outputs(wl, to64(o), o_ref, to64(lse), lse_ref)
     else:  # compare only query tiles whose lists agree
-        tid, _ = tiling.token_tile_and_row(wl.T, wl.H, wl.W)
+        tid, _ = tiling.token_tile_and_row(wl.T, wl.H, wl.W, wl.tile)
         for r, ok in enumerate(same):
             if ok:
                 b, h, i = r // (wl.heads * plan.N), (r // plan.N) % wl.heads, r % plan.N
@@ -126,7 +126,7 @@ def test_layer_full_size_sampled(bs, name):
     sub_wl = wl.__class__(**{**wl.__dict__, "heads": len(heads)})
     qn_, kn_, qa, ka, vn = _reference_inputs(sub_wl, torch.from_numpy(qn), torch.from_numpy(kn),
                                              torch.from_numpy(vn))
-    _, _, S, lists = attention.route(qn, kn, wl.T, wl.H, wl.W, wl.rule, k=wl.k, p=wl.p,
+    _, _, S, lists = attention.route(qn, kn, wl.T, wl.H, wl.W, wl.rule, tile=wl.tile, k=wl.k, p=wl.p,
                                      half=wl.win)
     got_all = lists_from_device(idx[:, heads], cnt[:, heads])
     # every list of the sampled heads: valid under fp64 scores; counts as the rule says
@@ -142,7 +142,7 @@ def test_layer_full_size_sampled(bs, name):
     rows = [(0, hi, i) for hi in range(len(heads)) for i in tiles
             if np.array_equal(got_all[hi * N + i], lists[hi * N + i])]
     assert rows
-    ref = attention.attention_rows(qa, ka, vn, lists, wl.T, wl.H, wl.W, rows=rows)
+    ref = attention.attention_rows(qa, ka, vn, lists, wl.T, wl.H, wl.W, wl.tile, rows=rows)
     o_sub = to64(o[:, :, heads, :])
     lse_sub = to64(lse[:, heads, :])
     for (b, hi, i), (tok, o_ref, lse_ref) in ref.items():

@@ -112,3 +112,23 @@ def test_fp8_qk_uses_tile_scales():
     np.testing.assert_array_equal(qc, kc)  # scaling by 3 scales amax and scale alike
     assert qs.shape == (1, 1, 2)
     np.testing.assert_allclose(qd, q, rtol=2 ** -4, atol=float(qs.max()) * 2 ** -9)
+
+
+@pytest.mark.parametrize("tile", [(2, 4, 8), (6, 8, 8)])
+def test_self_tile_lists_match_coordinate_blocks(tile):
+    """Each query tile keeping only itself is attention within the coordinate
+    block (t // tile_t, h // tile_h, w // tile_w), written out per token."""
+    T, H, W = 7, 10, 9
+    tt, th, tw = tile
+    rng = np.random.default_rng(8)
+    q, k, v = (rng.standard_normal((1, T * H * W, 1, 4)) for _ in range(3))
+    nb = tiling.n_blocks(T, H, W, tile)
+    o, _ = attention.attention_full(q, k, v, [np.array([j]) for j in range(nb)], T, H, W, tile)
+    t, h, w = np.meshgrid(np.arange(T), np.arange(H), np.arange(W), indexing="ij")
+    blk = np.stack([t.ravel() // tt, h.ravel() // th, w.ravel() // tw], axis=1)
+    for n in range(0, T * H * W, 7):
+        keys = np.nonzero((blk == blk[n]).all(axis=1))[0]
+        s = np.array([q[0, n, 0] @ k[0, m, 0] for m in keys]) / 2.0
+        p = np.exp(s - s.max())
+        ref = (p[:, None] * v[0, keys, 0]).sum(axis=0) / p.sum()
+        np.testing.assert_allclose(o[0, n, 0], ref, rtol=1e-12, atol=1e-13)

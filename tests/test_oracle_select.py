@@ -97,8 +97,9 @@ def test_topp_special_cases():
         np.testing.assert_array_equal(select.topp_row(uni, p, 1), np.arange(cnt))
 
 
-def test_window_closed_form(golden_dir):
-    g = json.load(open(os.path.join(golden_dir, "workload_counts.json")))["window_fp8"]
+@pytest.mark.parametrize("name", ["window_fp8", "window_fp8_t688"])
+def test_window_closed_form(golden_dir, name):
+    g = json.load(open(os.path.join(golden_dir, "workload_counts.json")))[name]
     nT, nH, nW = g["tiles"]
     total = sum(select.window_row(i, (nT, nH, nW), (1, 1, 0)).size for i in range(nT * nH * nW))
     assert total == g["kept_pairs_per_head"] == (3 * nT - 2) * (3 * nH - 2) * nW
