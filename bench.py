@@ -47,6 +47,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--heads", type=int, default=0,
+                    help="run a copy of the workload with this many heads (small profiling cases)")
     return ap.parse_args()
 
 
@@ -76,6 +78,14 @@ def measured_traffic(workload: str):
         return rec["per_launch_dram_bytes"].get(workload)
     except Exception:
         return None
+
+
+def workload_of(args):
+    """The named workload, with its head count replaced when --heads is given."""
+    import dataclasses
+
+    wl = WORKLOADS[args.workload]
+    return dataclasses.replace(wl, heads=args.heads) if args.heads > 0 else wl
 
 
 def kept_pairs_from_counts(cnt: torch.Tensor) -> int:
@@ -280,7 +290,7 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    wl = WORKLOADS[args.workload]
+    wl = workload_of(args)
     total_flops, total_s, text = 0.0, 0.0, ""
     per_step_target = max(0.05, 90.0 / max(1, args.steps + args.warmup))
     for s in range(args.warmup + args.steps):
@@ -342,7 +352,7 @@ def main():
 
     from block_sparse_attention_reorder_b200 import bsattn
 
-    wl = WORKLOADS[args.workload]
+    wl = workload_of(args)
     plan = bsattn.Plan.for_workload(wl)
     q, k, v = make_qkv(wl, "cuda", batch_offset=rank)
     o = torch.empty_like(q)
@@ -427,7 +437,6 @@ def main():
         "dtype": "bf16+e4m3" if wl.qk_fp8 else "bf16",
         "data": "synthetic",
         "config": workload_config(wl, {"kept_pairs": kept, "kept_tflop": flops / 1e12,
-                                        "tile": list(wl.tile),
                                         "mma_chunk_pairs": issued,
                                         "pair_efficiency": kept * nch2 / issued if issued else None,
                                         "kv_chunk_loads": loads,
@@ -440,7 +449,7 @@ def main():
                      "frac": achieved / pk["bf16_tflops"],
                      "achieved_mma": achieved_mma,
                      "peak_note": f"{pk['source']} bf16 burst (kernel timed alone)",
-                     "traffic": measured_traffic(wl.name)},
+                     "traffic": measured_traffic(wl.name) if args.heads == 0 else None},
         "memory_kernels": memory_kernel_rates(wl, plan, comp, pk),
         "e2e": e2e,
         "gpu_launches": launches_per_step(wl, plan) * args.steps,

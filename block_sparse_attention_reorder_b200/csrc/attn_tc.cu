@@ -134,7 +134,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   uint32_t* bmA = reinterpret_cast<uint32_t*>(smem + C::OFF_DYN);
   uint32_t* bmB = bmA + P.bm_words;
   uint32_t* ulist = bmB + P.bm_words;
-  uint32_t* uorg = ulist + P.umax;  // packed first-token offsets of the steps' key chunks
+  uint32_t* uext = ulist + P.umax;  // real extent of each step's key chunk (see below)
+  uint32_t* uorg = uext + P.umax;   // packed in-tile offsets of the steps' key chunks (several-chunk tiles)
 
   const Geom& g = P.g;
   const int nchunk = g.nchunk;
@@ -306,10 +307,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           if (nchunk > 1 && !chunk_real(j, c)) continue;
           if (pos < P.umax) {
             ulist[pos] = e | ((uint32_t)c << 21);
-            if (nchunk > 1) {
-              const ChunkOrigin o = chunk_origin(g, c);
-              uorg[pos] = (uint32_t)o.dt | ((uint32_t)o.dh << 10) | ((uint32_t)o.dw << 20);
-            }
+            const ChunkOrigin o = nchunk > 1 ? chunk_origin(g, c) : ChunkOrigin{0, 0, 0};
+            if (nchunk > 1) uorg[pos] = (uint32_t)o.dt | ((uint32_t)o.dh << 10) | ((uint32_t)o.dw << 20);
+            // Real extent of the key chunk from its first token along t, h, w
+            // (capped at 255), bit 31 set when it is smaller than the chunk
+            // box along some axis (padded keys to mask).
+            const int bt = j / (g.nH * g.nW), bhh = (j / g.nW) % g.nH, bw = j % g.nW;
+            const int vt = min(g.T - bt * g.tt - o.dt, 255), vh = min(g.H - bhh * g.th - o.dh, 255),
+                      vw = min(g.W - bw * g.tw - o.dw, 255);
+            const bool edge = vt < g.ct || vh < g.ch || vw < g.cw;
+            uext[pos] = (uint32_t)vt | ((uint32_t)vh << 8) | ((uint32_t)vw << 16) | (edge ? 1u << 31 : 0u);
           }
           ++pos;
         }
@@ -479,12 +486,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         uint32_t sr[64];
         tc::tmem_ld64_wait(sbuf, sr);
         const float c = P.scale_log2 * (FP8 ? qsc * __ldg(P.ks + bh * g.N + j) : 1.f);
-        const int bt = j / (g.nH * g.nW), bhh = (j / g.nW) % g.nH, bw = j % g.nW;
-        const ChunkOrigin ko = step_origin(n);
-        // Real extent of the key chunk along each axis, from its first token.
-        const int vt = g.T - bt * g.tt - ko.dt, vh = g.H - bhh * g.th - ko.dh, vw = g.W - bw * g.tw - ko.dw;
-        const bool edge = vt < g.ct || vh < g.ch || vw < g.cw;
+        const uint32_t ext = uext[n];
+        const bool edge = (ext >> 31) != 0;
         if (edge) {  // padded keys of an edge chunk
+          const int vt = (int)(ext & 0xffu), vh = (int)((ext >> 8) & 0xffu), vw = (int)((ext >> 16) & 0xffu);
 #pragma unroll
           for (int q = 0; q < 64; ++q) {
             const uint32_t cc = colc[q];
@@ -698,7 +703,8 @@ bsattn_status run(const bsattn_plan* p, const void* q, const void* k, const __nv
   if (NKV ? !make_map_nat(&mv, v, p)
           : !make_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, rows, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B))
     return BSATTN_ERR_CUDA;
-  size_t smem = 1024 + C::OFF_DYN + (size_t)prm.bm_words * 8 + (size_t)prm.umax * (p->nchunk > 1 ? 8 : 4);
+  // Step list, extents and (tiles of several chunks) chunk offsets.
+  size_t smem = 1024 + C::OFF_DYN + (size_t)prm.bm_words * 8 + (size_t)prm.umax * (p->nchunk > 1 ? 12 : 8);
   if (smem < 80 * 1024) smem = 80 * 1024;  // at most two CTAs (2 x 256 TMEM columns) per SM
   if (smem > 227 * 1024) return BSATTN_ERR_UNSUPPORTED;
   auto kern = attn_tc_kernel<D, FP8, NQO, NKV>;
