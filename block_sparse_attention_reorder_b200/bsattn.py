@@ -44,6 +44,10 @@ class Rule(ctypes.Structure):
                 ("win_t", ctypes.c_int), ("win_h", ctypes.c_int), ("win_w", ctypes.c_int)]
 
 
+class ScheduleEntry(ctypes.Structure):
+    _fields_ = [("first_step", ctypes.c_int), ("desc", Desc), ("rule", Rule)]
+
+
 class Info(ctypes.Structure):
     _fields_ = [("Tp", ctypes.c_int), ("Hp", ctypes.c_int), ("Wp", ctypes.c_int),
                 ("nT", ctypes.c_int), ("nH", ctypes.c_int), ("nW", ctypes.c_int),
@@ -77,12 +81,17 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "attn_forward_natural": [P, P, P, P, P, P, P, P, P, P, P, Z, P],
         "attn_layer": [P, P, P, P, P, P, P, P, P, Z, P],
         "attn_check_device_status": [P, P],
+        "attn_schedule_create": [ctypes.POINTER(ScheduleEntry), I, ctypes.POINTER(P)],
+        "attn_schedule_destroy": [P],
+        "attn_schedule_plan": [P, I, ctypes.POINTER(P)],
+        "attn_schedule_workspace_bytes": [P, ctypes.POINTER(Z)],
+        "attn_schedule_layer": [P, I, P, P, P, P, P, P, P, P, Z, P],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
         fn.argtypes = args
         fn.restype = ctypes.c_char_p if name == "attn_status_string" else (
-            None if name == "attn_plan_destroy" else ctypes.c_int)
+            None if name in ("attn_plan_destroy", "attn_schedule_destroy") else ctypes.c_int)
     return lib
 
 
@@ -91,7 +100,8 @@ EXPORTED = ("attn_plan_create", "attn_plan_destroy", "attn_plan_info", "attn_sta
             "attn_reorder", "attn_pool", "attn_unreorder", "attn_block_scores",
             "attn_select_from_scores", "attn_select", "attn_select_static", "attn_quantize_e4m3",
             "attn_forward", "attn_forward_natural",
-            "attn_layer", "attn_check_device_status")
+            "attn_layer", "attn_check_device_status", "attn_schedule_create", "attn_schedule_destroy",
+            "attn_schedule_plan", "attn_schedule_workspace_bytes", "attn_schedule_layer")
 
 
 def _check(code: int, where: str):
@@ -126,14 +136,18 @@ class Plan:
     """An immutable problem + rule description (attn_plan_create)."""
 
     def __init__(self, B, heads, head_dim, T, H, W, rule="topk", k=0, p=0.0, win=(0, 0, 0),
-                 tile=(4, 4, 4), softmax_scale=0.0, qk_fp8=False):
+                 tile=(4, 4, 4), softmax_scale=0.0, qk_fp8=False, _handle=None):
         self.desc = Desc(B, heads, head_dim, T, H, W, tile[0], tile[1], tile[2],
                          float(softmax_scale), int(bool(qk_fp8)))
         self.rule = Rule(_RULES[rule] if isinstance(rule, str) else int(rule), int(k), float(p),
                          int(win[0]), int(win[1]), int(win[2]))
-        h = ctypes.c_void_p()
-        _check(_lib.attn_plan_create(ctypes.byref(self.desc), ctypes.byref(self.rule),
-                                     ctypes.byref(h)), "attn_plan_create")
+        self._owned = _handle is None
+        if _handle is None:
+            h = ctypes.c_void_p()
+            _check(_lib.attn_plan_create(ctypes.byref(self.desc), ctypes.byref(self.rule),
+                                         ctypes.byref(h)), "attn_plan_create")
+        else:
+            h = _handle  # a plan owned by a Schedule
         self.handle = h
         info = Info()
         _check(_lib.attn_plan_info(h, ctypes.byref(info)), "attn_plan_info")
@@ -153,9 +167,9 @@ class Plan:
                    win=wl.win, tile=wl.tile, qk_fp8=wl.qk_fp8)
 
     def close(self):
-        if getattr(self, "handle", None):
+        if getattr(self, "handle", None) and getattr(self, "_owned", True):
             _lib.attn_plan_destroy(self.handle)
-            self.handle = None
+        self.handle = None
 
     def __del__(self):
         try:
@@ -178,6 +192,80 @@ class Plan:
                   "forward": self.info.forward_workspace_bytes,
                   "layer": self.info.layer_workspace_bytes}[which]
         return torch.empty(max(int(nbytes), 16), dtype=torch.uint8, device=device)
+
+
+class Schedule:
+    """Denoising-step-aware list of plans over the same tensors
+    (attn_schedule_create). `entries`: (first_step, dict of Plan keyword
+    arguments: rule, k, p, win, tile, qk_fp8, softmax_scale)."""
+
+    def __init__(self, B, heads, head_dim, T, H, W, entries):
+        arr = (ScheduleEntry * len(entries))()
+        for i, (first, kw) in enumerate(entries):
+            tile = kw.get("tile", (4, 4, 4))
+            rule = kw.get("rule", "topk")
+            win = kw.get("win", (0, 0, 0))
+            arr[i].first_step = int(first)
+            arr[i].desc = Desc(B, heads, head_dim, T, H, W, tile[0], tile[1], tile[2],
+                               float(kw.get("softmax_scale", 0.0)), int(bool(kw.get("qk_fp8", False))))
+            arr[i].rule = Rule(_RULES[rule] if isinstance(rule, str) else int(rule), int(kw.get("k", 0)),
+                               float(kw.get("p", 0.0)), int(win[0]), int(win[1]), int(win[2]))
+        h = ctypes.c_void_p()
+        _check(_lib.attn_schedule_create(arr, len(entries), ctypes.byref(h)), "attn_schedule_create")
+        self.handle = h
+        self.first_steps = [int(f) for f, _ in entries]
+        self.plans = []
+        for i, (first, kw) in enumerate(entries):
+            ph = ctypes.c_void_p()
+            _check(_lib.attn_schedule_plan(h, int(first), ctypes.byref(ph)), "attn_schedule_plan")
+            args = {k: v for k, v in kw.items() if k in ("rule", "k", "p", "win", "tile", "qk_fp8",
+                                                         "softmax_scale")}
+            self.plans.append(Plan(B, heads, head_dim, T, H, W, _handle=ph, **args))
+        nbytes = ctypes.c_size_t()
+        _check(_lib.attn_schedule_workspace_bytes(h, ctypes.byref(nbytes)), "attn_schedule_workspace_bytes")
+        self.workspace_bytes = int(nbytes.value)
+
+    def plan_for(self, step: int) -> Plan:
+        """The plan serving `step` (the same one the library picks)."""
+        ph = ctypes.c_void_p()
+        _check(_lib.attn_schedule_plan(self.handle, int(step), ctypes.byref(ph)), "attn_schedule_plan")
+        for p in self.plans:
+            if p.handle.value == ph.value:
+                return p
+        raise RuntimeError("schedule returned an unknown plan")
+
+    def workspace(self, device="cuda"):
+        return torch.empty(max(self.workspace_bytes, 16), dtype=torch.uint8, device=device)
+
+    def close(self):
+        if getattr(self, "handle", None):
+            for p in self.plans:
+                p.handle = None
+            _lib.attn_schedule_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def attn_schedule_layer(schedule: Schedule, step: int, q_nat, k_nat, v_nat, o_nat, ws, lse_nat=None,
+                        idx=None, cnt=None, stream=None):
+    plan = schedule.plan_for(step)
+    for name, t in (("q_nat", q_nat), ("k_nat", k_nat), ("v_nat", v_nat), ("o_nat", o_nat)):
+        _want(t, torch.bfloat16, plan.natural_shape(), name)
+    if lse_nat is not None:
+        _want(lse_nat, torch.float32, (plan.B, plan.heads, plan.L), "lse_nat")
+    if idx is not None:
+        si, sc = plan.list_shapes()
+        _want(idx, torch.int32, si, "idx")
+        _want(cnt, torch.int32, sc, "cnt")
+    _check(_lib.attn_schedule_layer(schedule.handle, int(step), _ptr(q_nat), _ptr(k_nat), _ptr(v_nat),
+                                    _ptr(o_nat), _ptr(lse_nat), _ptr(idx), _ptr(cnt), _ptr(ws),
+                                    ws.numel() * ws.element_size(), _stream(stream)),
+           "attn_schedule_layer")
 
 
 def attn_reorder(plan: Plan, x_nat, x_tiled, pooled=None, stream=None):

@@ -238,6 +238,42 @@ bsattn_status attn_layer(const bsattn_plan* plan, const void* q_nat, const void*
  * Returns OK, TIMEOUT or INTERNAL (bad list entry), or CUDA. */
 bsattn_status attn_check_device_status(const bsattn_plan* plan, void* stream);
 
+/* Denoising-step-aware schedule (FPSAttention page, Approach: the tile size,
+ * the sparsity window and FP8 change between early, middle and late
+ * denoising steps). Entry i is used for steps [first_step_i, first_step_{i+1})
+ * and the last entry for every later step. Entries are ordered by strictly
+ * increasing first_step starting at 0 and describe the same tensors (B,
+ * heads, head_dim, T, H, W equal); tile shape, rule and qk_fp8 may differ.
+ * At most BSATTN_MAX_SCHEDULE entries. */
+#define BSATTN_MAX_SCHEDULE 64
+typedef struct {
+  int first_step;    /* first denoising step served by this entry          */
+  bsattn_desc desc;
+  bsattn_rule rule;
+} bsattn_schedule_entry;
+typedef struct bsattn_schedule bsattn_schedule;
+
+/* Validate the entries (INVALID_ARG before any device call: null, n outside
+ * [1, BSATTN_MAX_SCHEDULE], first_step not 0 then strictly increasing,
+ * differing tensor shapes) and create one plan per entry (errors as
+ * attn_plan_create; nothing is left allocated on failure). The schedule owns
+ * its plans. */
+bsattn_status attn_schedule_create(const bsattn_schedule_entry* entries, int n,
+                                   bsattn_schedule** out);
+void attn_schedule_destroy(bsattn_schedule* schedule);
+/* The plan serving denoising step `step` (>= 0); owned by the schedule. */
+bsattn_status attn_schedule_plan(const bsattn_schedule* schedule, int step,
+                                 const bsattn_plan** plan);
+/* Workspace for attn_schedule_layer at any step: the largest
+ * info.layer_workspace_bytes of the schedule's plans. */
+bsattn_status attn_schedule_workspace_bytes(const bsattn_schedule* schedule, size_t* bytes);
+/* attn_layer with the plan serving `step`. idx_out/cnt_out (if non-NULL) are
+ * sized for that plan ([B, Hh, N, kmax] and [B, Hh, N] of its tiles). */
+bsattn_status attn_schedule_layer(const bsattn_schedule* schedule, int step, const void* q_nat,
+                                  const void* k_nat, const void* v_nat, void* o_nat,
+                                  float* lse_nat, int32_t* idx_out, int32_t* cnt_out, void* ws,
+                                  size_t ws_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -73,3 +73,43 @@ def test_null_plan_and_null_pointers_are_invalid():
     assert lib.attn_check_device_status(None, None) == 1
     assert lib.attn_plan_info(None, None) == 1
     lib.attn_plan_destroy(None)  # no-op
+
+
+_GRID = dict(B=1, heads=2, head_dim=64, T=8, H=16, W=16)
+
+
+@pytest.mark.parametrize("entries", [
+    [],                                                              # no entry
+    [(1, dict(rule="topk", k=8))],                                   # does not start at step 0
+    [(0, dict(rule="topk", k=8)), (0, dict(rule="topk", k=4))],      # first steps not increasing
+    [(0, dict(rule="topk", k=8)), (5, dict(rule="topk", k=4)), (3, dict(rule="topk", k=2))],
+    [(0, dict(rule="topk", k=8))] + [(i, dict(rule="topk", k=8)) for i in range(1, 65)],  # > 64
+])
+def test_schedule_rejects_bad_entries_before_any_device_call(entries):
+    from block_sparse_attention_reorder_b200 import bsattn
+    with pytest.raises(bsattn.BsattnError) as e:
+        bsattn.Schedule(**_GRID, entries=entries)
+    assert e.value.code == 1
+
+
+def test_schedule_rejects_entries_over_different_tensors():
+    from block_sparse_attention_reorder_b200 import bsattn
+    arr = (bsattn.ScheduleEntry * 2)()
+    for i, T in enumerate((8, 12)):  # a different grid in the second entry
+        arr[i].first_step = 10 * i
+        arr[i].desc = bsattn.Desc(1, 2, 64, T, 16, 16, 4, 4, 4, 0.0, 0)
+        arr[i].rule = bsattn.Rule(0, 8, 0.0, 0, 0, 0)
+    h = ctypes.c_void_p()
+    assert bsattn._lib.attn_schedule_create(arr, 2, ctypes.byref(h)) == 1
+    assert not h.value
+
+
+def test_null_schedule_calls_are_invalid():
+    from block_sparse_attention_reorder_b200 import bsattn
+    lib = bsattn._lib
+    assert lib.attn_schedule_create(None, 1, None) == 1
+    assert lib.attn_schedule_plan(None, 0, None) == 1
+    assert lib.attn_schedule_workspace_bytes(None, None) == 1
+    assert lib.attn_schedule_layer(None, 0, None, None, None, None, None, None, None, None, 0,
+                                   None) == 1
+    lib.attn_schedule_destroy(None)  # no-op

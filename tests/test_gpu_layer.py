@@ -149,3 +149,30 @@ def test_layer_full_size_sampled(bs, name):
         _check_outputs(wl, o_sub[b, tok, hi], o_ref, lse_sub[b, hi, tok], lse_ref)
     # untouched-by-sampling properties over the whole output
     assert torch.isfinite(o.float()).all()
+
+
+def test_schedule_steps_run_their_entry_plans(bs):
+    """A three-range step schedule (early: (6,8,8) tiles with a tile window;
+    middle: (4,4,4) top-k; late: (4,4,4) window with e4m3 Q/K) gives, at each
+    step, exactly what attn_layer gives with a stand-alone plan of that entry."""
+    grid = dict(B=1, heads=2, head_dim=128, T=9, H=12, W=13)
+    entries = [(0, dict(rule="window", win=(1, 1, 1), tile=(6, 8, 8))),
+               (10, dict(rule="topk", k=5)),
+               (30, dict(rule="window", win=(1, 1, 0), qk_fp8=True))]
+    sched = bs.Schedule(**grid, entries=entries)
+    wl = SMALL["ragged_topk"]
+    import dataclasses
+    wl = dataclasses.replace(wl, B=1, heads=2, T=9, H=12, W=13)
+    q, k, v = make_qkv(wl, "cuda")
+    ws = sched.workspace()
+    for step, which in ((0, 0), (9, 0), (10, 1), (29, 1), (30, 2), (500, 2)):
+        assert sched.plan_for(step) is sched.plans[which]
+        ref_plan = bs.Plan(**grid, **entries[which][1])
+        assert ref_plan.info.layer_workspace_bytes <= sched.workspace_bytes
+        o_ref = torch.empty_like(q)
+        bs.attn_layer(ref_plan, q, k, v, o_ref, ref_plan.workspace("layer"))
+        o = torch.full_like(q, float("nan"))
+        bs.attn_schedule_layer(sched, step, q, k, v, o, ws)
+        assert bs.attn_check_device_status(sched.plans[which]) == 0
+        assert torch.equal(o, o_ref), step
+    sched.close()
