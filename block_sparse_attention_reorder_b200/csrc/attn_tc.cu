@@ -38,6 +38,34 @@
 #include "internal.h"
 #include "tc_common.cuh"
 
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no
+// link-time dependency on the driver library).
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return (PFN_cuTensorMapEncodeTiled_v12000) nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }();
+  return fn;
+}
+
+bool bsattn_make_map_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int esz, int inner,
+                        uint64_t rows, int box_inner, int box_rows, CUtensorMapSwizzle sw) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)inner * esz};
+  cuuint32_t box[2] = {(cuuint32_t)box_inner, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 namespace {
 
 constexpr int kThreads = 192;
@@ -643,32 +671,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 }
 
 // ---------------------------------------------------------------- host side
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-      return (PFN_cuTensorMapEncodeTiled_v12000) nullptr;
-    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }();
-  return fn;
-}
-
-bool make_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int esz, int inner,
-              uint64_t rows, int box_inner, int box_rows, CUtensorMapSwizzle sw) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)inner * esz};
-  cuuint32_t box[2] = {(cuuint32_t)box_inner, (cuuint32_t)box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
 // Natural-layout tensor [B, T, H, W, Hh * D] as five dimensions, innermost
 // first, with a one-tile box of 64 columns (128 bytes, one swizzle span).
 bool make_map_nat(CUtensorMap* map, const void* base, const bsattn_plan* p) {
@@ -696,12 +698,12 @@ bsattn_status run(const bsattn_plan* p, const void* q, const void* k, const __nv
   CUtensorMap mq, mk, mv;
   const CUtensorMapDataType dqk = FP8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const CUtensorMapSwizzle sw = C::SWB == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
-  if (NQO && !FP8 ? !make_map_nat(&mq, q, p) : !make_map(&mq, q, dqk, C::ESZ, D, rows, C::SWB / C::ESZ, 64, sw))
+  if (NQO && !FP8 ? !make_map_nat(&mq, q, p) : !bsattn_make_map_2d(&mq, q, dqk, C::ESZ, D, rows, C::SWB / C::ESZ, 64, sw))
     return BSATTN_ERR_CUDA;
-  if (NKV && !FP8 ? !make_map_nat(&mk, k, p) : !make_map(&mk, k, dqk, C::ESZ, D, rows, C::SWB / C::ESZ, 64, sw))
+  if (NKV && !FP8 ? !make_map_nat(&mk, k, p) : !bsattn_make_map_2d(&mk, k, dqk, C::ESZ, D, rows, C::SWB / C::ESZ, 64, sw))
     return BSATTN_ERR_CUDA;
   if (NKV ? !make_map_nat(&mv, v, p)
-          : !make_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, rows, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+          : !bsattn_make_map_2d(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, rows, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B))
     return BSATTN_ERR_CUDA;
   // Step list, extents and (tiles of several chunks) chunk offsets.
   size_t smem = 1024 + C::OFF_DYN + (size_t)prm.bm_words * 8 + (size_t)prm.umax * (p->nchunk > 1 ? 12 : 8);

@@ -3,6 +3,7 @@
 
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cudaTypedefs.h>
 #include <stdint.h>
 #include <stddef.h>
 
@@ -83,8 +84,10 @@ bsattn_status launch_unreorder(const Geom& g, const __nv_bfloat16* x_tiled, __nv
                                const float* lse_tiled, float* lse_nat, cudaStream_t st);
 bsattn_status launch_quant_tiled(const Geom& g, const __nv_bfloat16* x_tiled, uint8_t* codes,
                                  float* scales, cudaStream_t st);
+// Block scores on the tensor cores (3xTF32); a bounded wait that gives up sets
+// BSATTN_DEVERR_TIMEOUT in *err.
 bsattn_status launch_block_scores(const Geom& g, const float* pq, const float* pk, float scale,
-                                  float* S, cudaStream_t st);
+                                  float* S, int* err, cudaStream_t st);
 bsattn_status launch_select_topk(int rows, int N, int k, const float* S, int32_t* idx,
                                  int32_t* cnt, int kmax, cudaStream_t st);
 bsattn_status launch_select_topp(int rows, int N, int k, double p, const float* S, int32_t* idx,
@@ -110,3 +113,6 @@ static inline bool layer_tiles_kv(const bsattn_plan* p) {
   return (long long)p->kmax * (p->nchunk == 1 ? 1 : (p->nchunk + 1) / 2) >= 64;
 }
 size_t attention_workspace_bytes(const bsattn_plan* p);
+// 2-D tiled tensor map over `rows` rows of `inner` elements of `esz` bytes.
+bool bsattn_make_map_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int esz, int inner,
+                        uint64_t rows, int box_inner, int box_rows, CUtensorMapSwizzle sw);

@@ -285,7 +285,7 @@ bsattn_status attn_block_scores(const bsattn_plan* p, const float* pq, const flo
   if (!p || !ok_ptr(pq) || !ok_ptr(pk) || !ok_ptr(S)) return BSATTN_ERR_INVALID_ARG;
   bsattn_status s = set_device(p);
   if (s) return s;
-  return launch_block_scores(make_geom(p), pq, pk, p->scale, S, (cudaStream_t)stream);
+  return launch_block_scores(make_geom(p), pq, pk, p->scale, S, p->d_err, (cudaStream_t)stream);
 }
 
 static bsattn_status select_core(const bsattn_plan* p, const float* S, int32_t* idx,
@@ -326,7 +326,7 @@ bsattn_status attn_select(const bsattn_plan* p, const void* q_nat, const void* k
   SelectWs w = carve_select(p, c);
   Geom g = make_geom(p);
   if ((s = launch_pool(g, (const __nv_bfloat16*)q_nat, w.pq, (const __nv_bfloat16*)k_nat, w.pk, st))) return s;
-  if ((s = launch_block_scores(g, w.pq, w.pk, p->scale, w.S, st))) return s;
+  if ((s = launch_block_scores(g, w.pq, w.pk, p->scale, w.S, p->d_err, st))) return s;
   return select_core(p, w.S, idx, cnt, st);
 }
 
@@ -412,7 +412,7 @@ bsattn_status attn_layer(const bsattn_plan* p, const void* q_nat, const void* k_
     if ((s = launch_reorder(g, (const __nv_bfloat16*)v_nat, w.vt, nullptr, nullptr, RO_WRITE_TILED, st))) return s;
     v = w.vt;
   }
-  if (pool && (s = launch_block_scores(g, w.sel.pq, w.sel.pk, p->scale, w.sel.S, st))) return s;
+  if (pool && (s = launch_block_scores(g, w.sel.pq, w.sel.pk, p->scale, w.sel.S, p->d_err, st))) return s;
   if ((s = select_core(p, w.sel.S, idx, cnt, st))) return s;
   return launch_attention(p, q, k, w.qs, w.ks, (const __nv_bfloat16*)v, idx, cnt, (__nv_bfloat16*)o_nat,
                           lse_nat, w.attn_ws, attention_workspace_bytes(p), st,

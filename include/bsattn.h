@@ -148,7 +148,11 @@ bsattn_status attn_unreorder(const bsattn_plan* plan, const void* x_tiled, void*
                              void* stream);
 
 /* Step 2: block scores S = softmax_scale * pooled_q . pooled_k^T per
- * (batch, head), fp32, accumulated in order d = 0..D-1. */
+ * (batch, head), fp32 out. Computed on the tensor cores as three TF32
+ * products per term (each input split as hi + lo, hi exact in TF32; hi*hi +
+ * hi*lo + lo*hi accumulated in fp32), within about 2^-20 of
+ * sum_d |q_d k_d| of the exact dot product; the result is deterministic. A
+ * bounded wait that gives up sets the device error word (TIMEOUT). */
 bsattn_status attn_block_scores(const bsattn_plan* plan, const float* pooled_q,
                                 const float* pooled_k, float* scores, void* stream);
 

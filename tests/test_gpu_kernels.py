@@ -322,3 +322,67 @@ def tiling_lse_natural(lse_t, wl, plan):
     out = np.stack([tiling.unreorder(x[:, h:h + 1, :, :, None], wl.T, wl.H, wl.W, wl.tile)[..., 0, 0]
                     for h in range(wl.heads)], axis=1)
     return torch.from_numpy(out.astype(np.float32))
+
+
+def _forward_vs_oracle(bs, wl, lists, tile=(4, 4, 4)):
+    """attn_forward on given lists (bf16) against the oracle; returns (O, lse) natural."""
+    plan = _plan(bs, wl, qk_fp8=False)
+    q, k, v, qn, kn, vn = _oracle_inputs(wl)
+    idx, cnt = lists_to_device(lists, plan.kmax)
+    tiled = []
+    for x in (q, k, v):
+        t = torch.empty(plan.tiled_shape(), dtype=torch.bfloat16, device="cuda")
+        bs.attn_reorder(plan, x.cuda(), t)
+        tiled.append(t)
+    o = torch.empty(plan.tiled_shape(), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((wl.B, wl.heads, plan.N, plan.V), dtype=torch.float32, device="cuda")
+    si, sc = plan.list_shapes()
+    bs.attn_forward(plan, tiled[0], tiled[1], tiled[2], idx.view(si), cnt.view(sc), o, lse)
+    assert bs.attn_check_device_status(plan) == 0
+    o_ref, lse_ref = attention.attention_full(qn, kn, vn, lists, wl.T, wl.H, wl.W, wl.tile)
+    o_nat = tiling.unreorder(to64(o), wl.T, wl.H, wl.W, wl.tile)
+    err = np.abs(o_nat - o_ref)
+    assert err.max() <= 2e-2 and err.mean() <= 2e-3, (err.max(), err.mean())
+    lse_nat = tiling_lse_natural(lse, wl, plan).numpy().astype(np.float64)
+    finite = np.isfinite(lse_ref)
+    np.testing.assert_array_equal(np.isfinite(lse_nat), finite)
+    np.testing.assert_allclose(lse_nat[finite], lse_ref[finite], rtol=0, atol=2e-2)
+    return o_nat, lse_nat, o_ref
+
+
+def test_forward_single_tile_grid(bs):
+    """A grid smaller than one tile: N = 1, most slots padding."""
+    from block_sparse_attention_reorder_b200.datagen import Workload
+    wl = Workload("one_tile", 1, 2, 128, 3, 2, 3, "topk", k=1, recipe="iid", seed=21)
+    _forward_vs_oracle(bs, wl, [np.array([0])] * 2)
+
+
+def test_forward_all_tiles_kept_is_dense_attention(bs):
+    """k = N: every tile keeps every tile, which is dense attention over the
+    real tokens (checked by the oracle against torch SDPA in fp64)."""
+    from block_sparse_attention_reorder_b200.datagen import Workload
+    wl = Workload("dense", 1, 2, 64, 7, 6, 9, "topk", k=12, recipe="iid", seed=22)
+    plan = _plan(bs, wl)
+    assert plan.N == 12
+    _forward_vs_oracle(bs, wl, [np.arange(12)] * (2 * 12))
+
+
+def test_forward_empty_lists_give_zero_rows(bs):
+    """Query tiles with an empty kept list: O rows are zero and lse is -inf,
+    as in the plain definition (a softmax over no keys contributes nothing);
+    the other tiles are unaffected."""
+    from block_sparse_attention_reorder_b200.datagen import Workload
+    wl = Workload("empty_rows", 1, 2, 128, 7, 10, 13, "topk", k=3, recipe="iid", seed=23)
+    plan = _plan(bs, wl)
+    rng = np.random.default_rng(5)
+    lists = []
+    for r in range(2 * plan.N):
+        lists.append(np.array([], dtype=np.int64) if r % 3 == 0 else
+                     np.sort(rng.choice(plan.N, size=3, replace=False)))
+    o_nat, lse_nat, o_ref = _forward_vs_oracle(bs, wl, lists)
+    tid, _ = tiling.token_tile_and_row(wl.T, wl.H, wl.W)
+    for h in range(2):
+        empty = [i for i in range(plan.N) if (h * plan.N + i) % 3 == 0]
+        tok = np.isin(tid, empty)
+        assert np.all(o_nat[0, tok, h] == 0)
+        assert np.all(np.isneginf(lse_nat[0, h, tok]))
