@@ -23,7 +23,10 @@ values (see ``e4m3``) and keeps V as given.
 Parity: pinned against torch's scaled_dot_product_attention in fp64 on CPU
 for the all-kept mask, a pure-Python triple loop on tiny inputs, softmax
 normalisation, the single-key closed form and in-tile permutation
-invariance (tests/test_oracle_attention.py).
+invariance (tests/test_oracle_attention.py). The backward
+(``dense_masked_backward``) is pinned by central finite differences of the
+forward on tiny masked cases and by torch autograd of fp64 SDPA for the
+all-kept mask.
 """
 
 from __future__ import annotations
@@ -104,6 +107,48 @@ def attention_rows(q_nat, k_nat, v_nat, lists, T, H, W, tile=(4, 4, 4), scale=No
                               scale)
         out[(b, h, i)] = (qi, o, lse)
     return out
+
+
+def dense_masked_backward(q: np.ndarray, k: np.ndarray, v: np.ndarray, allowed: np.ndarray,
+                          scale: float, do: np.ndarray):
+    """Gradients of L = sum(do * o) for o = dense_masked(q, k, v, allowed, scale)[0].
+
+    Plain differentiation of softmax attention (the trainable block-sparse
+    attention that "Faster Video Diffusion with Trainable Sparse Attention"
+    trains with, reproducibility record, Research Type row): with P the masked
+    softmax, dV = P^T dO, dP = dO V^T, dS = P * (dP - rowsum(dO * O)),
+    dQ = scale dS K, dK = scale dS^T Q. A row with no allowed key has P = 0 and
+    contributes nothing. Returns (dq [Lq, D], dk [Lk, D], dv [Lk, D]) in fp64.
+    """
+    q, k, v, do = (x.astype(np.float64) for x in (q, k, v, do))
+    s = scale * (q @ k.T)
+    s = np.where(allowed, s, -np.inf)
+    m = s.max(axis=1, keepdims=True)
+    m_safe = np.where(np.isfinite(m), m, 0.0)
+    e = np.exp(s - m_safe)
+    l = e.sum(axis=1, keepdims=True)
+    p = e / np.where(l > 0, l, 1.0)
+    o = p @ v
+    dv = p.T @ do
+    dp = do @ v.T
+    ds = p * (dp - (do * o).sum(axis=1, keepdims=True))
+    return scale * (ds @ k), scale * (ds.T @ q), dv
+
+
+def attention_backward_full(q_nat, k_nat, v_nat, do_nat, lists, T, H, W, tile=(4, 4, 4), scale=None):
+    """Gradients of the whole layer through the materialised [L, L] mask (small
+    grids only): natural [B, L, heads, D] in, (dq, dk, dv) natural fp64 out."""
+    B, L, Hh, D = q_nat.shape
+    nb = tiling.n_blocks(T, H, W, tile)
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    dq, dk, dv = (np.zeros((B, L, Hh, D), dtype=np.float64) for _ in range(3))
+    for b in range(B):
+        for h in range(Hh):
+            r0 = (b * Hh + h) * nb
+            mask = token_mask(lists[r0:r0 + nb], T, H, W, tile)
+            dq[b, :, h], dk[b, :, h], dv[b, :, h] = dense_masked_backward(
+                q_nat[b, :, h], k_nat[b, :, h], v_nat[b, :, h], mask, scale, do_nat[b, :, h])
+    return dq, dk, dv
 
 
 def fp8_qk(q_nat, k_nat, T, H, W, tile=(4, 4, 4)):

@@ -132,3 +132,48 @@ def test_self_tile_lists_match_coordinate_blocks(tile):
         p = np.exp(s - s.max())
         ref = (p[:, None] * v[0, keys, 0]).sum(axis=0) / p.sum()
         np.testing.assert_allclose(o[0, n, 0], ref, rtol=1e-12, atol=1e-13)
+
+
+def test_backward_matches_central_differences():
+    """dq, dk, dv of L = sum(do * o) against central differences of the
+    forward, on a masked case (some rows attend nothing, some partially)."""
+    rng = np.random.default_rng(9)
+    q, do = rng.standard_normal((6, 5)), rng.standard_normal((6, 5))  # 6 queries, D = 5
+    k, v = rng.standard_normal((5, 5)), rng.standard_normal((5, 5))    # 5 keys
+    allowed = rng.random((6, 5)) < 0.6
+    allowed[2] = False  # a row with no key
+    scale = 0.37
+    dq, dk, dv = attention.dense_masked_backward(q, k, v, allowed, scale, do)
+
+    def loss(qq, kk, vv):
+        return float((attention.dense_masked(qq, kk, vv, allowed, scale)[0] * do).sum())
+
+    h = 1e-6
+    for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        num = np.zeros_like(x)
+        for idx in np.ndindex(*x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            args_p = {"q": (xp, k, v), "k": (q, xp, v), "v": (q, k, xp)}[name]
+            args_m = {"q": (xm, k, v), "k": (q, xm, v), "v": (q, k, xm)}[name]
+            num[idx] = (loss(*args_p) - loss(*args_m)) / (2 * h)
+        np.testing.assert_allclose(g, num, rtol=1e-6, atol=1e-8, err_msg=name)
+    assert np.all(dq[2] == 0)
+
+
+def test_backward_all_kept_equals_torch_autograd():
+    """All tiles kept: the layer backward is dense attention's, as torch
+    autograd of fp64 scaled_dot_product_attention computes it."""
+    T, H, W = 5, 6, 7
+    rng = np.random.default_rng(10)
+    q, k, v, do = (rng.standard_normal((1, T * H * W, 2, 8)) for _ in range(4))
+    nb = tiling.n_blocks(T, H, W)
+    dq, dk, dv = attention.attention_backward_full(q, k, v, do, [np.arange(nb)] * (2 * nb), T, H, W)
+    for h in range(2):
+        tq, tk, tv = (torch.from_numpy(x[0, :, h].copy()).requires_grad_(True) for x in (q, k, v))
+        o = torch.nn.functional.scaled_dot_product_attention(tq[None, None], tk[None, None], tv[None, None])
+        o.backward(torch.from_numpy(do[0, :, h])[None, None])
+        np.testing.assert_allclose(dq[0, :, h], tq.grad.numpy(), rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(dk[0, :, h], tk.grad.numpy(), rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(dv[0, :, h], tv.grad.numpy(), rtol=1e-10, atol=1e-12)
