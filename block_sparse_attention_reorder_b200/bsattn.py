@@ -55,7 +55,8 @@ class Info(ctypes.Structure):
                 ("softmax_scale", ctypes.c_float),
                 ("select_workspace_bytes", ctypes.c_size_t),
                 ("forward_workspace_bytes", ctypes.c_size_t),
-                ("layer_workspace_bytes", ctypes.c_size_t)]
+                ("layer_workspace_bytes", ctypes.c_size_t),
+                ("backward_workspace_bytes", ctypes.c_size_t)]
 
 
 def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
@@ -81,6 +82,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "attn_forward_natural": [P, P, P, P, P, P, P, P, P, P, P, Z, P],
         "attn_layer": [P, P, P, P, P, P, P, P, P, Z, P],
         "attn_check_device_status": [P, P],
+        "attn_backward": [P, P, P, P, P, P, P, P, P, P, P, P, P, Z, P],
         "attn_schedule_create": [ctypes.POINTER(ScheduleEntry), I, ctypes.POINTER(P)],
         "attn_schedule_destroy": [P],
         "attn_schedule_plan": [P, I, ctypes.POINTER(P)],
@@ -101,7 +103,8 @@ EXPORTED = ("attn_plan_create", "attn_plan_destroy", "attn_plan_info", "attn_sta
             "attn_select_from_scores", "attn_select", "attn_select_static", "attn_quantize_e4m3",
             "attn_forward", "attn_forward_natural",
             "attn_layer", "attn_check_device_status", "attn_schedule_create", "attn_schedule_destroy",
-            "attn_schedule_plan", "attn_schedule_workspace_bytes", "attn_schedule_layer")
+            "attn_schedule_plan", "attn_schedule_workspace_bytes", "attn_schedule_layer",
+            "attn_backward")
 
 
 def _check(code: int, where: str):
@@ -190,7 +193,8 @@ class Plan:
     def workspace(self, which="layer", device="cuda"):
         nbytes = {"select": self.info.select_workspace_bytes,
                   "forward": self.info.forward_workspace_bytes,
-                  "layer": self.info.layer_workspace_bytes}[which]
+                  "layer": self.info.layer_workspace_bytes,
+                  "backward": self.info.backward_workspace_bytes}[which]
         return torch.empty(max(int(nbytes), 16), dtype=torch.uint8, device=device)
 
 
@@ -394,6 +398,20 @@ def attn_layer(plan: Plan, q_nat, k_nat, v_nat, o_nat, ws, lse_nat=None, idx=Non
     _check(_lib.attn_layer(plan.handle, _ptr(q_nat), _ptr(k_nat), _ptr(v_nat), _ptr(o_nat),
                            _ptr(lse_nat), _ptr(idx), _ptr(cnt), _ptr(ws),
                            ws.numel() * ws.element_size(), _stream(stream)), "attn_layer")
+
+
+def attn_backward(plan: Plan, q_t, k_t, v_t, o_t, do_t, lse_t, idx, cnt, dq_t, dk_t, dv_t, ws, stream=None):
+    ts = plan.tiled_shape()
+    for name, t in (("q", q_t), ("k", k_t), ("v", v_t), ("o", o_t), ("do", do_t), ("dq", dq_t), ("dk", dk_t),
+                    ("dv", dv_t)):
+        _want(t, torch.bfloat16, ts, name)
+    _want(lse_t, torch.float32, (plan.B, plan.heads, plan.N, plan.V), "lse")
+    si, sc = plan.list_shapes()
+    _want(idx, torch.int32, si, "idx")
+    _want(cnt, torch.int32, sc, "cnt")
+    _check(_lib.attn_backward(plan.handle, _ptr(q_t), _ptr(k_t), _ptr(v_t), _ptr(o_t), _ptr(do_t), _ptr(lse_t),
+                              _ptr(idx), _ptr(cnt), _ptr(dq_t), _ptr(dk_t), _ptr(dv_t), _ptr(ws),
+                              ws.numel() * ws.element_size(), _stream(stream)), "attn_backward")
 
 
 def attn_check_device_status(plan: Plan, stream=None) -> int:

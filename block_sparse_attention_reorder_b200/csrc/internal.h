@@ -113,6 +113,17 @@ static inline bool layer_tiles_kv(const bsattn_plan* p) {
   return (long long)p->kmax * (p->nchunk == 1 ? 1 : (p->nchunk + 1) / 2) >= 64;
 }
 size_t attention_workspace_bytes(const bsattn_plan* p);
+// Scratch of the backward pass (carved from the caller's workspace).
+struct BackwardWs {
+  float* delta;    // [B, Hh, N, 64] rowsum(dO * O)
+  uint32_t* bm;    // [B, Hh, N, ceil(N/32)] transposed kept-list bitmaps
+  int32_t* idxT;   // [B, Hh, N, N] query tiles keeping each key tile, ascending
+  int32_t* cntT;   // [B, Hh, N]
+};
+bsattn_status launch_backward(const bsattn_plan* p, const void* q, const void* k, const void* v, const void* o,
+                              const void* d_o, const float* lse, const int32_t* idx, const int32_t* cnt, void* dq,
+                              void* dk, void* dv, const BackwardWs& w, cudaStream_t st);
+
 // 2-D tiled tensor map over `rows` rows of `inner` elements of `esz` bytes.
 bool bsattn_make_map_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int esz, int inner,
                         uint64_t rows, int box_inner, int box_rows, CUtensorMapSwizzle sw);

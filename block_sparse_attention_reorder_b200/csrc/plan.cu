@@ -79,6 +79,16 @@ LayerWs carve_layer(const bsattn_plan* p, Carve& c) {
   return w;
 }
 
+BackwardWs carve_backward(const bsattn_plan* p, Carve& c) {
+  const size_t rows = (size_t)p->desc.B * p->desc.heads * p->N;
+  BackwardWs w;
+  w.delta = (float*)c.take(rows * 64 * sizeof(float));
+  w.bm = (uint32_t*)c.take(rows * ((p->N + 31) / 32) * sizeof(uint32_t));
+  w.idxT = (int32_t*)c.take(rows * p->N * sizeof(int32_t));
+  w.cntT = (int32_t*)c.take(rows * sizeof(int32_t));
+  return w;
+}
+
 bool ok_ptr(const void* x) { return x != nullptr && aligned16(x); }
 
 bsattn_status set_device(const bsattn_plan* p) {
@@ -246,6 +256,11 @@ bsattn_status attn_plan_info(const bsattn_plan* p, bsattn_info* o) {
     carve_layer(p, c);
     o->layer_workspace_bytes = align_up(c.off, 256);
   }
+  {
+    Carve c(nullptr);
+    carve_backward(p, c);
+    o->backward_workspace_bytes = align_up(c.off, 256);
+  }
   return BSATTN_OK;
 }
 
@@ -352,6 +367,23 @@ bsattn_status attn_forward(const bsattn_plan* p, const void* q, const void* k, c
   if (s) return s;
   return launch_attention(p, q, k, qs, ks, (const __nv_bfloat16*)v, idx, cnt, (__nv_bfloat16*)o,
                           lse, ws, ws_bytes, (cudaStream_t)stream, AttnLayout::Tiled);
+}
+
+bsattn_status attn_backward(const bsattn_plan* p, const void* q, const void* k, const void* v, const void* o,
+                            const void* d_o, const float* lse, const int32_t* idx, const int32_t* cnt, void* dq,
+                            void* dk, void* dv, void* ws, size_t ws_bytes, void* stream) {
+  if (!p || !ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(o) || !ok_ptr(d_o) || !ok_ptr(lse) ||
+      !ok_ptr(idx) || !ok_ptr(cnt) || !ok_ptr(dq) || !ok_ptr(dk) || !ok_ptr(dv))
+    return BSATTN_ERR_INVALID_ARG;
+  if (p->desc.qk_fp8 || p->V != 64) return BSATTN_ERR_UNSUPPORTED;
+  bsattn_info info;
+  attn_plan_info(p, &info);
+  if (!ws || !aligned16(ws) || ws_bytes < info.backward_workspace_bytes) return BSATTN_ERR_WORKSPACE;
+  bsattn_status s = set_device(p);
+  if (s) return s;
+  Carve c(ws);
+  const BackwardWs w = carve_backward(p, c);
+  return launch_backward(p, q, k, v, o, d_o, lse, idx, cnt, dq, dk, dv, w, (cudaStream_t)stream);
 }
 
 bsattn_status attn_forward_natural(const bsattn_plan* p, const void* q, const void* k, const float* qs,

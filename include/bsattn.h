@@ -102,6 +102,7 @@ typedef struct {
   size_t select_workspace_bytes;  /* attn_select                              */
   size_t forward_workspace_bytes; /* attn_forward                             */
   size_t layer_workspace_bytes;   /* attn_layer                               */
+  size_t backward_workspace_bytes; /* attn_backward                           */
 } bsattn_info;
 
 typedef struct bsattn_plan bsattn_plan;
@@ -237,6 +238,23 @@ bsattn_status attn_forward_natural(const bsattn_plan* plan, const void* q, const
 bsattn_status attn_layer(const bsattn_plan* plan, const void* q_nat, const void* k_nat,
                          const void* v_nat, void* o_nat, float* lse_nat, int32_t* idx_out,
                          int32_t* cnt_out, void* ws, size_t ws_bytes, void* stream);
+
+/* Backward of attn_forward (trainable block-sparse attention: "Faster Video
+ * Diffusion with Trainable Sparse Attention", reproducibility record,
+ * Research Type row). Tiled bf16 q, k, v, the forward's tiled bf16 o and fp32
+ * lse [B, Hh, N, 64], the incoming gradient d_o (tiled bf16) and the kept
+ * lists the forward used; writes tiled bf16 dq, dk, dv. With P the masked
+ * softmax recomputed from q, k and lse: dV = P^T dO, dS = P * (dO V^T -
+ * rowsum(dO * O)), dQ = scale dS K, dK = scale dS^T Q, over kept tile pairs
+ * and real (unpadded) tokens; rows of padded slots get zero gradients. P and
+ * dS are rounded to bf16 for the products (fp32 accumulation). Tiles of 64
+ * tokens and bf16 Q/K only (UNSUPPORTED otherwise). `ws` must hold
+ * info.backward_workspace_bytes (rowsum, transposed lists). A list entry
+ * outside [0, N) sets the device error word and is skipped. */
+bsattn_status attn_backward(const bsattn_plan* plan, const void* q, const void* k, const void* v,
+                            const void* o, const void* d_o, const float* lse, const int32_t* idx,
+                            const int32_t* cnt, void* dq, void* dk, void* dv, void* ws,
+                            size_t ws_bytes, void* stream);
 
 /* Synchronise `stream`, read and clear the plan's device error word.
  * Returns OK, TIMEOUT or INTERNAL (bad list entry), or CUDA. */

@@ -71,6 +71,8 @@ def test_null_plan_and_null_pointers_are_invalid():
                             None) == 1
     assert lib.attn_layer(None, None, None, None, None, None, None, None, None, 0, None) == 1
     assert lib.attn_check_device_status(None, None) == 1
+    assert lib.attn_backward(None, None, None, None, None, None, None, None, None, None, None, None, None, 0,
+                             None) == 1
     assert lib.attn_plan_info(None, None) == 1
     lib.attn_plan_destroy(None)  # no-op
 

@@ -1,0 +1,75 @@
+"""Backward parity: attn_backward (tiled) against the oracle's gradients of
+the plain masked-softmax definition, on small ragged grids."""
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_attention_reorder_b200.datagen import make_qkv
+from oracle import attention, tiling
+from tests.helpers import SMALL, lists_to_device, to64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def bs():
+    from block_sparse_attention_reorder_b200 import bsattn
+    assert torch.cuda.is_available()
+    return bsattn
+
+
+def _grad_close(got, ref, name):
+    err = got - ref
+    rel = np.linalg.norm(err) / max(np.linalg.norm(ref), 1e-30)
+    assert rel <= 1e-2, (name, rel)
+    assert np.abs(err).max() <= 3e-2 * np.abs(ref).max(), (name, np.abs(err).max(), np.abs(ref).max())
+
+
+@pytest.mark.parametrize("name", ["tiny_d64", "ragged_topk", "ragged_topp", "ragged_bf16_window"])
+def test_backward_against_oracle(bs, name):
+    wl = SMALL[name]
+    plan = bs.Plan.for_workload(wl)
+    q, k, v = make_qkv(wl, "cpu")
+    g = torch.Generator(device="cpu").manual_seed(100 + wl.seed)
+    d_o = torch.randn(q.shape, generator=g).to(torch.bfloat16)
+    qn, kn, vn, don = (to64(x) for x in (q, k, v, d_o))
+    _, _, _, lists = attention.route(qn, kn, wl.T, wl.H, wl.W, wl.rule, tile=wl.tile, k=wl.k, p=wl.p,
+                                     half=wl.win, score_dtype=np.float32)
+    idx, cnt = lists_to_device(lists, plan.kmax)
+    si, sc = plan.list_shapes()
+    idx, cnt = idx.view(si), cnt.view(sc)
+    ts = plan.tiled_shape()
+    tiled = []
+    for x in (q, k, v, d_o):
+        t = torch.empty(ts, dtype=torch.bfloat16, device="cuda")
+        bs.attn_reorder(plan, x.cuda(), t)
+        tiled.append(t)
+    qt, kt, vt, dot = tiled
+    ot = torch.empty(ts, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((wl.B, wl.heads, plan.N, plan.V), dtype=torch.float32, device="cuda")
+    bs.attn_forward(plan, qt, kt, vt, idx, cnt, ot, lse)
+    dq, dk, dv = (torch.full(ts, float("nan"), dtype=torch.bfloat16, device="cuda") for _ in range(3))
+    bs.attn_backward(plan, qt, kt, vt, ot, dot, lse, idx, cnt, dq, dk, dv, plan.workspace("backward"))
+    assert bs.attn_check_device_status(plan) == 0
+    rq, rk, rv = attention.attention_backward_full(qn, kn, vn, don, lists, wl.T, wl.H, wl.W, wl.tile)
+    for name_, got, ref in (("dq", dq, rq), ("dk", dk, rk), ("dv", dv, rv)):
+        nat = tiling.unreorder(to64(got), wl.T, wl.H, wl.W, wl.tile)
+        _grad_close(nat, ref, name_)
+    # Padded slots carry zero gradients.
+    valid = torch.from_numpy(tiling.tile_valid_rows(wl.T, wl.H, wl.W, wl.tile)).cuda()
+    for t in (dq, dk, dv):
+        assert torch.all(t[:, :, ~valid] == 0)
+
+
+def test_backward_rejects_unsupported_plans(bs):
+    wl = SMALL["ragged_window_fp8"]
+    plan = bs.Plan.for_workload(wl)  # e4m3 Q/K
+    ts = plan.tiled_shape()
+    x = torch.zeros(ts, dtype=torch.bfloat16, device="cuda")
+    lse = torch.zeros((wl.B, wl.heads, plan.N, plan.V), dtype=torch.float32, device="cuda")
+    si, sc = plan.list_shapes()
+    idx = torch.zeros(si, dtype=torch.int32, device="cuda")
+    cnt = torch.zeros(sc, dtype=torch.int32, device="cuda")
+    with pytest.raises(bs.BsattnError) as e:
+        bs.attn_backward(plan, x, x, x, x, x, lse, idx, cnt, x, x, x, plan.workspace("backward"))
+    assert e.value.code == 2
