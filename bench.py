@@ -47,6 +47,7 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--no-backward", action="store_true", help="skip the backward-pass timing")
     ap.add_argument("--heads", type=int, default=0,
                     help="run a copy of the workload with this many heads (small profiling cases)")
     return ap.parse_args()
@@ -194,24 +195,31 @@ class ClockSampler:
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, device_index: int):
-        self.proc = None
+        """Starts sampling every 100 ms and returns once the first sample is
+        in, so that the samples cover the work that follows."""
+        self.proc, self.first = None, ""
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
                  "-lms", "100", "-i", str(device_index)],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.first = self.proc.stdout.readline()
         except Exception:
             self.proc = None
 
     def stop(self):
+        """Stops after two more sampling periods (a short timed region still
+        gets samples on both sides) and summarises every sample taken."""
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
         self.proc.terminate()
         try:
             out, _ = self.proc.communicate(timeout=5)
         except Exception:
             self.proc.kill()
             out, _ = self.proc.communicate()
+        out = self.first + out
         sm, smax, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in out.strip().splitlines():
@@ -417,6 +425,8 @@ def main():
         return 0
 
     pk = peaks()
+    # The backward of the same layer (rank 0; not part of the timed step).
+    bwd = None if args.no_backward else backward_timing(bsattn, plan, wl, q, k, v, idx, cnt, flush, stream, pk)
     attn_ms = comp["attention"]
     achieved = flops / (attn_ms * 1e-3) / 1e12
     nch2 = (plan.V // 64) ** 2  # 64 x 64 chunk pairs per kept tile pair
@@ -451,6 +461,7 @@ def main():
                      "peak_note": f"{pk['source']} bf16 burst (kernel timed alone)",
                      "traffic": measured_traffic(wl.name) if args.heads == 0 else None},
         "memory_kernels": memory_kernel_rates(wl, plan, comp, pk),
+        "backward": bwd,
         "e2e": e2e,
         "gpu_launches": launches_per_step(wl, plan) * args.steps,
         "clocks": clocks,
@@ -540,6 +551,52 @@ def component_timing(bsattn, plan, wl, q, k, v, flush, stream, reps=20):
     out = {n: acc[n] / reps for n in names if acc[n] > 0}
     out["attention"] = out["attention_tiled" if tiles_kv else "attention_natural"]
     return out
+
+
+def backward_timing(bsattn, plan, wl, q, k, v, idx, cnt, flush, stream, pk):
+    """attn_backward on the layer's kept lists (tiled inputs, the forward's O
+    and lse, a seeded random dO): device time and TFLOP/s counting five
+    64x64xD products per kept pair (S, dP, dV, dK, dQ; the kernels recompute
+    S and dP once more). None where the backward does not apply."""
+    if wl.qk_fp8 or plan.V != 64:
+        return None
+    ts = plan.tiled_shape()
+    g = torch.Generator(device="cuda").manual_seed(7)
+    d_o = torch.randn(q.shape, generator=g, device="cuda").to(torch.bfloat16)
+    t = [torch.empty(ts, dtype=torch.bfloat16, device="cuda") for _ in range(4)]
+    for x, y in zip((q, k, v, d_o), t):
+        bsattn.attn_reorder(plan, x, y, None, stream)
+    o_t = torch.empty(ts, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((wl.B, wl.heads, plan.N, plan.V), dtype=torch.float32, device="cuda")
+    bsattn.attn_forward(plan, t[0], t[1], t[2], idx, cnt, o_t, lse, stream=stream)
+    grads = [torch.empty(ts, dtype=torch.bfloat16, device="cuda") for _ in range(3)]
+    ws = plan.workspace("backward")
+
+    def run():
+        bsattn.attn_backward(plan, t[0], t[1], t[2], o_t, t[3], lse, idx, cnt, *grads, ws, stream=stream)
+
+    run()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    run()
+    b.record(stream)
+    torch.cuda.synchronize()
+    reps = 3 if a.elapsed_time(b) > 50 else 10
+    total = 0.0
+    for _ in range(reps):
+        flush.fill_(1.0)
+        a.record(stream)
+        run()
+        b.record(stream)
+        torch.cuda.synchronize()
+        total += a.elapsed_time(b)
+    ms = total / reps
+    if bsattn.attn_check_device_status(plan) != 0:
+        raise SystemExit("device error word set in the backward")
+    tf = 2.5 * kept_pairs_from_counts(cnt) * pair_flops(wl.head_dim) / (ms * 1e-3) / 1e12
+    return {"ms": ms, "tflops": tf, "frac": tf / pk["bf16_tflops"],
+            "note": "attn_backward (dQ, dK, dV; bf16 mma.sync kernels), five 64x64xD products per kept pair"}
 
 
 def memory_kernel_rates(wl, plan, comp, pk):
