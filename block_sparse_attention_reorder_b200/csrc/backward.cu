@@ -8,11 +8,12 @@
 //   dK_j += scale dS_ij^T Q_i,  dQ_i += scale dS_ij K_j
 // over the kept tile pairs (i, j). Two kernels avoid atomics: one per key
 // tile walks the query tiles that keep it (a transposed list built from
-// bitmaps, ascending) and accumulates dK_j and dV_j; one per query tile walks
-// its own list and accumulates dQ_i. Both run on the warp-level bf16 tensor
-// core instruction (mma.sync m16n8k16, fp32 accumulate): each of four warps
-// owns 16 rows of the tile, so no cross-warp reduction is needed. P and dS
-// are rounded to bf16 for the products, as the forward rounds P.
+// bitmaps, ascending) and accumulates dK_j and dV_j (here, on the warp-level
+// bf16 tensor core instruction mma.sync m16n8k16 with fp32 accumulation;
+// each of four warps owns 16 rows of the tile, so no cross-warp reduction is
+// needed); one per pair of query tiles walks their kept lists and
+// accumulates dQ_i on tcgen05 (csrc/bwd_tc.cu). P and dS are rounded to bf16
+// for the products, as the forward rounds P.
 //
 // Tiles of 64 tokens (tiled layout [B, Hh, N, 64, D], D in {64, 128}); padded
 // key and query slots are masked from their tile's real extent.
@@ -316,85 +317,6 @@ bwd_dkdv_kernel(Geom g, const __nv_bfloat16* __restrict__ q, const __nv_bfloat16
   store_rows<D>(dv + tj * D, dva, w, lane, 1.f);
 }
 
-// dQ_i: one CTA per (query tile i, head, batch); warp w owns query rows
-// 16w .. 16w + 15 and walks the key tiles i keeps.
-template <int D>
-__global__ void __launch_bounds__(kThreadsB)
-bwd_dq_kernel(Geom g, const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
-              const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ d_o, const float* __restrict__ lse,
-              const float* __restrict__ delta, const int32_t* __restrict__ idx, const int32_t* __restrict__ cnt,
-              int kmax, float c_log2, float scale, __nv_bfloat16* __restrict__ dq, int* err) {
-  // Q_i, dO_i, then two stages of (K_j, V_j).
-  extern __shared__ __align__(16) uint8_t sm[];
-  constexpr int STAGE = 2 * TileS<D>::BYTES;
-  uint8_t* Qs = sm;
-  uint8_t* Os = Qs + TileS<D>::BYTES;
-  uint8_t* stage0 = Os + TileS<D>::BYTES;
-  const int i = blockIdx.x, head = blockIdx.y, b = blockIdx.z;
-  const size_t bh = (size_t)b * g.Hh + head;
-  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const size_t ti = (bh * g.N + i) * kRowsT;
-  const size_t row = bh * g.N + i;
-  const int nk = min(max(cnt[row], 0), kmax);
-  const int32_t* klist = idx + row * kmax;
-  // A bad entry is loaded as tile 0 (in bounds) and skipped below.
-  auto key_of = [&](int e) { const int j = klist[e]; return (j < 0 || j >= g.N) ? -1 : j; };
-  auto load_key = [&](int e) {
-    const int j = max(key_of(e), 0);
-    uint8_t* st = stage0 + (e & 1) * STAGE;
-    const size_t tj = (bh * g.N + j) * kRowsT;
-    load_tile<D>(st, k + tj * D);
-    load_tile<D>(st + TileS<D>::BYTES, v + tj * D);
-  };
-  load_tile<D>(Qs, q + ti * D);
-  load_tile<D>(Os, d_o + ti * D);
-  if (nk > 0) load_key(0);
-  cp_async_commit();
-  const uint64_t qreal = real_rows(g, i);
-  const int qr0 = w * 16 + (lane >> 2);
-  const bool qv0 = (qreal >> qr0) & 1, qv1 = (qreal >> (qr0 + 8)) & 1;
-  const float l20 = lse[ti + qr0] * 1.4426950408889634f, l21 = lse[ti + qr0 + 8] * 1.4426950408889634f;
-  const float d0 = delta[ti + qr0], d1 = delta[ti + qr0 + 8];
-  float dqa[D / 8][4];
-#pragma unroll
-  for (int n = 0; n < D / 8; ++n) dqa[n][0] = dqa[n][1] = dqa[n][2] = dqa[n][3] = 0.f;
-  for (int e = 0; e < nk; ++e) {
-    if (e + 1 < nk) load_key(e + 1);
-    cp_async_commit();
-    cp_async_wait<1>();
-    __syncthreads();
-    const int j = key_of(e);
-    if (j < 0) {  // uniform over the CTA
-      if (threadIdx.x == 0) atomicOr(err, BSATTN_DEVERR_BAD_INDEX);
-      __syncthreads();
-      continue;
-    }
-    uint8_t* Ks = stage0 + (e & 1) * STAGE;
-    uint8_t* Vs = Ks + TileS<D>::BYTES;
-    const uint64_t kreal = real_rows(g, j);
-    float s[8][4], dp[8][4];
-    xyt<D>(Qs, Ks, w, lane, s);   // S = Q K^T
-    xyt<D>(Os, Vs, w, lane, dp);  // dP = dO V^T
-#pragma unroll
-    for (int t = 0; t < 8; ++t) {
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int kc = t * 8 + (lane & 3) * 2 + h;  // key column
-        const bool kvv = (kreal >> kc) & 1;
-        const float p0 = (qv0 && kvv) ? ex2(s[t][h] * c_log2 - l20) : 0.f;
-        const float p1 = (qv1 && kvv) ? ex2(s[t][2 + h] * c_log2 - l21) : 0.f;
-        dp[t][h] = p0 * (dp[t][h] - d0);
-        dp[t][2 + h] = p1 * (dp[t][2 + h] - d1);
-      }
-    }
-    uint32_t sf[4][4];
-    to_afrag(dp, sf);
-    az<D>(sf, Ks, lane, dqa);  // dQ += dS K
-    __syncthreads();  // this stage is refilled two iterations on
-  }
-  store_rows<D>(dq + ti * D, dqa, w, lane, scale);
-}
-
 template <int D>
 bsattn_status run_backward(const bsattn_plan* p, const __nv_bfloat16* q, const __nv_bfloat16* k,
                            const __nv_bfloat16* v, const __nv_bfloat16* o, const __nv_bfloat16* d_o, const float* lse,
@@ -409,17 +331,14 @@ bsattn_status run_backward(const bsattn_plan* p, const __nv_bfloat16* q, const _
   bwd_bitmap_kernel<<<(unsigned)rows, 64, 0, st>>>(idx, cnt, g.N, p->kmax, words, w.bm, p->d_err);
   bwd_compact_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(w.bm, g.N, words, rows, w.idxT, w.cntT);
   const size_t smem_kv = 2 * (size_t)TileS<D>::BYTES + 2 * (2 * (size_t)TileS<D>::BYTES + 2 * kRowsT * 4);
-  const size_t smem_q = 2 * (size_t)TileS<D>::BYTES + 2 * (2 * (size_t)TileS<D>::BYTES);
   auto kkv = bwd_dkdv_kernel<D>;
-  auto kq = bwd_dq_kernel<D>;
-  if (cudaFuncSetAttribute(kkv, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_kv) != cudaSuccess ||
-      cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_q) != cudaSuccess)
+  if (cudaFuncSetAttribute(kkv, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_kv) != cudaSuccess)
     return BSATTN_ERR_CUDA;
   dim3 grid(g.N, g.Hh, g.B);
   kkv<<<grid, kThreadsB, smem_kv, st>>>(g, q, k, v, d_o, lse, w.delta, w.idxT, w.cntT, c_log2, scale, dk, dv);
-  kq<<<grid, kThreadsB, smem_q, st>>>(g, q, k, v, d_o, lse, w.delta, idx, cnt, p->kmax, c_log2, scale, dq,
-                                      p->d_err);
-  return cudaGetLastError() == cudaSuccess ? BSATTN_OK : BSATTN_ERR_CUDA;
+  if (cudaGetLastError() != cudaSuccess) return BSATTN_ERR_CUDA;
+  // dQ on the tensor cores (csrc/bwd_tc.cu).
+  return launch_backward_dq_tc(p, q, k, v, d_o, lse, w.delta, idx, cnt, dq, st);
 }
 
 }  // namespace
