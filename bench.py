@@ -596,7 +596,7 @@ def backward_timing(bsattn, plan, wl, q, k, v, idx, cnt, flush, stream, pk):
         raise SystemExit("device error word set in the backward")
     tf = 2.5 * kept_pairs_from_counts(cnt) * pair_flops(wl.head_dim) / (ms * 1e-3) / 1e12
     return {"ms": ms, "tflops": tf, "frac": tf / pk["bf16_tflops"],
-            "note": "attn_backward (dQ, dK, dV; bf16 mma.sync kernels), five 64x64xD products per kept pair"}
+            "note": "attn_backward (dQ, dK, dV on tcgen05), five 64x64xD products per kept pair"}
 
 
 def memory_kernel_rates(wl, plan, comp, pk):

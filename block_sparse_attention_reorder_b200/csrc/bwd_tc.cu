@@ -459,6 +459,462 @@ bsattn_status run_dq(const bsattn_plan* p, const void* q, const void* k, const v
   return cudaGetLastError() == cudaSuccess ? BSATTN_OK : BSATTN_ERR_CUDA;
 }
 
+// ---------------------------------------------------------------- dK, dV
+// Two adjacent key tiles j0, j1 stacked into one 128-row block walk the union
+// of their transposed lists (the query tiles that keep them), on the same
+// pattern with rows and columns exchanged:
+//   S^T = K Q_i^T and dP^T = V dO_i^T (SS, N = 64) into TMEM double buffers;
+//   P^T = 2^(S^T scale log2(e) - lse_i log2(e)) per query column,
+//   dS^T = P^T (dP^T - Delta_i), both written back as bf16 over the first 16
+//   columns of each key half of their buffers by eight warps;
+//   dV += P^T dO_i and dK += dS^T Q_i (A from TMEM, dO_i and Q_i as MN-major
+//   shared-memory operands), accumulated in TMEM; dK is scaled at the end.
+// Per step the TMA warp brings Q_i, dO_i and the 64 lse and Delta values of
+// query tile i into a three-stage ring.
+struct KvParams {
+  Geom g;
+  const int32_t* idxT;  // [B, Hh, N, N] query tiles keeping each key tile, ascending
+  const int32_t* cntT;  // [B, Hh, N]
+  const float* lse;
+  const float* delta;
+  __nv_bfloat16* dk;
+  __nv_bfloat16* dv;
+  float scale;
+  float scale_log2;
+  int* err;
+  int umax;
+  int bm_words;
+  int pair_axis;
+  int pdim[3];
+};
+
+template <int D>
+struct KvCfg {
+  static constexpr int QRB = D * 2;
+  static constexpr int QBLK = QRB / 128;
+  static constexpr int NKS = QRB / 32;
+  static constexpr int BLK_BYTES = 128 * QRB;   // K or V block (two key tiles)
+  static constexpr int T_BYTES = 64 * QRB;      // Q or dO tile
+  static constexpr int STAGE = 2 * T_BYTES + 1024;  // Q, dO, lse (256 B), Delta (256 B), pad
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = OFF_K + BLK_BYTES;
+  static constexpr int OFF_RING = OFF_V + BLK_BYTES;
+  static constexpr int OFF_BAR = OFF_RING + kStages * STAGE;
+  static constexpr int NBAR = 1 + 2 * kStages + 5;  // kv, full[S], empty[S], sfull[2], pfull[2], final
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int OFF_COL = OFF_MISC + 16;
+  static constexpr int OFF_SCAN = OFF_COL + 256;
+  static constexpr int OFF_DYN = OFF_SCAN + 64;
+  static constexpr int O_PITCH = D * 2 + 16;
+  static_assert(STAGE % 1024 == 0, "stage alignment");
+  static_assert(2 * 128 * O_PITCH <= OFF_BAR - OFF_RING, "epilogue staging fits in the ring");
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
+                   const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, KvParams P) {
+  using C = KvCfg<D>;
+  constexpr uint32_t kColST = 0, kColDPT = 128, kColDV = 256, kColDK = 256 + D;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sb = tc::smem_addr(smem);
+  const uint32_t bar_kv = sb + C::OFF_BAR;
+  auto bar_full = [&](int s) { return sb + C::OFF_BAR + 8u * (1 + s); };
+  auto bar_empty = [&](int s) { return sb + C::OFF_BAR + 8u * (1 + kStages + s); };
+  auto bar_sfull = [&](int b) { return sb + C::OFF_BAR + 8u * (1 + 2 * kStages + b); };
+  auto bar_pfull = [&](int b) { return sb + C::OFF_BAR + 8u * (3 + 2 * kStages + b); };
+  const uint32_t bar_final = sb + C::OFF_BAR + 8u * (5 + 2 * kStages);
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
+  volatile int* never = reinterpret_cast<volatile int*>(misc + 3);
+  uint32_t* colc = reinterpret_cast<uint32_t*>(smem + C::OFF_COL);
+  int* scan = reinterpret_cast<int*>(smem + C::OFF_SCAN);
+  uint32_t* bmA = reinterpret_cast<uint32_t*>(smem + C::OFF_DYN);
+  uint32_t* bmB = bmA + P.bm_words;
+  uint32_t* ulist = bmB + P.bm_words;
+  uint32_t* uext = ulist + P.umax;
+
+  const Geom& g = P.g;
+  int j0, j1;
+  {
+    const int nd[3] = {g.nT, g.nH, g.nW};
+    int c[3], rem = blockIdx.x;
+    c[2] = rem % P.pdim[2];
+    rem /= P.pdim[2];
+    c[1] = rem % P.pdim[1];
+    c[0] = rem / P.pdim[1];
+    c[P.pair_axis] *= 2;
+    j0 = (c[0] * g.nH + c[1]) * g.nW + c[2];
+    c[P.pair_axis] += 1;
+    j1 = c[P.pair_axis] < nd[P.pair_axis] ? (c[0] * g.nH + c[1]) * g.nW + c[2] : -1;
+  }
+  const int head = blockIdx.y, b = blockIdx.z;
+  const size_t bh = (size_t)b * g.Hh + head;
+  const bool has1 = j1 >= 0;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  auto tile_row = [&](int j) -> int { return (int)((bh * g.N + j) * 64); };
+  // Bit r set when in-tile row r of tile j is a real token.
+  auto real_rows = [&](int j) -> uint64_t {
+    const int bt = j / (g.nH * g.nW), bhh = (j / g.nW) % g.nH, bw = j % g.nW;
+    const int vt = g.T - bt * g.tt, vh = g.H - bhh * g.th, vw = g.W - bw * g.tw;
+    if (vt >= g.tt && vh >= g.th && vw >= g.tw) return ~0ull;
+    uint64_t m = 0;
+    for (int r = 0; r < 64; ++r) {
+      const uint32_t cc = colc[r];
+      if ((int)(cc & 0xffu) < vt && (int)((cc >> 8) & 0xffu) < vh && (int)((cc >> 16) & 0xffu) < vw) m |= 1ull << r;
+    }
+    return m;
+  };
+
+  // ------------------------------------------------------------ setup
+  if (tid == 0) {
+    tc::mbar_init(bar_kv, 1);
+    for (int s = 0; s < kStages; ++s) {
+      tc::mbar_init(bar_full(s), 1);
+      tc::mbar_init(bar_empty(s), 1);
+    }
+    for (int x = 0; x < 2; ++x) {
+      tc::mbar_init(bar_sfull(x), 1);
+      tc::mbar_init(bar_pfull(x), kSoftmaxThreads);
+    }
+    tc::mbar_init(bar_final, 1);
+    misc[1] = 0;
+    misc[3] = 0;
+    tc::mbar_fence_init();
+  }
+  if (warp == 9) {
+    tc::tmem_alloc(sb + C::OFF_MISC, kTmemCols);
+    tc::tmem_relinquish();
+  }
+  if (tid < 64) {
+    const int dt = tid / (g.th * g.tw), dh = (tid / g.tw) % g.th, dw = tid % g.tw;
+    colc[tid] = (uint32_t)dt | ((uint32_t)dh << 8) | ((uint32_t)dw << 16);
+  }
+  for (int w = tid; w < 2 * P.bm_words; w += kThreads) bmA[w] = 0u;
+  if (!has1) {  // rows 64..127 have no key tile: zero their K and V
+    for (int x = tid; x < C::QBLK * 64 * 128 / 16; x += kThreads) {
+      const int cb = x / (64 * 128 / 16), off = x % (64 * 128 / 16);
+      reinterpret_cast<uint4*>(smem + C::OFF_K + cb * 128 * 128 + 64 * 128)[off] = make_uint4(0, 0, 0, 0);
+      reinterpret_cast<uint4*>(smem + C::OFF_V + cb * 128 * 128 + 64 * 128)[off] = make_uint4(0, 0, 0, 0);
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  __syncthreads();
+
+  // Union of the two transposed lists, ascending: query tile in bits 0-29,
+  // bit 30 (31) when it keeps j0 (j1); uext holds the query tile's real
+  // extent and bit 31 when it has padded rows.
+  {
+    const int nA = min(max(P.cntT[bh * g.N + j0], 0), g.N);
+    const int nB = has1 ? min(max(P.cntT[bh * g.N + j1], 0), g.N) : 0;
+    const int32_t* lA = P.idxT + (bh * g.N + j0) * (size_t)g.N;
+    const int32_t* lB = has1 ? P.idxT + (bh * g.N + j1) * (size_t)g.N : lA;
+    for (int e = tid; e < nA + nB; e += kThreads) {
+      const int i = e < nA ? __ldg(lA + e) : __ldg(lB + (e - nA));
+      if (i < 0 || i >= g.N) continue;  // the transposed lists are built in range
+      atomicOr(e < nA ? &bmA[i >> 5] : &bmB[i >> 5], 1u << (i & 31));
+    }
+  }
+  __syncthreads();
+  {
+    const int wpt = (P.bm_words + kThreads - 1) / kThreads;
+    const int w0 = min(tid * wpt, P.bm_words), w1 = min(w0 + wpt, P.bm_words);
+    int mine = 0;
+    for (int w = w0; w < w1; ++w) mine += __popc(bmA[w] | bmB[w]);
+    int x = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) scan[warp] = x;
+    __syncthreads();
+    int off = 0, tot = 0;
+#pragma unroll
+    for (int i = 0; i < kThreads / 32; ++i) {
+      off += i < warp ? scan[i] : 0;
+      tot += scan[i];
+    }
+    int pos = off + x - mine;
+    for (int w = w0; w < w1; ++w) {
+      const uint32_t a = bmA[w], bb = bmB[w];
+      uint32_t bits = a | bb;
+      while (bits) {
+        const int bit = __ffs(bits) - 1;
+        bits &= bits - 1;
+        const int i = w * 32 + bit;
+        if (pos < P.umax) {
+          ulist[pos] = (uint32_t)i | (((a >> bit) & 1u) << 30) | (((bb >> bit) & 1u) << 31);
+          const int bt = i / (g.nH * g.nW), bhh = (i / g.nW) % g.nH, bw = i % g.nW;
+          const int vt = min(g.T - bt * g.tt, 255), vh = min(g.H - bhh * g.th, 255), vw = min(g.W - bw * g.tw, 255);
+          const bool edge = vt < g.tt || vh < g.th || vw < g.tw;
+          uext[pos] = (uint32_t)vt | ((uint32_t)vh << 8) | ((uint32_t)vw << 16) | (edge ? 1u << 31 : 0u);
+        }
+        ++pos;
+      }
+    }
+    if (tid == 0) misc[2] = (uint32_t)min(tot, P.umax);
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = misc[0];
+  const int L = (int)misc[2];
+
+  // ------------------------------------------------------------ roles
+  if (warp == 8) {
+    if (lane == 0 && L > 0) {
+      tc::tma_prefetch_desc(&tmQ);
+      tc::tma_prefetch_desc(&tmDO);
+      tc::tma_prefetch_desc(&tmK);
+      tc::tma_prefetch_desc(&tmV);
+      tc::mbar_arrive_expect_tx(bar_kv, (has1 ? 2 : 1) * 2 * 64 * C::QRB);
+      for (int x = 0; x < (has1 ? 2 : 1); ++x) {
+        const int tile = x ? j1 : j0;
+#pragma unroll
+        for (int cb = 0; cb < C::QBLK; ++cb) {
+          const uint32_t d = cb * 128 * 128 + x * 64 * 128;
+          tc::tma_load_2d(sb + C::OFF_K + d, &tmK, bar_kv, cb * 64, tile_row(tile));
+          tc::tma_load_2d(sb + C::OFF_V + d, &tmV, bar_kv, cb * 64, tile_row(tile));
+        }
+      }
+      int last[kStages];
+#pragma unroll
+      for (int s = 0; s < kStages; ++s) last[s] = -1;
+      for (int m = 0; m < L; ++m) {
+        const int s = m % kStages;
+        if (m >= kStages && !tc::mbar_wait(bar_empty(s), ((m / kStages) - 1) & 1, abort_flag, kWaitLimit)) {
+          *abort_flag = 1;
+          atomicOr(P.err, BSATTN_DEVERR_TIMEOUT);
+          break;
+        }
+        const int qt = (int)(ulist[m] & 0x3FFFFFFFu);
+        const uint32_t st = sb + C::OFF_RING + s * C::STAGE;
+        tc::mbar_arrive_expect_tx(bar_full(s), 2 * C::T_BYTES + 512);
+#pragma unroll
+        for (int cb = 0; cb < C::QBLK; ++cb) {
+          tc::tma_load_2d(st + cb * 64 * 128, &tmQ, bar_full(s), cb * 64, tile_row(qt));
+          tc::tma_load_2d(st + C::T_BYTES + cb * 64 * 128, &tmDO, bar_full(s), cb * 64, tile_row(qt));
+        }
+        tc::bulk_load(st + 2 * C::T_BYTES, P.lse + tile_row(qt), 256, bar_full(s));
+        tc::bulk_load(st + 2 * C::T_BYTES + 256, P.delta + tile_row(qt), 256, bar_full(s));
+        last[s] = m;
+      }
+      if (*abort_flag) {
+        tc::mbar_wait(bar_kv, 0, never, kWaitLimit);
+        for (int s = 0; s < kStages; ++s)
+          if (last[s] >= 0) tc::mbar_wait(bar_full(s), (last[s] / kStages) & 1, never, kWaitLimit);
+      }
+    }
+  } else if (warp == 9) {
+    if (lane == 0 && L > 0) {
+      constexpr uint32_t idS = tc::instr_desc(1, 1, 0, 0, 64, 128);  // K-major A and B, N = 64
+      constexpr uint32_t idG = tc::instr_desc(1, 1, 0, 1, D, 128);   // B MN-major, N = D
+      bool ok = tc::mbar_wait(bar_kv, 0, abort_flag, kWaitLimit);
+      auto issue_sdp = [&](int m) -> bool {
+        const int s = m % kStages;
+        if (!tc::mbar_wait(bar_full(s), (m / kStages) & 1, abort_flag, kWaitLimit)) return false;
+        tc::fence_after_sync();
+        const uint32_t st = sb + C::OFF_RING + s * C::STAGE;
+        const uint32_t dS = tmem + kColST + (m & 1) * 64, dP = tmem + kColDPT + (m & 1) * 64;
+#pragma unroll
+        for (int kk = 0; kk < C::NKS; ++kk) {
+          const int cb = kk / 4, within = kk % 4;
+          const uint32_t aoff = cb * 128 * 128 + within * 32, boff = cb * 64 * 128 + within * 32;
+          tc::mma_ss_f16(dS, tc::smem_desc(sb + C::OFF_K + aoff, 16, 1024, tc::kLayoutSW128),
+                         tc::smem_desc(st + boff, 16, 1024, tc::kLayoutSW128), idS, kk > 0 ? 1u : 0u);
+          tc::mma_ss_f16(dP, tc::smem_desc(sb + C::OFF_V + aoff, 16, 1024, tc::kLayoutSW128),
+                         tc::smem_desc(st + C::T_BYTES + boff, 16, 1024, tc::kLayoutSW128), idS, kk > 0 ? 1u : 0u);
+        }
+        tc::mma_commit(bar_sfull(m & 1));
+        return true;
+      };
+      if (ok) ok = issue_sdp(0);
+      if (ok && L > 1) ok = issue_sdp(1);
+      for (int n = 0; ok && n < L; ++n) {
+        const int s = n % kStages;
+        if (!tc::mbar_wait(bar_pfull(n & 1), (n >> 1) & 1, abort_flag, kWaitLimit)) {
+          ok = false;
+          break;
+        }
+        tc::fence_after_sync();
+        const uint32_t st = sb + C::OFF_RING + s * C::STAGE;
+        // P^T and dS^T (bf16): queries 0-31 in columns 0-15, 32-63 in 32-47.
+        const uint32_t pA = tmem + kColST + (n & 1) * 64, dsA = tmem + kColDPT + (n & 1) * 64;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {  // 16 queries per MMA: 2048 bytes of the dO / Q tile
+          const uint32_t acol = kk < 2 ? kk * 8 : 32 + (kk - 2) * 8;
+          const uint32_t acc = (n > 0 || kk > 0) ? 1u : 0u;
+          tc::mma_ts_f16(tmem + kColDV, pA + acol,
+                         tc::smem_desc(st + C::T_BYTES + kk * 2048, 8192, 1024, tc::kLayoutSW128), idG, acc);
+          tc::mma_ts_f16(tmem + kColDK, dsA + acol, tc::smem_desc(st + kk * 2048, 8192, 1024, tc::kLayoutSW128),
+                         idG, acc);
+        }
+        tc::mma_commit(bar_empty(s));
+        if (n + 2 < L && !issue_sdp(n + 2)) {
+          ok = false;
+          break;
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        atomicOr(P.err, BSATTN_DEVERR_TIMEOUT);
+      }
+      tc::mma_commit(bar_final);
+      tc::mbar_wait(bar_final, 0, never, kWaitLimit);
+    }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------- P^T, dS^T
+    const int quad = warp & 3, part = warp >> 2;  // lane quadrant, query half
+    const int r = quad * 32 + lane;                // key row of the block
+    const int half = r >> 6;                       // 0: tile j0, 1: tile j1
+    const bool row_exists = half == 0 || has1;
+    const bool key_real = row_exists && ((real_rows(half ? j1 : j0) >> (r & 63)) & 1);
+    const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
+    const float c = P.scale_log2;
+    bool ok = true;
+    for (int n = 0; n < L; ++n) {
+      const uint32_t e = ulist[n];
+      const bool keep = row_exists && ((e >> (30 + half)) & 1u) != 0;  // uniform within the warp
+      if (!__all_sync(0xffffffffu, tc::mbar_wait(bar_sfull(n & 1), (n >> 1) & 1, abort_flag, kWaitLimit))) {
+        ok = false;
+        break;
+      }
+      tc::fence_after_sync();
+      const uint32_t sbuf = tmem + lane_base + kColST + (n & 1) * 64 + 32 * part;
+      const uint32_t pbuf = tmem + lane_base + kColDPT + (n & 1) * 64 + 32 * part;
+      // lse and Delta of this step's query tile came with its TMA copies:
+      // observe their barrier before reading them.
+      if (!__all_sync(0xffffffffu, tc::mbar_wait(bar_full(n % kStages), (n / kStages) & 1, abort_flag, kWaitLimit))) {
+        ok = false;
+        break;
+      }
+      uint32_t pw[16], dw[16];
+      if (keep) {
+        const float* ld = reinterpret_cast<const float*>(smem + C::OFF_RING + (n % kStages) * C::STAGE + 2 * C::T_BYTES);
+        const uint32_t ext = uext[n];
+        const bool edge = (ext >> 31) != 0;
+        const int vt = (int)(ext & 0xffu), vh = (int)((ext >> 8) & 0xffu), vw = (int)((ext >> 16) & 0xffu);
+        uint32_t sr[32], pr[32];
+        tc::tmem_ld32_wait(sbuf, sr);
+        tc::tmem_ld32_wait(pbuf, pr);
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+          float pp[2], d2[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int qc = 32 * part + 2 * q + u;  // query column
+            bool real = key_real;
+            if (edge) {
+              const uint32_t cc = colc[qc];
+              real = real && (int)(cc & 0xffu) < vt && (int)((cc >> 8) & 0xffu) < vh && (int)((cc >> 16) & 0xffu) < vw;
+            }
+            const float p = real ? tc::ex2(__uint_as_float(sr[2 * q + u]) * c - ld[qc] * 1.4426950408889634f) : 0.f;
+            pp[u] = p;
+            d2[u] = p * (__uint_as_float(pr[2 * q + u]) - ld[64 + qc]);
+          }
+          __nv_bfloat162 hp = __floats2bfloat162_rn(pp[0], pp[1]), hd = __floats2bfloat162_rn(d2[0], d2[1]);
+          pw[q] = *reinterpret_cast<uint32_t*>(&hp);
+          dw[q] = *reinterpret_cast<uint32_t*>(&hd);
+        }
+      } else {
+#pragma unroll
+        for (int q = 0; q < 16; ++q) pw[q] = dw[q] = 0u;
+      }
+      tc::tmem_st16(sbuf, pw);  // P^T over the first 16 columns of this half of S^T
+      tc::tmem_st16(pbuf, dw);  // dS^T over the first 16 columns of this half of dP^T
+      tc::tmem_wait_st();
+      tc::fence_before_sync();
+      tc::mbar_arrive(bar_pfull(n & 1));
+    }
+    if (!ok) {
+      *abort_flag = 1;
+      atomicOr(P.err, BSATTN_DEVERR_TIMEOUT);
+    }
+    // ---------------------------------------------------------- epilogue
+    if (ok && L > 0) {
+      if (!__all_sync(0xffffffffu, tc::mbar_wait(bar_final, 0, abort_flag, kWaitLimit))) {
+        *abort_flag = 1;
+        atomicOr(P.err, BSATTN_DEVERR_TIMEOUT);
+        ok = false;
+      }
+      tc::fence_after_sync();
+    }
+    // dK (scaled) and dV rows staged in the ring: dK at rows 0-127, dV at 128-255.
+    constexpr int OC = D / 2;
+#pragma unroll
+    for (int which = 0; which < 2; ++which) {
+      uint8_t* stage = smem + C::OFF_RING + (which * 128 + r) * C::O_PITCH;
+      const float mul = which == 0 ? P.scale : 1.f;
+      const uint32_t base = which == 0 ? kColDK : kColDV;
+#pragma unroll
+      for (int col = part * OC; col < part * OC + OC; col += 32) {
+        uint32_t o[32];
+        if (ok && L > 0) {
+          tc::tmem_ld32_wait(tmem + lane_base + base + col, o);
+        } else {
+#pragma unroll
+          for (int q = 0; q < 32; ++q) o[q] = 0u;
+        }
+        uint32_t w[16];
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+          __nv_bfloat162 hv = __floats2bfloat162_rn(__uint_as_float(o[2 * q]) * mul, __uint_as_float(o[2 * q + 1]) * mul);
+          w[q] = *reinterpret_cast<uint32_t*>(&hv);
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          reinterpret_cast<uint4*>(stage + col * 2)[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+      }
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(kSoftmaxThreads) : "memory");
+    constexpr int CPR = D / 8;
+    const int rows = has1 ? 128 : 64;
+    for (int e2 = tid; e2 < 2 * rows * CPR; e2 += kSoftmaxThreads) {
+      const int which = e2 / (rows * CPR), rem = e2 % (rows * CPR);
+      const int rr = rem / CPR, cc = rem % CPR;
+      const uint4 val = *reinterpret_cast<const uint4*>(smem + C::OFF_RING + (which * 128 + rr) * C::O_PITCH + cc * 16);
+      __nv_bfloat16* dst = which == 0 ? P.dk : P.dv;
+      uint4* og = reinterpret_cast<uint4*>(dst + (size_t)tile_row(rr >> 6 ? j1 : j0) * D);
+      og[(rr & 63) * CPR + cc] = val;
+    }
+  }
+
+  // ------------------------------------------------------------ teardown
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 9) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+template <int D>
+bsattn_status run_dkdv(const bsattn_plan* p, const void* q, const void* k, const void* v, const void* d_o,
+                       KvParams prm, cudaStream_t st) {
+  using C = KvCfg<D>;
+  const uint64_t rows = (uint64_t)p->desc.B * p->desc.heads * p->N * 64;
+  if (rows + 128 >= (1ull << 31)) return BSATTN_ERR_UNSUPPORTED;
+  CUtensorMap mq, mdo, mk, mv;
+  const auto bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  if (!bsattn_make_map_2d(&mq, q, bf, 2, D, rows, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !bsattn_make_map_2d(&mdo, d_o, bf, 2, D, rows, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !bsattn_make_map_2d(&mk, k, bf, 2, D, rows, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !bsattn_make_map_2d(&mv, v, bf, 2, D, rows, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+    return BSATTN_ERR_CUDA;
+  const size_t smem = 1024 + C::OFF_DYN + (size_t)prm.bm_words * 8 + (size_t)prm.umax * 8;
+  if (smem > 227 * 1024) return BSATTN_ERR_UNSUPPORTED;
+  auto kern = bwd_dkdv_tc_kernel<D>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return BSATTN_ERR_CUDA;
+  dim3 grid(prm.pdim[0] * prm.pdim[1] * prm.pdim[2], p->desc.heads, p->desc.B);
+  kern<<<grid, kThreads, smem, st>>>(mq, mdo, mk, mv, prm);
+  return cudaGetLastError() == cudaSuccess ? BSATTN_OK : BSATTN_ERR_CUDA;
+}
+
 }  // namespace
 
 bsattn_status launch_backward_dq_tc(const bsattn_plan* p, const void* q, const void* k, const void* v,
@@ -481,4 +937,27 @@ bsattn_status launch_backward_dq_tc(const bsattn_plan* p, const void* q, const v
   const int nd[3] = {p->nT, p->nH, p->nW};
   for (int a = 0; a < 3; ++a) prm.pdim[a] = a == prm.pair_axis ? (nd[a] + 1) / 2 : nd[a];
   return p->desc.head_dim == 128 ? run_dq<128>(p, q, k, v, d_o, prm, st) : run_dq<64>(p, q, k, v, d_o, prm, st);
+}
+
+bsattn_status launch_backward_dkdv_tc(const bsattn_plan* p, const void* q, const void* k, const void* v,
+                                      const void* d_o, const float* lse, const float* delta, const int32_t* idxT,
+                                      const int32_t* cntT, void* dk, void* dv, cudaStream_t st) {
+  KvParams prm;
+  prm.g = make_geom(p);
+  prm.idxT = idxT;
+  prm.cntT = cntT;
+  prm.lse = lse;
+  prm.delta = delta;
+  prm.dk = (__nv_bfloat16*)dk;
+  prm.dv = (__nv_bfloat16*)dv;
+  prm.scale = p->scale;
+  prm.scale_log2 = p->scale * 1.4426950408889634f;
+  prm.err = p->d_err;
+  prm.umax = p->N;  // the union of two transposed lists holds at most N query tiles
+  prm.bm_words = (p->N + 31) / 32;
+  prm.pair_axis = (p->rule.kind == BSATTN_RULE_WINDOW && p->rule.win_w == 0) ? 0 : 2;
+  const int nd[3] = {p->nT, p->nH, p->nW};
+  for (int a = 0; a < 3; ++a) prm.pdim[a] = a == prm.pair_axis ? (nd[a] + 1) / 2 : nd[a];
+  return p->desc.head_dim == 128 ? run_dkdv<128>(p, q, k, v, d_o, prm, st)
+                                 : run_dkdv<64>(p, q, k, v, d_o, prm, st);
 }

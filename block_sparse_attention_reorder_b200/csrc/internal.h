@@ -130,6 +130,11 @@ bsattn_status launch_backward_dq_tc(const bsattn_plan* p, const void* q, const v
                                     const void* d_o, const float* lse, const float* delta, const int32_t* idx,
                                     const int32_t* cnt, void* dq, cudaStream_t st);
 
+// dK and dV of the backward on the tensor cores, over the transposed lists.
+bsattn_status launch_backward_dkdv_tc(const bsattn_plan* p, const void* q, const void* k, const void* v,
+                                      const void* d_o, const float* lse, const float* delta, const int32_t* idxT,
+                                      const int32_t* cntT, void* dk, void* dv, cudaStream_t st);
+
 // 2-D tiled tensor map over `rows` rows of `inner` elements of `esz` bytes.
 bool bsattn_make_map_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int esz, int inner,
                         uint64_t rows, int box_inner, int box_rows, CUtensorMapSwizzle sw);
