@@ -151,6 +151,60 @@ def attention_backward_full(q_nat, k_nat, v_nat, do_nat, lists, T, H, W, tile=(4
     return dq, dk, dv
 
 
+def attention_backward_tiles(q_nat, k_nat, v_nat, do_nat, lists, T, H, W, tile=(4, 4, 4), scale=None,
+                             b=0, h=0, qtiles=(), ktiles=()):
+    """Gradients for selected tiles of one (batch, head), without the [L, L]
+    mask (large grids): dQ of the valid tokens of each query tile in
+    `qtiles`, and dK, dV of the valid tokens of each key tile in `ktiles`.
+
+    dQ_i needs only query tile i and its kept key tiles. dK_j and dV_j sum
+    over the query tiles that keep j; each such query row's softmax is taken
+    over all of its own kept keys (as the full layer does). Returns
+    ({i: (token ids, dq)}, {j: (token ids, dk, dv)}) in fp64.
+    """
+    B, L, Hh, D = q_nat.shape
+    nb = tiling.n_blocks(T, H, W, tile)
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    tid, _ = tiling.token_tile_and_row(T, H, W, tile)
+    members = [np.nonzero(tid == t)[0] for t in range(nb)]
+    rows = lists[(b * Hh + h) * nb:(b * Hh + h + 1) * nb]
+    q, k, v, do = (x[b, :, h].astype(np.float64) for x in (q_nat, k_nat, v_nat, do_nat))
+
+    def row_softmax(i):
+        """P over query tile i's kept keys, the key token ids, and Delta."""
+        qi = members[i]
+        kj = np.concatenate([members[j] for j in rows[i]]) if len(rows[i]) else np.zeros(0, int)
+        s = scale * (q[qi] @ k[kj].T)
+        m = s.max(axis=1, keepdims=True) if kj.size else np.zeros((qi.size, 1))
+        e = np.exp(s - m)
+        p = e / e.sum(axis=1, keepdims=True) if kj.size else e
+        o = p @ v[kj]
+        delta = (do[qi] * o).sum(axis=1)
+        return qi, kj, p, delta
+
+    dq_out = {}
+    for i in qtiles:
+        qi, kj, p, delta = row_softmax(i)
+        ds = p * (do[qi] @ v[kj].T - delta[:, None])
+        dq_out[i] = (qi, scale * (ds @ k[kj]))
+    dkv_out = {}
+    for j in ktiles:
+        kj_tokens = members[j]
+        dk = np.zeros((kj_tokens.size, D))
+        dv = np.zeros((kj_tokens.size, D))
+        for i in range(nb):
+            if j not in set(int(x) for x in rows[i]):
+                continue
+            qi, kj, p, delta = row_softmax(i)
+            cols = np.isin(kj, kj_tokens)  # this key tile's columns, in token order
+            pj = p[:, cols]
+            dsj = pj * (do[qi] @ v[kj[cols]].T - delta[:, None])
+            dv += pj.T @ do[qi]
+            dk += scale * (dsj.T @ q[qi])
+        dkv_out[j] = (kj_tokens, dk, dv)
+    return dq_out, dkv_out
+
+
 def fp8_qk(q_nat, k_nat, T, H, W, tile=(4, 4, 4)):
     """Per-tile e4m3 quantise-dequantise of Q and K.
 

@@ -73,3 +73,52 @@ def test_backward_rejects_unsupported_plans(bs):
     with pytest.raises(bs.BsattnError) as e:
         bs.attn_backward(plan, x, x, x, x, x, lse, idx, cnt, x, x, x, plan.workspace("backward"))
     assert e.value.code == 2
+
+
+@pytest.mark.parametrize("name", ["wan1.3b", "wan14b"])
+def test_backward_full_size_sampled(bs, name):
+    """Full-size layers: dQ of sampled query tiles and dK, dV of sampled key
+    tiles (edge tiles included) against the oracle computed tile by tile."""
+    from block_sparse_attention_reorder_b200.datagen import WORKLOADS
+    wl = WORKLOADS[name]
+    plan = bs.Plan.for_workload(wl)
+    q, k, v = make_qkv(wl, "cuda")
+    g = torch.Generator(device="cuda").manual_seed(200)
+    d_o = torch.randn(q.shape, generator=g, device="cuda").to(torch.bfloat16)
+    si, sc = plan.list_shapes()
+    idx = torch.empty(si, dtype=torch.int32, device="cuda")
+    cnt = torch.empty(sc, dtype=torch.int32, device="cuda")
+    bs.attn_select(plan, q, k, idx, cnt, plan.workspace("select"))
+    ts = plan.tiled_shape()
+    t = [torch.empty(ts, dtype=torch.bfloat16, device="cuda") for _ in range(4)]
+    for x, y in zip((q, k, v, d_o), t):
+        bs.attn_reorder(plan, x, y)
+    ot = torch.empty(ts, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((wl.B, wl.heads, plan.N, plan.V), dtype=torch.float32, device="cuda")
+    bs.attn_forward(plan, t[0], t[1], t[2], idx, cnt, ot, lse)
+    grads = [torch.empty(ts, dtype=torch.bfloat16, device="cuda") for _ in range(3)]
+    bs.attn_backward(plan, t[0], t[1], t[2], ot, t[3], lse, idx, cnt, *grads, plan.workspace("backward"))
+    assert bs.attn_check_device_status(plan) == 0
+    h = 3
+    nat = []
+    for gt in grads:
+        back = torch.empty_like(q)
+        bs.attn_unreorder(plan, gt, back)
+        nat.append(to64(back[:, :, h:h + 1]))
+    del grads, t
+    idx_h = idx[0, h].cpu().numpy()
+    cnt_h = cnt[0, h].cpu().numpy()
+    qn, kn, vn, don = (to64(x[:, :, h:h + 1]) for x in (q, k, v, d_o))
+    lists_h = [idx_h[i, :cnt_h[i]].astype(np.int64) for i in range(plan.N)]
+    qt_s, kt_s = [0, plan.N // 3, plan.N - 1], [1, plan.N // 2, plan.N - 1]
+    dq_t, dkv_t = attention.attention_backward_tiles(qn, kn, vn, don, lists_h, wl.T, wl.H, wl.W, wl.tile,
+                                                     h=0, qtiles=qt_s, ktiles=kt_s)
+    got_q = np.concatenate([nat[0][0, tok, 0] for tok, _ in dq_t.values()])
+    ref_q = np.concatenate([gq for _, gq in dq_t.values()])
+    _grad_close(got_q, ref_q, "dq")
+    got_k = np.concatenate([nat[1][0, tok, 0] for tok, _, _ in dkv_t.values()])
+    ref_k = np.concatenate([gk for _, gk, _ in dkv_t.values()])
+    _grad_close(got_k, ref_k, "dk")
+    got_v = np.concatenate([nat[2][0, tok, 0] for tok, _, _ in dkv_t.values()])
+    ref_v = np.concatenate([gv for _, _, gv in dkv_t.values()])
+    _grad_close(got_v, ref_v, "dv")

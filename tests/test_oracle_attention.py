@@ -177,3 +177,22 @@ def test_backward_all_kept_equals_torch_autograd():
         np.testing.assert_allclose(dq[0, :, h], tq.grad.numpy(), rtol=1e-10, atol=1e-12)
         np.testing.assert_allclose(dk[0, :, h], tk.grad.numpy(), rtol=1e-10, atol=1e-12)
         np.testing.assert_allclose(dv[0, :, h], tv.grad.numpy(), rtol=1e-10, atol=1e-12)
+
+
+def test_backward_tiles_form_equals_full_mask_form():
+    """The per-tile backward (for large grids) equals the [L, L]-mask form."""
+    T, H, W = 5, 6, 9
+    rng = np.random.default_rng(11)
+    q, k, v, do = (rng.standard_normal((1, T * H * W, 2, 8)) for _ in range(4))
+    nb = tiling.n_blocks(T, H, W)
+    lists = [np.sort(rng.choice(nb, size=3, replace=False)) for _ in range(2 * nb)]
+    lists[5] = np.array([], dtype=np.int64)  # a query tile that keeps nothing
+    dq, dk, dv = attention.attention_backward_full(q, k, v, do, lists, T, H, W)
+    for h in range(2):
+        dq_t, dkv_t = attention.attention_backward_tiles(q, k, v, do, lists, T, H, W, h=h,
+                                                         qtiles=range(nb), ktiles=range(nb))
+        for i, (tok, g) in dq_t.items():
+            np.testing.assert_allclose(g, dq[0, tok, h], rtol=1e-12, atol=1e-13)
+        for j, (tok, gk, gv) in dkv_t.items():
+            np.testing.assert_allclose(gk, dk[0, tok, h], rtol=1e-12, atol=1e-13)
+            np.testing.assert_allclose(gv, dv[0, tok, h], rtol=1e-12, atol=1e-13)
