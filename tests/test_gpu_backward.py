@@ -122,3 +122,65 @@ def test_backward_full_size_sampled(bs, name):
     got_v = np.concatenate([nat[2][0, tok, 0] for tok, _, _ in dkv_t.values()])
     ref_v = np.concatenate([gv for _, _, gv in dkv_t.values()])
     _grad_close(got_v, ref_v, "dv")
+
+
+def _backward_vs_oracle(bs, wl, lists):
+    plan = bs.Plan.for_workload(wl)
+    q, k, v = make_qkv(wl, "cpu")
+    g = torch.Generator(device="cpu").manual_seed(300 + wl.seed)
+    d_o = torch.randn(q.shape, generator=g).to(torch.bfloat16)
+    qn, kn, vn, don = (to64(x) for x in (q, k, v, d_o))
+    idx, cnt = lists_to_device(lists, plan.kmax)
+    si, sc = plan.list_shapes()
+    idx, cnt = idx.view(si), cnt.view(sc)
+    ts = plan.tiled_shape()
+    t = []
+    for x in (q, k, v, d_o):
+        y = torch.empty(ts, dtype=torch.bfloat16, device="cuda")
+        bs.attn_reorder(plan, x.cuda(), y)
+        t.append(y)
+    ot = torch.empty(ts, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((wl.B, wl.heads, plan.N, plan.V), dtype=torch.float32, device="cuda")
+    bs.attn_forward(plan, t[0], t[1], t[2], idx, cnt, ot, lse)
+    grads = [torch.full(ts, float("nan"), dtype=torch.bfloat16, device="cuda") for _ in range(3)]
+    bs.attn_backward(plan, t[0], t[1], t[2], ot, t[3], lse, idx, cnt, *grads, plan.workspace("backward"))
+    assert bs.attn_check_device_status(plan) == 0
+    ref = attention.attention_backward_full(qn, kn, vn, don, lists, wl.T, wl.H, wl.W, wl.tile)
+    out = []
+    for name_, got, r in zip(("dq", "dk", "dv"), grads, ref):
+        nat = tiling.unreorder(to64(got), wl.T, wl.H, wl.W, wl.tile)
+        if np.abs(r).max() > 0:
+            _grad_close(nat, r, name_)
+        else:
+            assert np.all(nat == 0), name_
+        out.append(nat)
+    return plan, out
+
+
+def test_backward_single_tile_grid(bs):
+    from block_sparse_attention_reorder_b200.datagen import Workload
+    wl = Workload("one_tile", 1, 2, 128, 3, 2, 3, "topk", k=1, recipe="iid", seed=21)
+    _backward_vs_oracle(bs, wl, [np.array([0])] * 2)
+
+
+def test_backward_empty_lists_and_all_kept(bs):
+    """Query tiles that keep nothing get zero dQ and give nothing to dK, dV;
+    a key tile nobody keeps gets zero dK, dV."""
+    from block_sparse_attention_reorder_b200.datagen import Workload
+    wl = Workload("empty_rows", 1, 2, 128, 7, 10, 13, "topk", k=3, recipe="iid", seed=23)
+    plan = bs.Plan.for_workload(wl)
+    rng = np.random.default_rng(6)
+    lists = []
+    for r in range(2 * plan.N):
+        if r % 3 == 0:
+            lists.append(np.array([], dtype=np.int64))
+        else:
+            choice = rng.choice(plan.N - 1, size=3, replace=False)  # key tile N-1 is never kept
+            lists.append(np.sort(choice))
+    _, (dq, dk, dv) = _backward_vs_oracle(bs, wl, lists)
+    tid, _ = tiling.token_tile_and_row(wl.T, wl.H, wl.W)
+    last = tid == plan.N - 1
+    assert np.all(dk[0, last] == 0) and np.all(dv[0, last] == 0)
+    for h in range(2):
+        empty = [i for i in range(plan.N) if (h * plan.N + i) % 3 == 0]
+        assert np.all(dq[0, np.isin(tid, empty), h] == 0)
