@@ -555,10 +555,10 @@ def component_timing(bsattn, plan, wl, q, k, v, flush, stream, reps=20):
 
 def backward_timing(bsattn, plan, wl, q, k, v, idx, cnt, flush, stream, pk):
     """attn_backward on the layer's kept lists (tiled inputs, the forward's O
-    and lse, a seeded random dO): device time and TFLOP/s counting five
-    64x64xD products per kept pair (S, dP, dV, dK, dQ; the kernels recompute
-    S and dP once more). None where the backward does not apply."""
-    if wl.qk_fp8 or plan.V != 64:
+    and lse, a seeded random dO): device time and TFLOP/s counting five VxVxD
+    products per kept tile pair (S, dP, dV, dK, dQ; the kernels compute S and
+    dP once more). None for e4m3 Q/K, which the backward does not take."""
+    if wl.qk_fp8:
         return None
     ts = plan.tiled_shape()
     g = torch.Generator(device="cuda").manual_seed(7)
@@ -594,9 +594,9 @@ def backward_timing(bsattn, plan, wl, q, k, v, idx, cnt, flush, stream, pk):
     ms = total / reps
     if bsattn.attn_check_device_status(plan) != 0:
         raise SystemExit("device error word set in the backward")
-    tf = 2.5 * kept_pairs_from_counts(cnt) * pair_flops(wl.head_dim) / (ms * 1e-3) / 1e12
+    tf = 2.5 * kept_pairs_from_counts(cnt) * pair_flops(wl.head_dim, plan.V) / (ms * 1e-3) / 1e12
     return {"ms": ms, "tflops": tf, "frac": tf / pk["bf16_tflops"],
-            "note": "attn_backward (dQ, dK, dV on tcgen05), five 64x64xD products per kept pair"}
+            "note": "attn_backward (dQ, dK, dV on tcgen05), five VxVxD products per kept tile pair"}
 
 
 def memory_kernel_rates(wl, plan, comp, pk):

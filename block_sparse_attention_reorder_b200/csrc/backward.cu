@@ -13,13 +13,12 @@
 // dQ per pair of query tiles over the kept lists. P and dS are rounded to
 // bf16 for the products, as the forward rounds P.
 //
-// Tiles of 64 tokens (tiled layout [B, Hh, N, 64, D], D in {64, 128}); padded
-// key and query slots are masked from their tile's real extent.
+// Tiled layout [B, Hh, N, V, D] (D in {64, 128}); the kernels work on 64-row
+// chunks of the tiles as the forward does; padded key and query slots are
+// masked from their chunk's real extent.
 #include "internal.h"
 
 namespace {
-
-constexpr int kRowsT = 64;  // tile rows
 
 // Delta = rowsum(dO * O) per query row (fp32 of the bf16 values).
 template <int D>
@@ -102,7 +101,8 @@ bsattn_status run_backward(const bsattn_plan* p, const __nv_bfloat16* q, const _
   const Geom g = make_geom(p);
   const size_t rows = (size_t)g.B * g.Hh * g.N;  // tile rows of the lists
   const int words = (g.N + 31) / 32;
-  bwd_delta_kernel<D><<<(unsigned)((rows * kRowsT + 63) / 64), 256, 0, st>>>(o, d_o, w.delta, rows * kRowsT);
+  const size_t qrows = rows * g.V;  // query rows of the tiled layout
+  bwd_delta_kernel<D><<<(unsigned)((qrows + 63) / 64), 256, 0, st>>>(o, d_o, w.delta, qrows);
   BSATTN_CUDA_TRY(cudaMemsetAsync(w.bm, 0, rows * words * sizeof(uint32_t), st));
   bwd_bitmap_kernel<<<(unsigned)rows, 64, 0, st>>>(idx, cnt, g.N, p->kmax, words, w.bm, p->d_err);
   bwd_compact_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(w.bm, g.N, words, rows, w.idxT, w.cntT);

@@ -5,10 +5,12 @@
 //   dQ_i = scale * sum_j dS_ij K_j,  dS_ij = P_ij * (dO_i V_j^T - Delta_i),
 //   P_ij = 2^(scale log2(e) Q_i K_j^T - lse_i log2(e)),  Delta = rowsum(dO * O).
 //
-// Work unit, as in the forward kernel: two adjacent query tiles (w for top-k
-// and top-p, t for a window without w reach) stacked into one 128-row block,
-// walking the union of their kept lists; a key tile kept by only one of the
-// two gives zero dS to the other's rows.
+// Work unit, as in the forward kernel: a 128-row block of two 64-row chunks.
+// With 64-token tiles, two adjacent query tiles (w for top-k and top-p, t for
+// a window without w reach) walking the union of their kept lists (a key tile
+// kept by only one of the two gives zero dS to the other's rows); with tiles
+// of several chunks, chunks 2b and 2b + 1 of one query tile walking every
+// real chunk of each kept key tile.
 //
 // Roles (320 threads, one CTA per SM):
 //   warps 0-7  warps w and w + 4 own query rows 32 (w % 4) .. (TMEM lanes);
@@ -81,6 +83,106 @@ struct DqCfg {
   static_assert(128 * O_PITCH <= OFF_BAR - OFF_K, "epilogue staging fits in the rings");
 };
 
+// Work item -> its two (tile, chunk) halves; i1 = -1 when the second half is
+// absent. 64-token tiles: adjacent tiles along the pair axis. Tiles of several
+// chunks: chunks 2b and 2b + 1 of one tile (padding-only chunks included, so
+// that their rows of the tiled gradients are written, as zeros).
+__device__ __forceinline__ void block_halves(const Geom& g, int pair_axis, const int* pdim, int item, int* i0,
+                                             int* i1, int* c0, int* c1) {
+  if (g.nchunk > 1) {
+    const int per = (g.nchunk + 1) / 2;
+    *i0 = *i1 = item / per;
+    *c0 = 2 * (item % per);
+    *c1 = *c0 + 1;
+    if (*c1 >= g.nchunk) *i1 = -1;
+    return;
+  }
+  const int nd[3] = {g.nT, g.nH, g.nW};
+  int c[3], rem = item;
+  c[2] = rem % pdim[2];
+  rem /= pdim[2];
+  c[1] = rem % pdim[1];
+  c[0] = rem / pdim[1];
+  c[pair_axis] *= 2;
+  *i0 = (c[0] * g.nH + c[1]) * g.nW + c[2];
+  c[pair_axis] += 1;
+  *i1 = c[pair_axis] < nd[pair_axis] ? (c[0] * g.nH + c[1]) * g.nW + c[2] : -1;
+  *c0 = *c1 = 0;
+}
+
+// Whether chunk c of tile j holds a real token (its first row is in the grid).
+__device__ __forceinline__ bool chunk_is_real(const Geom& g, int j, int c) {
+  const ChunkOrigin o = chunk_origin(g, c);
+  const int bt = j / (g.nH * g.nW), bhh = (j / g.nW) % g.nH, bw = j % g.nW;
+  return bt * g.tt + o.dt < g.T && bhh * g.th + o.dh < g.H && bw * g.tw + o.dw < g.W;
+}
+
+// Compacts the union of two tile bitmaps into the ascending step list, one
+// step per real 64-row chunk of each listed tile: tile in bits 0-20, chunk in
+// bits 21-29, bit 30 (31) from the first (second) bitmap; ext gets the
+// chunk's real extent from its first token (t, h, w bytes, capped at 255) and
+// bit 31 when the chunk has padded rows. *count = steps (capped at cap). All
+// threads of the CTA take part; the block-scan scratch holds one int per warp.
+template <int NT>
+__device__ __forceinline__ void compact_steps(const Geom& g, const uint32_t* bmA, const uint32_t* bmB, int words,
+                                              uint32_t* list, uint32_t* ext, int cap, int* scan, uint32_t* count) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int wpt = (words + NT - 1) / NT;
+  const int w0 = min(tid * wpt, words), w1 = min(w0 + wpt, words);
+  int mine = 0;
+  for (int w = w0; w < w1; ++w) {
+    uint32_t bits = bmA[w] | bmB[w];
+    if (g.nchunk == 1) {
+      mine += __popc(bits);
+    } else {
+      while (bits) {
+        const int j = w * 32 + __ffs(bits) - 1;
+        for (int c = 0; c < g.nchunk; ++c) mine += chunk_is_real(g, j, c) ? 1 : 0;
+        bits &= bits - 1;
+      }
+    }
+  }
+  int x = mine;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) scan[warp] = x;
+  __syncthreads();
+  int off = 0, tot = 0;
+#pragma unroll
+  for (int i = 0; i < NT / 32; ++i) {
+    off += i < warp ? scan[i] : 0;
+    tot += scan[i];
+  }
+  int pos = off + x - mine;
+  for (int w = w0; w < w1; ++w) {
+    const uint32_t a = bmA[w], bb = bmB[w];
+    uint32_t bits = a | bb;
+    while (bits) {
+      const int bit = __ffs(bits) - 1;
+      bits &= bits - 1;
+      const int j = w * 32 + bit;
+      const uint32_t e = (uint32_t)j | (((a >> bit) & 1u) << 30) | (((bb >> bit) & 1u) << 31);
+      const int bt = j / (g.nH * g.nW), bhh = (j / g.nW) % g.nH, bw = j % g.nW;
+      for (int c = 0; c < g.nchunk; ++c) {
+        if (g.nchunk > 1 && !chunk_is_real(g, j, c)) continue;
+        if (pos < cap) {
+          const ChunkOrigin o = chunk_origin(g, c);
+          const int vt = min(g.T - bt * g.tt - o.dt, 255), vh = min(g.H - bhh * g.th - o.dh, 255),
+                    vw = min(g.W - bw * g.tw - o.dw, 255);
+          const bool edge = vt < g.ct || vh < g.ch || vw < g.cw;
+          list[pos] = e | ((uint32_t)c << 21);
+          ext[pos] = (uint32_t)vt | ((uint32_t)vh << 8) | ((uint32_t)vw << 16) | (edge ? 1u << 31 : 0u);
+        }
+        ++pos;
+      }
+    }
+  }
+  if (tid == 0) *count = (uint32_t)min(tot, cap);
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
@@ -107,24 +209,14 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   uint32_t* uext = ulist + P.umax;
 
   const Geom& g = P.g;
-  int i0, i1;
-  {
-    const int nd[3] = {g.nT, g.nH, g.nW};
-    int c[3], rem = blockIdx.x;
-    c[2] = rem % P.pdim[2];
-    rem /= P.pdim[2];
-    c[1] = rem % P.pdim[1];
-    c[0] = rem / P.pdim[1];
-    c[P.pair_axis] *= 2;
-    i0 = (c[0] * g.nH + c[1]) * g.nW + c[2];
-    c[P.pair_axis] += 1;
-    i1 = c[P.pair_axis] < nd[P.pair_axis] ? (c[0] * g.nH + c[1]) * g.nW + c[2] : -1;
-  }
+  int i0, i1, c0 = 0, c1 = 0;
+  block_halves(g, P.pair_axis, P.pdim, blockIdx.x, &i0, &i1, &c0, &c1);
   const int head = blockIdx.y, b = blockIdx.z;
   const size_t bh = (size_t)b * g.Hh + head;
   const bool has1 = i1 >= 0;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  auto tile_row = [&](int j) -> int { return (int)((bh * g.N + j) * 64); };
+  // First tiled-layout row of chunk c of tile j.
+  auto tile_row = [&](int j, int c) -> int { return (int)((bh * g.N + j) * g.V) + 64 * c; };
 
   // ------------------------------------------------------------ setup
   if (tid == 0) {
@@ -146,8 +238,8 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     tc::tmem_alloc(sb + C::OFF_MISC, kTmemCols);
     tc::tmem_relinquish();
   }
-  if (tid < 64) {
-    const int dt = tid / (g.th * g.tw), dh = (tid / g.tw) % g.th, dw = tid % g.tw;
+  if (tid < 64) {  // in-chunk (t, h, w) offsets of each chunk row
+    const int dt = tid / (g.ch * g.cw), dh = (tid / g.cw) % g.ch, dw = tid % g.cw;
     colc[tid] = (uint32_t)dt | ((uint32_t)dh << 8) | ((uint32_t)dw << 16);
   }
   for (int w = tid; w < 2 * P.bm_words; w += kThreads) bmA[w] = 0u;
@@ -161,9 +253,11 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   }
   __syncthreads();
 
-  // Union of the two kept lists, ascending: key tile in bits 0-29, bit 30
-  // (31) when the first (second) query tile keeps it; uext holds each key
-  // tile's real extent (t, h, w bytes) and bit 31 when it has padded keys.
+  // Union of the two kept lists, ascending, one step per real 64-key chunk:
+  // key tile in bits 0-20, chunk in bits 21-29, bit 30 (31) when the first
+  // (second) query half keeps the tile; uext holds the key chunk's real
+  // extent from its first token (t, h, w bytes) and bit 31 when it has
+  // padded keys.
   int nA = P.cnt[bh * g.N + i0];
   int nB = has1 ? P.cnt[bh * g.N + i1] : 0;
   if (nA < 0 || nA > P.kmax || nB < 0 || nB > P.kmax) {
@@ -184,45 +278,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     }
   }
   __syncthreads();
-  {
-    const int wpt = (P.bm_words + kThreads - 1) / kThreads;
-    const int w0 = min(tid * wpt, P.bm_words), w1 = min(w0 + wpt, P.bm_words);
-    int mine = 0;
-    for (int w = w0; w < w1; ++w) mine += __popc(bmA[w] | bmB[w]);
-    int x = mine;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, x, o);
-      if (lane >= o) x += y;
-    }
-    if (lane == 31) scan[warp] = x;
-    __syncthreads();
-    int off = 0, tot = 0;
-#pragma unroll
-    for (int i = 0; i < kThreads / 32; ++i) {
-      off += i < warp ? scan[i] : 0;
-      tot += scan[i];
-    }
-    int pos = off + x - mine;
-    for (int w = w0; w < w1; ++w) {
-      const uint32_t a = bmA[w], bb = bmB[w];
-      uint32_t bits = a | bb;
-      while (bits) {
-        const int bit = __ffs(bits) - 1;
-        bits &= bits - 1;
-        const int j = w * 32 + bit;
-        if (pos < P.umax) {
-          ulist[pos] = (uint32_t)j | (((a >> bit) & 1u) << 30) | (((bb >> bit) & 1u) << 31);
-          const int bt = j / (g.nH * g.nW), bhh = (j / g.nW) % g.nH, bw = j % g.nW;
-          const int vt = min(g.T - bt * g.tt, 255), vh = min(g.H - bhh * g.th, 255), vw = min(g.W - bw * g.tw, 255);
-          const bool edge = vt < g.tt || vh < g.th || vw < g.tw;
-          uext[pos] = (uint32_t)vt | ((uint32_t)vh << 8) | ((uint32_t)vw << 16) | (edge ? 1u << 31 : 0u);
-        }
-        ++pos;
-      }
-    }
-    if (tid == 0) misc[2] = (uint32_t)min(tot, P.umax);
-  }
+  compact_steps<kThreads>(g, bmA, bmB, P.bm_words, ulist, uext, P.umax, scan, misc + 2);
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
@@ -238,12 +294,12 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       tc::tma_prefetch_desc(&tmV);
       tc::mbar_arrive_expect_tx(bar_q, (has1 ? 2 : 1) * 2 * 64 * C::QRB);
       for (int x = 0; x < (has1 ? 2 : 1); ++x) {
-        const int tile = x ? i1 : i0;
+        const int row = x ? tile_row(i1, c1) : tile_row(i0, c0);
 #pragma unroll
         for (int cb = 0; cb < C::QBLK; ++cb) {
           const uint32_t d = cb * 128 * 128 + x * 64 * 128;
-          tc::tma_load_2d(sb + C::OFF_Q + d, &tmQ, bar_q, cb * 64, tile_row(tile));
-          tc::tma_load_2d(sb + C::OFF_DO + d, &tmDO, bar_q, cb * 64, tile_row(tile));
+          tc::tma_load_2d(sb + C::OFF_Q + d, &tmQ, bar_q, cb * 64, row);
+          tc::tma_load_2d(sb + C::OFF_DO + d, &tmDO, bar_q, cb * 64, row);
         }
       }
       int last[kStages];
@@ -256,12 +312,12 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
           atomicOr(P.err, BSATTN_DEVERR_TIMEOUT);
           break;
         }
-        const int kt = (int)(ulist[m] & 0x3FFFFFFFu);
+        const int krow = tile_row((int)(ulist[m] & 0x1FFFFFu), (int)((ulist[m] >> 21) & 0x1FFu));
         tc::mbar_arrive_expect_tx(bar_full(s), 2 * C::T_BYTES);
 #pragma unroll
         for (int cb = 0; cb < C::QBLK; ++cb) {
-          tc::tma_load_2d(sb + C::OFF_K + s * C::T_BYTES + cb * 64 * 128, &tmK, bar_full(s), cb * 64, tile_row(kt));
-          tc::tma_load_2d(sb + C::OFF_V + s * C::T_BYTES + cb * 64 * 128, &tmV, bar_full(s), cb * 64, tile_row(kt));
+          tc::tma_load_2d(sb + C::OFF_K + s * C::T_BYTES + cb * 64 * 128, &tmK, bar_full(s), cb * 64, krow);
+          tc::tma_load_2d(sb + C::OFF_V + s * C::T_BYTES + cb * 64 * 128, &tmV, bar_full(s), cb * 64, krow);
         }
         last[s] = m;
       }
@@ -332,8 +388,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     const int half = r >> 6;
     const bool row_exists = half == 0 || has1;
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
-    const int qtile = half ? i1 : i0;
-    const size_t lrow = row_exists ? (size_t)tile_row(qtile) + (r & 63) : 0;
+    const size_t lrow = row_exists ? (size_t)(half ? tile_row(i1, c1) : tile_row(i0, c0)) + (r & 63) : 0;
     const float lse2 = row_exists ? P.lse[lrow] * 1.4426950408889634f : 0.f;
     const float dlt = row_exists ? P.delta[lrow] : 0.f;
     const float c = P.scale_log2;
@@ -422,7 +477,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     for (int e2 = tid; e2 < rows * CPR; e2 += kSoftmaxThreads) {
       const int rr = e2 / CPR, cc = e2 % CPR;
       const uint4 val = *reinterpret_cast<const uint4*>(smem + C::OFF_K + rr * C::O_PITCH + cc * 16);
-      uint4* og = reinterpret_cast<uint4*>(P.dq + (size_t)tile_row(rr >> 6 ? i1 : i0) * D);
+      uint4* og = reinterpret_cast<uint4*>(P.dq + (size_t)(rr >> 6 ? tile_row(i1, c1) : tile_row(i0, c0)) * D);
       og[(rr & 63) * CPR + cc] = val;
     }
   }
@@ -440,7 +495,7 @@ template <int D>
 bsattn_status run_dq(const bsattn_plan* p, const void* q, const void* k, const void* v, const void* d_o,
                      DqParams prm, cudaStream_t st) {
   using C = DqCfg<D>;
-  const uint64_t rows = (uint64_t)p->desc.B * p->desc.heads * p->N * 64;
+  const uint64_t rows = (uint64_t)p->desc.B * p->desc.heads * p->N * p->V;
   if (rows + 128 >= (1ull << 31)) return BSATTN_ERR_UNSUPPORTED;
   CUtensorMap mq, mdo, mk, mv;
   const auto bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
@@ -454,7 +509,8 @@ bsattn_status run_dq(const bsattn_plan* p, const void* q, const void* k, const v
   auto kern = bwd_dq_tc_kernel<D>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return BSATTN_ERR_CUDA;
-  dim3 grid(prm.pdim[0] * prm.pdim[1] * prm.pdim[2], p->desc.heads, p->desc.B);
+  const int items = p->nchunk > 1 ? p->N * ((p->nchunk + 1) / 2) : prm.pdim[0] * prm.pdim[1] * prm.pdim[2];
+  dim3 grid(items, p->desc.heads, p->desc.B);
   kern<<<grid, kThreads, smem, st>>>(mq, mdo, mk, mv, prm);
   return cudaGetLastError() == cudaSuccess ? BSATTN_OK : BSATTN_ERR_CUDA;
 }
@@ -537,35 +593,21 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   uint32_t* uext = ulist + P.umax;
 
   const Geom& g = P.g;
-  int j0, j1;
-  {
-    const int nd[3] = {g.nT, g.nH, g.nW};
-    int c[3], rem = blockIdx.x;
-    c[2] = rem % P.pdim[2];
-    rem /= P.pdim[2];
-    c[1] = rem % P.pdim[1];
-    c[0] = rem / P.pdim[1];
-    c[P.pair_axis] *= 2;
-    j0 = (c[0] * g.nH + c[1]) * g.nW + c[2];
-    c[P.pair_axis] += 1;
-    j1 = c[P.pair_axis] < nd[P.pair_axis] ? (c[0] * g.nH + c[1]) * g.nW + c[2] : -1;
-  }
+  int j0, j1, kc0 = 0, kc1 = 0;
+  block_halves(g, P.pair_axis, P.pdim, blockIdx.x, &j0, &j1, &kc0, &kc1);
   const int head = blockIdx.y, b = blockIdx.z;
   const size_t bh = (size_t)b * g.Hh + head;
   const bool has1 = j1 >= 0;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  auto tile_row = [&](int j) -> int { return (int)((bh * g.N + j) * 64); };
-  // Bit r set when in-tile row r of tile j is a real token.
-  auto real_rows = [&](int j) -> uint64_t {
+  // First tiled-layout row of chunk c of tile j.
+  auto tile_row = [&](int j, int c) -> int { return (int)((bh * g.N + j) * g.V) + 64 * c; };
+  // Whether row q of chunk c of tile j is a real token.
+  auto row_is_real = [&](int j, int c, int q) -> bool {
+    const ChunkOrigin o = chunk_origin(g, c);
     const int bt = j / (g.nH * g.nW), bhh = (j / g.nW) % g.nH, bw = j % g.nW;
-    const int vt = g.T - bt * g.tt, vh = g.H - bhh * g.th, vw = g.W - bw * g.tw;
-    if (vt >= g.tt && vh >= g.th && vw >= g.tw) return ~0ull;
-    uint64_t m = 0;
-    for (int r = 0; r < 64; ++r) {
-      const uint32_t cc = colc[r];
-      if ((int)(cc & 0xffu) < vt && (int)((cc >> 8) & 0xffu) < vh && (int)((cc >> 16) & 0xffu) < vw) m |= 1ull << r;
-    }
-    return m;
+    const uint32_t cc = colc[q];
+    return bt * g.tt + o.dt + (int)(cc & 0xffu) < g.T && bhh * g.th + o.dh + (int)((cc >> 8) & 0xffu) < g.H &&
+           bw * g.tw + o.dw + (int)((cc >> 16) & 0xffu) < g.W;
   };
 
   // ------------------------------------------------------------ setup
@@ -588,8 +630,8 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     tc::tmem_alloc(sb + C::OFF_MISC, kTmemCols);
     tc::tmem_relinquish();
   }
-  if (tid < 64) {
-    const int dt = tid / (g.th * g.tw), dh = (tid / g.tw) % g.th, dw = tid % g.tw;
+  if (tid < 64) {  // in-chunk (t, h, w) offsets of each chunk row
+    const int dt = tid / (g.ch * g.cw), dh = (tid / g.cw) % g.ch, dw = tid % g.cw;
     colc[tid] = (uint32_t)dt | ((uint32_t)dh << 8) | ((uint32_t)dw << 16);
   }
   for (int w = tid; w < 2 * P.bm_words; w += kThreads) bmA[w] = 0u;
@@ -603,9 +645,10 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   }
   __syncthreads();
 
-  // Union of the two transposed lists, ascending: query tile in bits 0-29,
-  // bit 30 (31) when it keeps j0 (j1); uext holds the query tile's real
-  // extent and bit 31 when it has padded rows.
+  // Union of the two transposed lists, ascending, one step per real chunk of
+  // each listed query tile: query tile in bits 0-20, chunk in bits 21-29, bit
+  // 30 (31) when it keeps j0 (j1); uext holds the query chunk's real extent
+  // and bit 31 when it has padded rows.
   {
     const int nA = min(max(P.cntT[bh * g.N + j0], 0), g.N);
     const int nB = has1 ? min(max(P.cntT[bh * g.N + j1], 0), g.N) : 0;
@@ -618,45 +661,7 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     }
   }
   __syncthreads();
-  {
-    const int wpt = (P.bm_words + kThreads - 1) / kThreads;
-    const int w0 = min(tid * wpt, P.bm_words), w1 = min(w0 + wpt, P.bm_words);
-    int mine = 0;
-    for (int w = w0; w < w1; ++w) mine += __popc(bmA[w] | bmB[w]);
-    int x = mine;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, x, o);
-      if (lane >= o) x += y;
-    }
-    if (lane == 31) scan[warp] = x;
-    __syncthreads();
-    int off = 0, tot = 0;
-#pragma unroll
-    for (int i = 0; i < kThreads / 32; ++i) {
-      off += i < warp ? scan[i] : 0;
-      tot += scan[i];
-    }
-    int pos = off + x - mine;
-    for (int w = w0; w < w1; ++w) {
-      const uint32_t a = bmA[w], bb = bmB[w];
-      uint32_t bits = a | bb;
-      while (bits) {
-        const int bit = __ffs(bits) - 1;
-        bits &= bits - 1;
-        const int i = w * 32 + bit;
-        if (pos < P.umax) {
-          ulist[pos] = (uint32_t)i | (((a >> bit) & 1u) << 30) | (((bb >> bit) & 1u) << 31);
-          const int bt = i / (g.nH * g.nW), bhh = (i / g.nW) % g.nH, bw = i % g.nW;
-          const int vt = min(g.T - bt * g.tt, 255), vh = min(g.H - bhh * g.th, 255), vw = min(g.W - bw * g.tw, 255);
-          const bool edge = vt < g.tt || vh < g.th || vw < g.tw;
-          uext[pos] = (uint32_t)vt | ((uint32_t)vh << 8) | ((uint32_t)vw << 16) | (edge ? 1u << 31 : 0u);
-        }
-        ++pos;
-      }
-    }
-    if (tid == 0) misc[2] = (uint32_t)min(tot, P.umax);
-  }
+  compact_steps<kThreads>(g, bmA, bmB, P.bm_words, ulist, uext, P.umax, scan, misc + 2);
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
@@ -672,12 +677,12 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       tc::tma_prefetch_desc(&tmV);
       tc::mbar_arrive_expect_tx(bar_kv, (has1 ? 2 : 1) * 2 * 64 * C::QRB);
       for (int x = 0; x < (has1 ? 2 : 1); ++x) {
-        const int tile = x ? j1 : j0;
+        const int row = x ? tile_row(j1, kc1) : tile_row(j0, kc0);
 #pragma unroll
         for (int cb = 0; cb < C::QBLK; ++cb) {
           const uint32_t d = cb * 128 * 128 + x * 64 * 128;
-          tc::tma_load_2d(sb + C::OFF_K + d, &tmK, bar_kv, cb * 64, tile_row(tile));
-          tc::tma_load_2d(sb + C::OFF_V + d, &tmV, bar_kv, cb * 64, tile_row(tile));
+          tc::tma_load_2d(sb + C::OFF_K + d, &tmK, bar_kv, cb * 64, row);
+          tc::tma_load_2d(sb + C::OFF_V + d, &tmV, bar_kv, cb * 64, row);
         }
       }
       int last[kStages];
@@ -690,16 +695,16 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
           atomicOr(P.err, BSATTN_DEVERR_TIMEOUT);
           break;
         }
-        const int qt = (int)(ulist[m] & 0x3FFFFFFFu);
+        const int qrow = tile_row((int)(ulist[m] & 0x1FFFFFu), (int)((ulist[m] >> 21) & 0x1FFu));
         const uint32_t st = sb + C::OFF_RING + s * C::STAGE;
         tc::mbar_arrive_expect_tx(bar_full(s), 2 * C::T_BYTES + 512);
 #pragma unroll
         for (int cb = 0; cb < C::QBLK; ++cb) {
-          tc::tma_load_2d(st + cb * 64 * 128, &tmQ, bar_full(s), cb * 64, tile_row(qt));
-          tc::tma_load_2d(st + C::T_BYTES + cb * 64 * 128, &tmDO, bar_full(s), cb * 64, tile_row(qt));
+          tc::tma_load_2d(st + cb * 64 * 128, &tmQ, bar_full(s), cb * 64, qrow);
+          tc::tma_load_2d(st + C::T_BYTES + cb * 64 * 128, &tmDO, bar_full(s), cb * 64, qrow);
         }
-        tc::bulk_load(st + 2 * C::T_BYTES, P.lse + tile_row(qt), 256, bar_full(s));
-        tc::bulk_load(st + 2 * C::T_BYTES + 256, P.delta + tile_row(qt), 256, bar_full(s));
+        tc::bulk_load(st + 2 * C::T_BYTES, P.lse + qrow, 256, bar_full(s));
+        tc::bulk_load(st + 2 * C::T_BYTES + 256, P.delta + qrow, 256, bar_full(s));
         last[s] = m;
       }
       if (*abort_flag) {
@@ -772,7 +777,7 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     const int r = quad * 32 + lane;                // key row of the block
     const int half = r >> 6;                       // 0: tile j0, 1: tile j1
     const bool row_exists = half == 0 || has1;
-    const bool key_real = row_exists && ((real_rows(half ? j1 : j0) >> (r & 63)) & 1);
+    const bool key_real = row_exists && (half ? row_is_real(j1, kc1, r & 63) : row_is_real(j0, kc0, r & 63));
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
     const float c = P.scale_log2;
     bool ok = true;
@@ -878,7 +883,7 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       const int rr = rem / CPR, cc = rem % CPR;
       const uint4 val = *reinterpret_cast<const uint4*>(smem + C::OFF_RING + (which * 128 + rr) * C::O_PITCH + cc * 16);
       __nv_bfloat16* dst = which == 0 ? P.dk : P.dv;
-      uint4* og = reinterpret_cast<uint4*>(dst + (size_t)tile_row(rr >> 6 ? j1 : j0) * D);
+      uint4* og = reinterpret_cast<uint4*>(dst + (size_t)(rr >> 6 ? tile_row(j1, kc1) : tile_row(j0, kc0)) * D);
       og[(rr & 63) * CPR + cc] = val;
     }
   }
@@ -896,7 +901,7 @@ template <int D>
 bsattn_status run_dkdv(const bsattn_plan* p, const void* q, const void* k, const void* v, const void* d_o,
                        KvParams prm, cudaStream_t st) {
   using C = KvCfg<D>;
-  const uint64_t rows = (uint64_t)p->desc.B * p->desc.heads * p->N * 64;
+  const uint64_t rows = (uint64_t)p->desc.B * p->desc.heads * p->N * p->V;
   if (rows + 128 >= (1ull << 31)) return BSATTN_ERR_UNSUPPORTED;
   CUtensorMap mq, mdo, mk, mv;
   const auto bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
@@ -910,7 +915,8 @@ bsattn_status run_dkdv(const bsattn_plan* p, const void* q, const void* k, const
   auto kern = bwd_dkdv_tc_kernel<D>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return BSATTN_ERR_CUDA;
-  dim3 grid(prm.pdim[0] * prm.pdim[1] * prm.pdim[2], p->desc.heads, p->desc.B);
+  const int items = p->nchunk > 1 ? p->N * ((p->nchunk + 1) / 2) : prm.pdim[0] * prm.pdim[1] * prm.pdim[2];
+  dim3 grid(items, p->desc.heads, p->desc.B);
   kern<<<grid, kThreads, smem, st>>>(mq, mdo, mk, mv, prm);
   return cudaGetLastError() == cudaSuccess ? BSATTN_OK : BSATTN_ERR_CUDA;
 }
@@ -931,7 +937,8 @@ bsattn_status launch_backward_dq_tc(const bsattn_plan* p, const void* q, const v
   prm.scale = p->scale;
   prm.scale_log2 = p->scale * 1.4426950408889634f;
   prm.err = p->d_err;
-  prm.umax = p->N < 2 * p->kmax ? p->N : 2 * p->kmax;
+  // Steps: the union of two kept lists (one list for tiles of several chunks), times the chunks.
+  prm.umax = p->nchunk == 1 ? (p->N < 2 * p->kmax ? p->N : 2 * p->kmax) : (p->N < p->kmax ? p->N : p->kmax) * p->nchunk;
   prm.bm_words = (p->N + 31) / 32;
   prm.pair_axis = (p->rule.kind == BSATTN_RULE_WINDOW && p->rule.win_w == 0) ? 0 : 2;
   const int nd[3] = {p->nT, p->nH, p->nW};
@@ -953,7 +960,8 @@ bsattn_status launch_backward_dkdv_tc(const bsattn_plan* p, const void* q, const
   prm.scale = p->scale;
   prm.scale_log2 = p->scale * 1.4426950408889634f;
   prm.err = p->d_err;
-  prm.umax = p->N;  // the union of two transposed lists holds at most N query tiles
+  // Steps: at most N query tiles in the union of two transposed lists, times their chunks.
+  prm.umax = p->N * p->nchunk;
   prm.bm_words = (p->N + 31) / 32;
   prm.pair_axis = (p->rule.kind == BSATTN_RULE_WINDOW && p->rule.win_w == 0) ? 0 : 2;
   const int nd[3] = {p->nT, p->nH, p->nW};

@@ -115,7 +115,7 @@ static inline bool layer_tiles_kv(const bsattn_plan* p) {
 size_t attention_workspace_bytes(const bsattn_plan* p);
 // Scratch of the backward pass (carved from the caller's workspace).
 struct BackwardWs {
-  float* delta;    // [B, Hh, N, 64] rowsum(dO * O)
+  float* delta;    // [B, Hh, N, V] rowsum(dO * O)
   uint32_t* bm;    // [B, Hh, N, ceil(N/32)] transposed kept-list bitmaps
   int32_t* idxT;   // [B, Hh, N, N] query tiles keeping each key tile, ascending
   int32_t* cntT;   // [B, Hh, N]

@@ -82,7 +82,7 @@ LayerWs carve_layer(const bsattn_plan* p, Carve& c) {
 BackwardWs carve_backward(const bsattn_plan* p, Carve& c) {
   const size_t rows = (size_t)p->desc.B * p->desc.heads * p->N;
   BackwardWs w;
-  w.delta = (float*)c.take(rows * 64 * sizeof(float));
+  w.delta = (float*)c.take(rows * p->V * sizeof(float));
   w.bm = (uint32_t*)c.take(rows * ((p->N + 31) / 32) * sizeof(uint32_t));
   w.idxT = (int32_t*)c.take(rows * p->N * sizeof(int32_t));
   w.cntT = (int32_t*)c.take(rows * sizeof(int32_t));
@@ -375,7 +375,7 @@ bsattn_status attn_backward(const bsattn_plan* p, const void* q, const void* k, 
   if (!p || !ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(o) || !ok_ptr(d_o) || !ok_ptr(lse) ||
       !ok_ptr(idx) || !ok_ptr(cnt) || !ok_ptr(dq) || !ok_ptr(dk) || !ok_ptr(dv))
     return BSATTN_ERR_INVALID_ARG;
-  if (p->desc.qk_fp8 || p->V != 64) return BSATTN_ERR_UNSUPPORTED;
+  if (p->desc.qk_fp8) return BSATTN_ERR_UNSUPPORTED;
   bsattn_info info;
   attn_plan_info(p, &info);
   if (!ws || !aligned16(ws) || ws_bytes < info.backward_workspace_bytes) return BSATTN_ERR_WORKSPACE;

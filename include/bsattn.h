@@ -245,13 +245,14 @@ bsattn_status attn_layer(const bsattn_plan* plan, const void* q_nat, const void*
 /* Backward of attn_forward (trainable block-sparse attention: "Faster Video
  * Diffusion with Trainable Sparse Attention", reproducibility record,
  * Research Type row). Tiled bf16 q, k, v, the forward's tiled bf16 o and fp32
- * lse [B, Hh, N, 64], the incoming gradient d_o (tiled bf16) and the kept
+ * lse [B, Hh, N, V], the incoming gradient d_o (tiled bf16) and the kept
  * lists the forward used; writes tiled bf16 dq, dk, dv. With P the masked
  * softmax recomputed from q, k and lse: dV = P^T dO, dS = P * (dO V^T -
  * rowsum(dO * O)), dQ = scale dS K, dK = scale dS^T Q, over kept tile pairs
  * and real (unpadded) tokens; rows of padded slots get zero gradients. P and
- * dS are rounded to bf16 for the products (fp32 accumulation). Tiles of 64
- * tokens and bf16 Q/K only (UNSUPPORTED otherwise). `ws` must hold
+ * dS are rounded to bf16 for the products (fp32 accumulation). Any tile
+ * shape attn_plan_create accepts; bf16 Q/K only (UNSUPPORTED for qk_fp8
+ * plans). `ws` must hold
  * info.backward_workspace_bytes (rowsum, transposed lists). A list entry
  * outside [0, N) sets the device error word and is skipped. */
 bsattn_status attn_backward(const bsattn_plan* plan, const void* q, const void* k, const void* v,

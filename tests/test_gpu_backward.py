@@ -25,7 +25,8 @@ def _grad_close(got, ref, name):
     assert np.abs(err).max() <= 3e-2 * np.abs(ref).max(), (name, np.abs(err).max(), np.abs(ref).max())
 
 
-@pytest.mark.parametrize("name", ["tiny_d64", "ragged_topk", "ragged_topp", "ragged_bf16_window"])
+@pytest.mark.parametrize("name", ["tiny_d64", "ragged_topk", "ragged_topp", "ragged_bf16_window",
+                                  "tile688_topk", "tile488_topp", "tile11x128_d64"])
 def test_backward_against_oracle(bs, name):
     wl = SMALL[name]
     plan = bs.Plan.for_workload(wl)
