@@ -5,12 +5,24 @@
 // accumulates hi*hi + hi*lo + lo*hi in fp32 in TMEM. What is left out (lo*lo
 // and the TF32 rounding of lo) stays below 2^-20 of |a||b| per product.
 //
-// One CTA computes a 128 x 128 block of S: for each 32-column slice of D, TMA
-// brings the Pq and Pk row slices (128 rows x 128 bytes, 128-byte swizzle)
-// into shared memory, the CTA splits them in place into hi and a lo copy (an
-// element-wise pass keeps the swizzled layout), one thread issues the twelve
-// MMAs, and at the end the accumulator is read back with tcgen05.ld, scaled
-// and stored. Three CTAs per SM overlap one another's loads, splits and MMAs.
+// The output is cut into 128 x 128 blocks; a persistent CTA (one per SM)
+// takes a contiguous run of blocks, so that consecutive blocks share their
+// query rows (bh, bi). Roles:
+//   warp 8    TMA: the Pq block (all of D) into a staging buffer when the row
+//             block changes, and Pk row slices of 32 columns (128 rows x 128
+//             bytes, 128-byte swizzle) into a ring;
+//   warps 4-7 split: the Pq block goes to TMEM as hi and lo columns (TMEM
+//             lane = row; the MMAs take A from TMEM, so it costs no shared
+//             memory bandwidth per block), each Pk slice is split in place
+//             into hi and a lo copy;
+//   warp 9    one thread issues the twelve MMAs per slice into one of two TMEM
+//             accumulators;
+//   warps 0-3 read a finished accumulator with tcgen05.ld (lane = output row),
+//             scale it, transpose 32 x 32 pieces through shared memory and
+//             store whole 128-byte row segments, while the next block runs.
+// Every block is accumulated in the same order (slices ascending, then the
+// 8-wide K steps, hi*hi, hi*lo, lo*hi), so the result does not depend on how
+// blocks are shared among CTAs.
 #include "internal.h"
 #include "tc_common.cuh"
 
@@ -19,142 +31,355 @@ namespace {
 constexpr int kRows = 128;                       // output block edge (M = N = 128)
 constexpr int kSlice = 32;                       // fp32 columns of D per slice (128 bytes)
 constexpr int kSliceBytes = kRows * kSlice * 4;  // 16 KB per operand slice
-constexpr int OFF_AHI = 0, OFF_BHI = kSliceBytes, OFF_ALO = 2 * kSliceBytes, OFF_BLO = 3 * kSliceBytes;
-constexpr int OFF_BAR = 4 * kSliceBytes;         // load barrier, MMA barrier
-constexpr int OFF_TMEM = OFF_BAR + 16;           // TMEM base address, then a word that stays 0
-constexpr int kSmem = OFF_TMEM + 16 + 1024;      // + alignment slack
+constexpr int kStages = 4;                       // Pk slice ring
+constexpr int kThreads = 320;
+constexpr int kSplitThreads = 128;
+constexpr int kEpiBytes = 32 * 128;              // one warp's 32 x 32 transpose buffer
 constexpr long long kWaitLimit = 4000000000LL;   // SM cycles (~2 s)
 
-__device__ __forceinline__ void mma_tf32(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+template <int D>
+struct ScoresCfg {
+  static constexpr int KS = D / kSlice;                   // slices per block
+  static constexpr int OFF_ASTG = 0;                      // Pq block staging, KS slices
+  static constexpr int OFF_RING = KS * kSliceBytes;       // stage s: Pk hi, then Pk lo
+  static constexpr int STAGE = 2 * kSliceBytes;
+  static constexpr int OFF_EPI = OFF_RING + kStages * STAGE;
+  static constexpr int OFF_BAR = OFF_EPI + 4 * kEpiBytes;
+  // a_full, a_stage_free, a_split, a_free, b_full[S], b_split[S], b_empty[S], acc_full[2],
+  // acc_empty[2], final
+  static constexpr int NBAR = 4 + 3 * kStages + 4 + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;     // TMEM base, abort flag, a word that stays 0
+  static constexpr int SMEM = OFF_MISC + 16 + 1024;       // + alignment slack
+  // TMEM columns: Pq hi [0, D), Pq lo [D, 2D), accumulators at 2D and 2D + 128.
+  static constexpr uint32_t COL_LO = D, COL_ACC = 2 * D;
+  static_assert(SMEM <= 232448, "block scores shared memory");
+  static_assert(2 * D + 2 * kRows <= 512, "TMEM columns");
+};
+
+struct ScoresParams {
+  int N;              // tiles per (batch, head)
+  int nb;             // 128-row blocks per (batch, head)
+  long long blocks;   // B * Hh * nb * nb
+  float scale;
+  float* S;
+  int* err;
+};
+
+// D[tmem] (+)= A[tmem] * B[smem desc], TF32 operands.
+__device__ __forceinline__ void mma_ts_tf32(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc,
+                                            uint32_t acc) {
   asm volatile(
       "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
-      "l"(a), "l"(b), "r"(idesc), "r"(acc)
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc)
       : "memory");
 }
 
+__device__ __forceinline__ uint32_t hi_bits(uint32_t x) { return x & 0xFFFFE000u; }
+
+// Split one Pk slice in place: hi over the loaded values, lo = x - hi into
+// the slice after it. Thread t takes 16-byte pieces t, t + 128, ...
+__device__ __forceinline__ void split_slice(uint8_t* hi, int t) {
+  float4 x[kSliceBytes / 16 / kSplitThreads];
+#pragma unroll
+  for (int u = 0; u < kSliceBytes / 16 / kSplitThreads; ++u)
+    x[u] = reinterpret_cast<const float4*>(hi)[t + u * kSplitThreads];
+#pragma unroll
+  for (int u = 0; u < kSliceBytes / 16 / kSplitThreads; ++u) {
+    const float4 h = make_float4(__uint_as_float(hi_bits(__float_as_uint(x[u].x))),
+                                 __uint_as_float(hi_bits(__float_as_uint(x[u].y))),
+                                 __uint_as_float(hi_bits(__float_as_uint(x[u].z))),
+                                 __uint_as_float(hi_bits(__float_as_uint(x[u].w))));
+    reinterpret_cast<float4*>(hi)[t + u * kSplitThreads] = h;
+    reinterpret_cast<float4*>(hi + kSliceBytes)[t + u * kSplitThreads] =
+        make_float4(x[u].x - h.x, x[u].y - h.y, x[u].z - h.z, x[u].w - h.w);
+  }
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 template <int D>
-__global__ void __launch_bounds__(128)
-block_scores_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int N,
-                       float scale, float* __restrict__ S, int* err) {
+__global__ void __launch_bounds__(kThreads, 1)
+block_scores_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                       ScoresParams P) {
+  using C = ScoresCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   const uint32_t sb = tc::smem_addr(smem);
-  const uint32_t bar_ld = sb + OFF_BAR, bar_mma = sb + OFF_BAR + 8;
-  volatile int* never = reinterpret_cast<volatile int*>(smem + OFF_TMEM + 8);
+  const uint32_t bar_afull = sb + C::OFF_BAR, bar_astg = bar_afull + 8, bar_asplit = bar_afull + 16,
+                 bar_afree = bar_afull + 24;
+  auto bar_bfull = [&](int s) { return sb + C::OFF_BAR + 8u * (4 + s); };
+  auto bar_bsplit = [&](int s) { return sb + C::OFF_BAR + 8u * (4 + kStages + s); };
+  auto bar_bempty = [&](int s) { return sb + C::OFF_BAR + 8u * (4 + 2 * kStages + s); };
+  auto bar_accfull = [&](int a) { return sb + C::OFF_BAR + 8u * (4 + 3 * kStages + a); };
+  auto bar_accempty = [&](int a) { return sb + C::OFF_BAR + 8u * (6 + 3 * kStages + a); };
+  const uint32_t bar_final = sb + C::OFF_BAR + 8u * (8 + 3 * kStages);
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
+  volatile int* never = reinterpret_cast<volatile int*>(misc + 2);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int bh = blockIdx.z, i0 = blockIdx.y * kRows, j0 = blockIdx.x * kRows;
+  // This CTA's contiguous run of blocks; block = ((bh * nb) + bi) * nb + bj.
+  const long long blk0 = P.blocks * blockIdx.x / gridDim.x;
+  const long long blk1 = P.blocks * (blockIdx.x + 1) / gridDim.x;
+  const int nb = P.nb;
+
   if (tid == 0) {
-    tc::mbar_init(bar_ld, 1);
-    tc::mbar_init(bar_mma, 1);
-    *never = 0;
+    tc::mbar_init(bar_afull, 1);
+    tc::mbar_init(bar_astg, kSplitThreads);
+    tc::mbar_init(bar_asplit, kSplitThreads);
+    tc::mbar_init(bar_afree, 1);
+    for (int s = 0; s < kStages; ++s) {
+      tc::mbar_init(bar_bfull(s), 1);
+      tc::mbar_init(bar_bsplit(s), kSplitThreads);
+      tc::mbar_init(bar_bempty(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      tc::mbar_init(bar_accfull(a), 1);
+      tc::mbar_init(bar_accempty(a), 128);
+    }
+    tc::mbar_init(bar_final, 1);
+    misc[1] = 0;
+    misc[2] = 0;
     tc::mbar_fence_init();
   }
-  if (warp == 0) {
-    tc::tmem_alloc(sb + OFF_TMEM, kRows);
+  if (warp == 9) {
+    tc::tmem_alloc(sb + C::OFF_MISC, 512);
     tc::tmem_relinquish();
   }
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
-  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + OFF_TMEM);
-  // TF32 inputs, fp32 accumulator, both operands K-major, M = N = 128.
-  constexpr uint32_t idesc = tc::instr_desc(2, 2, 0, 0, kRows, kRows);
-  bool ok = true;
-  int ld_pending = -1, mma_pending = -1;  // phase of a wait that gave up
-  for (int kc = 0; kc < D / kSlice; ++kc) {
-    if (tid == 0) {
-      tc::mbar_arrive_expect_tx(bar_ld, 2 * kSliceBytes);
-      tc::tma_load_2d(sb + OFF_AHI, &tmA, bar_ld, kc * kSlice, bh * N + i0);
-      tc::tma_load_2d(sb + OFF_BHI, &tmB, bar_ld, kc * kSlice, bh * N + j0);
-    }
-    if (!tc::mbar_wait(bar_ld, kc & 1, never, kWaitLimit)) ok = false;
-    if (!__syncthreads_and(ok)) {
-      ok = false;
-      ld_pending = kc & 1;
-      break;
-    }
-    // Split in place: hi keeps sign, exponent and the top 10 mantissa bits.
-    for (int q = tid; q < 2 * kSliceBytes / 16; q += 128) {
-      float4* hp = reinterpret_cast<float4*>(smem + OFF_AHI + q * 16);  // A slice, then B slice
-      float4* lp = reinterpret_cast<float4*>(smem + OFF_ALO + q * 16);
-      const float4 x = *hp;
-      const float4 h = make_float4(__uint_as_float(__float_as_uint(x.x) & 0xFFFFE000u),
-                                   __uint_as_float(__float_as_uint(x.y) & 0xFFFFE000u),
-                                   __uint_as_float(__float_as_uint(x.z) & 0xFFFFE000u),
-                                   __uint_as_float(__float_as_uint(x.w) & 0xFFFFE000u));
-      *hp = h;
-      *lp = make_float4(x.x - h.x, x.y - h.y, x.z - h.z, x.w - h.w);
-    }
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    __syncthreads();
-    if (tid == 0) {
-      tc::fence_after_sync();
-#pragma unroll
-      for (int kk = 0; kk < kSlice / 8; ++kk) {  // 8 fp32 (32 bytes) of K per MMA
-        const uint64_t ah = tc::smem_desc(sb + OFF_AHI + kk * 32, 16, 1024, tc::kLayoutSW128);
-        const uint64_t bhi = tc::smem_desc(sb + OFF_BHI + kk * 32, 16, 1024, tc::kLayoutSW128);
-        const uint64_t al = tc::smem_desc(sb + OFF_ALO + kk * 32, 16, 1024, tc::kLayoutSW128);
-        const uint64_t bl = tc::smem_desc(sb + OFF_BLO + kk * 32, 16, 1024, tc::kLayoutSW128);
-        mma_tf32(tmem, ah, bhi, idesc, (kc > 0 || kk > 0) ? 1u : 0u);
-        mma_tf32(tmem, ah, bl, idesc, 1u);
-        mma_tf32(tmem, al, bhi, idesc, 1u);
+  const uint32_t tmem = misc[0];
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ TMA
+    if (lane == 0) {
+      tc::tma_prefetch_desc(&tmA);
+      tc::tma_prefetch_desc(&tmB);
+      long long m = 0, prev = -1, last_b[kStages];
+      int arow = 0;
+      for (int s = 0; s < kStages; ++s) last_b[s] = -1;
+      bool ok = true;
+      for (long long blk = blk0; ok && blk < blk1; ++blk) {
+        const long long rk = blk / nb, bh = rk / nb;
+        const int bi = (int)(rk % nb), bj = (int)(blk % nb);
+        if (rk != prev) {
+          // The split warps must have read the previous Pq block out of staging.
+          if (arow > 0 && !tc::mbar_wait(bar_astg, (arow - 1) & 1, abort_flag, kWaitLimit)) {
+            ok = false;
+            break;
+          }
+          tc::mbar_arrive_expect_tx(bar_afull, C::KS * kSliceBytes);
+          for (int kc = 0; kc < C::KS; ++kc)
+            tc::tma_load_2d(sb + C::OFF_ASTG + kc * kSliceBytes, &tmA, bar_afull, kc * kSlice,
+                            (int)(bh * P.N + (long long)bi * kRows));
+          ++arow;
+          prev = rk;
+        }
+        for (int kc = 0; kc < C::KS; ++kc, ++m) {
+          const int s = (int)(m % kStages);
+          if (m >= kStages && !tc::mbar_wait(bar_bempty(s), (int)((m / kStages) - 1) & 1, abort_flag, kWaitLimit)) {
+            ok = false;
+            break;
+          }
+          tc::mbar_arrive_expect_tx(bar_bfull(s), kSliceBytes);
+          tc::tma_load_2d(sb + C::OFF_RING + s * C::STAGE, &tmB, bar_bfull(s), kc * kSlice,
+                          (int)(bh * P.N + (long long)bj * kRows));
+          last_b[s] = m;
+        }
       }
-      tc::mma_commit(bar_mma);
+      if (!ok) {
+        *abort_flag = 1;
+        atomicOr(P.err, BSATTN_DEVERR_TIMEOUT);
+      }
+      if (*abort_flag) {  // let this thread's copies land before the CTA goes away
+        if (arow > 0) tc::mbar_wait(bar_afull, (arow - 1) & 1, never, kWaitLimit);
+        for (int s = 0; s < kStages; ++s)
+          if (last_b[s] >= 0) tc::mbar_wait(bar_bfull(s), (int)(last_b[s] / kStages) & 1, never, kWaitLimit);
+      }
     }
-    // The slice buffers are refilled only after the MMAs have read them.
-    if (!tc::mbar_wait(bar_mma, kc & 1, never, kWaitLimit)) ok = false;
-    tc::fence_after_sync();
-    if (!__syncthreads_and(ok)) {
-      ok = false;
-      mma_pending = kc & 1;
-      break;
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA
+    if (lane == 0) {
+      // TF32 inputs, fp32 accumulator, A (TMEM) and B K-major, M = N = 128.
+      constexpr uint32_t idesc = tc::instr_desc(2, 2, 0, 0, kRows, kRows);
+      long long m = 0, prev = -1;
+      int arow = 0, t = 0;
+      bool ok = true;
+      for (long long blk = blk0; ok && blk < blk1; ++blk, ++t) {
+        const long long rk = blk / nb;
+        if (rk != prev) {
+          if (!tc::mbar_wait(bar_asplit, arow & 1, abort_flag, kWaitLimit)) {
+            ok = false;
+            break;
+          }
+          ++arow;
+          prev = rk;
+        }
+        const int a = t & 1;
+        if (t >= 2 && !tc::mbar_wait(bar_accempty(a), ((t >> 1) - 1) & 1, abort_flag, kWaitLimit)) {
+          ok = false;
+          break;
+        }
+        tc::fence_after_sync();
+        const uint32_t d = tmem + C::COL_ACC + (uint32_t)(a * kRows);
+        for (int kc = 0; kc < C::KS; ++kc, ++m) {
+          const int s = (int)(m % kStages);
+          if (!tc::mbar_wait(bar_bsplit(s), (int)(m / kStages) & 1, abort_flag, kWaitLimit)) {
+            ok = false;
+            break;
+          }
+          tc::fence_after_sync();
+          const uint32_t stg = sb + C::OFF_RING + s * C::STAGE;
+#pragma unroll
+          for (int kk = 0; kk < kSlice / 8; ++kk) {  // 8 fp32 of K per MMA
+            const uint32_t ah = tmem + (uint32_t)(kc * kSlice + kk * 8), al = ah + C::COL_LO;
+            const uint64_t bhi = tc::smem_desc(stg + kk * 32, 16, 1024, tc::kLayoutSW128);
+            const uint64_t blo = tc::smem_desc(stg + kSliceBytes + kk * 32, 16, 1024, tc::kLayoutSW128);
+            mma_ts_tf32(d, ah, bhi, idesc, (kc > 0 || kk > 0) ? 1u : 0u);
+            mma_ts_tf32(d, ah, blo, idesc, 1u);
+            mma_ts_tf32(d, al, bhi, idesc, 1u);
+          }
+          tc::mma_commit(bar_bempty(s));
+        }
+        if (!ok) break;
+        tc::mma_commit(bar_accfull(a));
+        // Pq columns of TMEM are rewritten for the next row block only after
+        // this one's MMAs are done.
+        if (blk + 1 < blk1 && (blk + 1) / nb != rk) tc::mma_commit(bar_afree);
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        atomicOr(P.err, BSATTN_DEVERR_TIMEOUT);
+      }
+      tc::mma_commit(bar_final);  // drain every issued MMA before TMEM and shared memory go away
+      tc::mbar_wait(bar_final, 0, never, kWaitLimit);
     }
-  }
-  if (!ok) {
-    // Let the copies and MMAs already issued finish (bounded) before the
-    // shared memory and TMEM go away.
-    if (tid == 0) {
-      atomicOr(err, BSATTN_DEVERR_TIMEOUT);
-      if (ld_pending >= 0) tc::mbar_wait(bar_ld, ld_pending, never, kWaitLimit);
-      if (mma_pending >= 0) tc::mbar_wait(bar_mma, mma_pending, never, kWaitLimit);
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ split
+    const int t = tid - 128, r = t;  // thread t owns row r of the Pq block (TMEM lane r)
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    long long m = 0, prev = -1;
+    int arow = 0;
+    bool ok = true;
+    for (long long blk = blk0; ok && blk < blk1; ++blk) {
+      const long long rk = blk / nb;
+      if (rk != prev) {
+        if (!__all_sync(0xffffffffu, tc::mbar_wait(bar_afull, arow & 1, abort_flag, kWaitLimit)) ||
+            (arow > 0 && !__all_sync(0xffffffffu, tc::mbar_wait(bar_afree, (arow - 1) & 1, abort_flag, kWaitLimit)))) {
+          ok = false;
+          break;
+        }
+        tc::fence_after_sync();
+#pragma unroll 1
+        for (int kc = 0; kc < C::KS; ++kc) {
+          // Row r of a 128-byte-swizzled slice: 16-byte piece c sits at c ^ (r & 7).
+          const uint8_t* row = smem + C::OFF_ASTG + kc * kSliceBytes + r * 128;
+          uint32_t h[32], l[32];
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const float4 x = *reinterpret_cast<const float4*>(row + ((c ^ (r & 7)) << 4));
+            const float xv[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const uint32_t hb = hi_bits(__float_as_uint(xv[e]));
+              h[4 * c + e] = hb;
+              l[4 * c + e] = __float_as_uint(xv[e] - __uint_as_float(hb));
+            }
+          }
+          tc::tmem_st32(tmem + lane_base + (uint32_t)(kc * kSlice), h);
+          tc::tmem_st32(tmem + lane_base + C::COL_LO + (uint32_t)(kc * kSlice), l);
+        }
+        tc::tmem_wait_st();
+        tc::mbar_arrive(bar_astg);
+        tc::fence_before_sync();
+        tc::mbar_arrive(bar_asplit);
+        ++arow;
+        prev = rk;
+      }
+      for (int kc = 0; kc < C::KS; ++kc, ++m) {
+        const int s = (int)(m % kStages);
+        if (!__all_sync(0xffffffffu, tc::mbar_wait(bar_bfull(s), (int)(m / kStages) & 1, abort_flag, kWaitLimit))) {
+          ok = false;
+          break;
+        }
+        split_slice(smem + C::OFF_RING + s * C::STAGE, t);
+        tc::mbar_arrive(bar_bsplit(s));
+      }
+    }
+    if (!ok) {
+      *abort_flag = 1;
+      if (lane == 0) atomicOr(P.err, BSATTN_DEVERR_TIMEOUT);
     }
   } else {
-    // Row i0 + 32 warp + lane of the block, 32 columns at a time.
-    const int i = i0 + warp * 32 + lane;
-    float* row = S + ((size_t)bh * N + i) * N;
-    const bool vec = (N & 3) == 0;
-#pragma unroll
-    for (int c = 0; c < kRows; c += 32) {
-      uint32_t v[32];
-      tc::tmem_ld32_wait(tmem + ((uint32_t)(warp * 32) << 16) + c, v);
-      if (i >= N) continue;
-      const int j = j0 + c;
-      if (vec && j + 32 <= N) {
-#pragma unroll
-        for (int q = 0; q < 32; q += 4)
-          *reinterpret_cast<float4*>(row + j + q) =
-              make_float4(__uint_as_float(v[q]) * scale, __uint_as_float(v[q + 1]) * scale,
-                          __uint_as_float(v[q + 2]) * scale, __uint_as_float(v[q + 3]) * scale);
-      } else {
-#pragma unroll
-        for (int q = 0; q < 32; ++q)
-          if (j + q < N) row[j + q] = __uint_as_float(v[q]) * scale;
+    // ------------------------------------------------------------ epilogue
+    uint8_t* epi = smem + C::OFF_EPI + warp * kEpiBytes;  // 32 rows x 128 bytes, swizzled
+    int t = 0;
+    bool ok = true;
+    const bool vec = (P.N & 3) == 0;
+    for (long long blk = blk0; blk < blk1; ++blk, ++t) {
+      const int a = t & 1;
+      if (!__all_sync(0xffffffffu, tc::mbar_wait(bar_accfull(a), (t >> 1) & 1, abort_flag, kWaitLimit))) {
+        ok = false;
+        break;
       }
+      tc::fence_after_sync();
+      const long long rk = blk / nb, bh = rk / nb;
+      const int i0 = (int)(rk % nb) * kRows + warp * 32;  // first output row of this warp
+      const int j0 = (int)(blk % nb) * kRows;
+#pragma unroll 1
+      for (int c = 0; c < kRows; c += 32) {
+        uint32_t v[32];
+        tc::tmem_ld32_wait(tmem + ((uint32_t)(warp * 32) << 16) + C::COL_ACC + (uint32_t)(a * kRows + c), v);
+        // This lane's row, 32 columns, into the transpose buffer (piece q at q ^ (lane & 7)).
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          *reinterpret_cast<float4*>(epi + lane * 128 + ((q ^ (lane & 7)) << 4)) =
+              make_float4(__uint_as_float(v[4 * q]) * P.scale, __uint_as_float(v[4 * q + 1]) * P.scale,
+                          __uint_as_float(v[4 * q + 2]) * P.scale, __uint_as_float(v[4 * q + 3]) * P.scale);
+        __syncwarp();
+        // Four rows of 128 bytes per store instruction.
+        const int q = lane & 7, j = j0 + c + 4 * q;
+#pragma unroll
+        for (int it = 0; it < 8; ++it) {
+          const int rr = it * 4 + (lane >> 3), i = i0 + rr;
+          const float4 x = *reinterpret_cast<const float4*>(epi + rr * 128 + ((q ^ (rr & 7)) << 4));
+          if (i < P.N) {
+            float* dst = P.S + ((size_t)bh * P.N + (size_t)i) * P.N + j;
+            if (vec && j + 4 <= P.N) {
+              *reinterpret_cast<float4*>(dst) = x;
+            } else {
+              if (j < P.N) dst[0] = x.x;
+              if (j + 1 < P.N) dst[1] = x.y;
+              if (j + 2 < P.N) dst[2] = x.z;
+              if (j + 3 < P.N) dst[3] = x.w;
+            }
+          }
+        }
+        __syncwarp();
+      }
+      tc::fence_before_sync();
+      tc::mbar_arrive(bar_accempty(a));
+    }
+    if (!ok) {
+      *abort_flag = 1;
+      if (lane == 0) atomicOr(P.err, BSATTN_DEVERR_TIMEOUT);
     }
   }
+
   tc::fence_before_sync();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == 9) {
     tc::fence_after_sync();
-    tc::tmem_dealloc(tmem, kRows);
+    tc::tmem_dealloc(tmem, 512);
   }
 }
 
 template <int D>
 bsattn_status run_scores(const Geom& g, const float* pq, const float* pk, float scale, float* S, int* err,
                          cudaStream_t st) {
+  using C = ScoresCfg<D>;
   const uint64_t rows = (uint64_t)g.B * g.Hh * g.N;
   CUtensorMap ma, mb;
   if (!bsattn_make_map_2d(&ma, pq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, D, rows, kSlice, kRows,
@@ -163,11 +388,21 @@ bsattn_status run_scores(const Geom& g, const float* pq, const float* pk, float 
                           CU_TENSOR_MAP_SWIZZLE_128B))
     return BSATTN_ERR_CUDA;
   auto kern = block_scores_tc_kernel<D>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) != cudaSuccess)
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
     return BSATTN_ERR_CUDA;
-  const int nb = (g.N + kRows - 1) / kRows;
-  dim3 grid(nb, nb, g.B * g.Hh);
-  kern<<<grid, 128, kSmem, st>>>(ma, mb, g.N, scale, S, err);
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+    return BSATTN_ERR_CUDA;
+  ScoresParams prm;
+  prm.N = g.N;
+  prm.nb = (g.N + kRows - 1) / kRows;
+  prm.blocks = (long long)g.B * g.Hh * prm.nb * prm.nb;
+  prm.scale = scale;
+  prm.S = S;
+  prm.err = err;
+  const int grid = (int)(prm.blocks < sms ? prm.blocks : sms);
+  kern<<<grid, kThreads, C::SMEM, st>>>(ma, mb, prm);
   return cudaGetLastError() == cudaSuccess ? BSATTN_OK : BSATTN_ERR_CUDA;
 }
 
@@ -177,6 +412,7 @@ bsattn_status launch_block_scores(const Geom& g, const float* pq, const float* p
                                   float* S, int* err, cudaStream_t st) {
   // Row coordinates of the tensor maps (B * Hh * N rows, plus a block) stay in int32.
   if ((uint64_t)g.B * g.Hh * g.N + kRows >= (1ull << 31)) return BSATTN_ERR_UNSUPPORTED;
+  if (g.B <= 0 || g.Hh <= 0 || g.N <= 0) return BSATTN_OK;
   return g.D == 128 ? run_scores<128>(g, pq, pk, scale, S, err, st)
                     : run_scores<64>(g, pq, pk, scale, S, err, st);
 }
