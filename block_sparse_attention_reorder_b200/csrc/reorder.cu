@@ -58,15 +58,32 @@ __device__ __forceinline__ float block_max(float v, float* red) {
   return m;
 }
 
-// e4m3 codes of 8 values divided by `scale` (IEEE fp32 division), RNE, satfinite.
-__device__ __forceinline__ uint2 quant8(const float* f, float scale) {
+// x / scale as the e4m3 conversion sees it. The code is that of the IEEE
+// fp32 quotient fl(x / scale); the product p = x * rscale (rscale the
+// correctly rounded 1 / scale) is within 3 fp32 ulps of that quotient (two
+// roundings of 2^-24 relative each, plus the quotient's own half ulp), so it
+// rounds to the same e4m3 code unless it lies within a few ulps of an e4m3
+// rounding midpoint (fp32 mantissa bits 19..0 equal to 0x80000 for e4m3
+// normals) or in the e4m3 subnormal range (|p| < 2^-6); those rare values
+// take the exact division. Zero is exact either way.
+__device__ __forceinline__ float e4m3_quotient(float x, float scale, float rscale) {
+  const float p = x * rscale;
+  const uint32_t a = __float_as_uint(p) & 0x7fffffffu;
+  const uint32_t low = a & 0xFFFFFu;
+  const bool safe = a == 0u || (a >= 0x3C800000u && low + 4u - 0x80000u > 8u);
+  return safe ? p : __fdiv_rn(x, scale);
+}
+
+// e4m3 codes of 8 values divided by `scale` (as the IEEE fp32 division), RNE, satfinite.
+__device__ __forceinline__ uint2 quant8(const float* f, float scale, float rscale) {
   uint32_t w[2];
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     uint32_t acc = 0;
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
-      float2 x = make_float2(__fdiv_rn(f[4 * h + 2 * i], scale), __fdiv_rn(f[4 * h + 2 * i + 1], scale));
+      float2 x = make_float2(e4m3_quotient(f[4 * h + 2 * i], scale, rscale),
+                             e4m3_quotient(f[4 * h + 2 * i + 1], scale, rscale));
       __nv_fp8x2_storage_t p = __nv_cvt_float2_to_fp8x2(x, __NV_SATFINITE, __NV_E4M3);
       acc |= (uint32_t)p << (16 * i);
     }
@@ -123,13 +140,13 @@ reorder_kernel(Geom g, const __nv_bfloat16* __restrict__ x_nat, __nv_bfloat16* _
 #pragma unroll
       for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(f[e]));
     }
-    float scale = tile_scale_from_amax(block_max(m, wred));
+    const float scale = tile_scale_from_amax(block_max(m, wred)), rscale = __frcp_rn(scale);
 #pragma unroll
     for (int i = 0; i < ITER; ++i) {
       int r = r0 + RSTEP * i;
       float f[8];
       bf16x8_to_f32(v[i], f);
-      reinterpret_cast<uint2*>(codes + (tile_off + r) * D)[c] = quant8(f, scale);
+      reinterpret_cast<uint2*>(codes + (tile_off + r) * D)[c] = quant8(f, scale, rscale);
     }
     if (threadIdx.x == 0) scales[((size_t)b * g.Hh + head) * g.N + j] = scale;
   }
@@ -181,13 +198,13 @@ quant_tiled_kernel(Geom g, const __nv_bfloat16* __restrict__ x_tiled, uint8_t* _
 #pragma unroll
     for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(f[e]));
   }
-  float scale = tile_scale_from_amax(block_max(m, wred));
+  const float scale = tile_scale_from_amax(block_max(m, wred)), rscale = __frcp_rn(scale);
   uint2* dst = reinterpret_cast<uint2*>(codes + tile * 64 * D);
 #pragma unroll
   for (int i = 0; i < ITER; ++i) {
     float f[8];
     bf16x8_to_f32(v[i], f);
-    dst[threadIdx.x + kThreads * i] = quant8(f, scale);
+    dst[threadIdx.x + kThreads * i] = quant8(f, scale, rscale);
   }
   if (threadIdx.x == 0) scales[tile] = scale;
 }
@@ -230,7 +247,7 @@ quant_multi_kernel(Geom g, const __nv_bfloat16* __restrict__ src, __nv_bfloat16*
       for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(f[e]));
     }
   }
-  const float scale = tile_scale_from_amax(block_max(m, wred));
+  const float scale = tile_scale_from_amax(block_max(m, wred)), rscale = __frcp_rn(scale);
   for (int row0 = 0; row0 < g.V; row0 += 64) {
     uint4 v[ITER];
 #pragma unroll
@@ -241,7 +258,7 @@ quant_multi_kernel(Geom g, const __nv_bfloat16* __restrict__ src, __nv_bfloat16*
       if (NAT && x_tiled) reinterpret_cast<uint4*>(x_tiled + row * D)[c] = v[i];
       float f[8];
       bf16x8_to_f32(v[i], f);
-      reinterpret_cast<uint2*>(codes + row * D)[c] = quant8(f, scale);
+      reinterpret_cast<uint2*>(codes + row * D)[c] = quant8(f, scale, rscale);
     }
   }
   if (threadIdx.x == 0) scales[tile] = scale;

@@ -183,6 +183,58 @@ def test_quantize_e4m3_bytes(bs, name):
     np.testing.assert_array_equal(codes.cpu().numpy(), rc)
 
 
+def test_quantize_e4m3_every_bf16_magnitude(bs):
+    """Tiles holding every bf16 magnitude of the 32 binades up to the tile's
+    amax (both signs, zeros to fill the 64 x 128 tile), under 24 different
+    amax values: e4m3 codes byte-identical to the oracle's fp32-division
+    quantisation. Many of these quotients fall exactly on, or next to, e4m3
+    rounding midpoints (bf16 ratios have short binary expansions), and the
+    smallest ones in the e4m3 subnormal range and below it."""
+    T, H, W = 4, 4, 4 * 12  # 12 tiles of 64 tokens
+    heads = 2
+    plan = bs.Plan(1, heads, 128, T, H, W, rule="window", win=(0, 0, 1), qk_fp8=True)
+    rng = np.random.default_rng(5)
+    tiles = np.zeros((1, heads, plan.N, 64, 128), dtype=np.float32)
+    for h in range(heads):
+        for t in range(plan.N):
+            amax = np.float32(rng.uniform(0.5, 2.0) * 10.0 ** rng.uniform(-4, 4))
+            amax = (np.array([amax], np.float32).view(np.uint32) & 0xFFFF0000).view(np.float32)[0]  # bf16
+            e = int(np.frexp(amax)[1]) - 1
+            base = (np.float32(2.0) ** np.arange(e - 31, e + 1, dtype=np.float32)).view(np.uint32)
+            mags = (base[:, None] + (np.arange(128, dtype=np.uint32) << 16)[None, :]).reshape(-1).view(np.float32)
+            mags = mags[mags < amax]
+            vals = np.concatenate([[amax, -amax], mags, -mags])[:8192].astype(np.float32)
+            flat = np.zeros(8192, np.float32)
+            flat[:vals.size] = vals
+            tiles[0, h, t] = rng.permutation(flat).reshape(64, 128)
+    xt = torch.from_numpy(tiles).to(torch.bfloat16).cuda()
+    assert torch.equal(xt.float().cpu(), torch.from_numpy(tiles))  # every value is a bf16 value
+    codes = torch.empty(plan.tiled_shape(), dtype=torch.uint8, device="cuda")
+    scales = torch.empty((1, heads, plan.N), dtype=torch.float32, device="cuda")
+    bs.attn_quantize_e4m3(plan, xt, codes, scales)
+    rc, rs = e4m3.quantize_tiled(tiles)
+    np.testing.assert_array_equal(scales.cpu().numpy(), rs)
+    np.testing.assert_array_equal(codes.cpu().numpy(), rc)
+    # attn_layer quantises while it reorders (natural source): its output is
+    # bit-identical to attn_forward on the codes above.
+    x_nat = torch.from_numpy(tiling.unreorder(tiles, T, H, W, (4, 4, 4))).to(torch.bfloat16).cuda()
+    v_nat = torch.randn(x_nat.shape, generator=torch.Generator().manual_seed(3)).to(torch.bfloat16).cuda()
+    si, sc = plan.list_shapes()
+    idx = torch.empty(si, dtype=torch.int32, device="cuda")
+    cnt = torch.empty(sc, dtype=torch.int32, device="cuda")
+    bs.attn_select_from_scores(plan, None, idx, cnt)
+    o_layer = torch.empty_like(x_nat)
+    bs.attn_layer(plan, x_nat, x_nat, v_nat, o_layer, plan.workspace("layer"))
+    vt = torch.empty(plan.tiled_shape(), dtype=torch.bfloat16, device="cuda")
+    bs.attn_reorder(plan, v_nat, vt)
+    ot = torch.empty_like(vt)
+    bs.attn_forward(plan, codes, codes, vt, idx, cnt, ot, q_scale=scales, k_scale=scales)
+    o_chain = torch.empty_like(x_nat)
+    bs.attn_unreorder(plan, ot, o_chain)
+    assert bs.attn_check_device_status(plan) == 0
+    assert torch.equal(o_layer, o_chain)
+
+
 def _oracle_inputs(wl):
     q, k, v = make_qkv(wl, "cpu")
     return q, k, v, to64(q), to64(k), to64(v)
