@@ -115,10 +115,14 @@ def chunk_real_table(wl, plan):
 
 
 def group_axes(wl):
-    """(pair axis, unused) of the attention kernel's query-tile pairs."""
-    if wl.rule == "window" and wl.win[2] == 0:
-        return 0, 1
-    return 2, 0
+    """(pair axis, another axis) of the attention kernel's query-tile pairs:
+    t for top-k / top-p, the window's widest axis (t first on ties)."""
+    pa = 0
+    if wl.rule == "window":
+        for x in (1, 2):
+            if wl.win[x] > wl.win[pa]:
+                pa = x
+    return pa, 1 if pa != 1 else 0
 
 
 def group_accounting(wl, plan, idx: torch.Tensor, cnt: torch.Tensor):

@@ -5,7 +5,7 @@
 // and PV product is an M = 128 tcgen05.mma, and a step is one 64-key chunk.
 // Tiles of 64 tokens (one chunk): the block stacks two adjacent query tiles
 // i0, i1 of one (batch, head), next to each other along one axis of the tile
-// grid (w for top-k / top-p, t for a window that does not reach along w),
+// grid (t for top-k / top-p, the window's widest axis for a window),
 // and walks the union of their kept key-tile lists in ascending order; a key
 // tile kept by only one of the two gives zero probabilities to the other
 // tile's rows. Adjacent query tiles of a smooth video latent keep mostly the
@@ -743,10 +743,7 @@ bsattn_status launch_attention(const bsattn_plan* p, const void* q, const void* 
   prm.umax = p->nchunk == 1 ? (p->N < 2 * p->kmax ? p->N : 2 * p->kmax)
                             : (p->N < p->kmax ? p->N : p->kmax) * p->nchunk;
   prm.bm_words = (p->N + 31) / 32;
-  // Pairs along w for top-k / top-p (neighbouring query tiles keep similar
-  // key tiles); along t for a window that does not reach along w, whose
-  // w-neighbours share no key tile.
-  prm.pair_axis = (p->rule.kind == BSATTN_RULE_WINDOW && p->rule.win_w == 0) ? 0 : 2;
+  prm.pair_axis = pair_axis_of(p);
   const int nd[3] = {p->nT, p->nH, p->nW};
   for (int a = 0; a < 3; ++a) prm.pdim[a] = a == prm.pair_axis ? (nd[a] + 1) / 2 : nd[a];
   const bool fp8 = p->desc.qk_fp8 != 0, d128 = p->desc.head_dim == 128;

@@ -940,7 +940,7 @@ bsattn_status launch_backward_dq_tc(const bsattn_plan* p, const void* q, const v
   // Steps: the union of two kept lists (one list for tiles of several chunks), times the chunks.
   prm.umax = p->nchunk == 1 ? (p->N < 2 * p->kmax ? p->N : 2 * p->kmax) : (p->N < p->kmax ? p->N : p->kmax) * p->nchunk;
   prm.bm_words = (p->N + 31) / 32;
-  prm.pair_axis = (p->rule.kind == BSATTN_RULE_WINDOW && p->rule.win_w == 0) ? 0 : 2;
+  prm.pair_axis = pair_axis_of(p);
   const int nd[3] = {p->nT, p->nH, p->nW};
   for (int a = 0; a < 3; ++a) prm.pdim[a] = a == prm.pair_axis ? (nd[a] + 1) / 2 : nd[a];
   return p->desc.head_dim == 128 ? run_dq<128>(p, q, k, v, d_o, prm, st) : run_dq<64>(p, q, k, v, d_o, prm, st);
@@ -963,7 +963,7 @@ bsattn_status launch_backward_dkdv_tc(const bsattn_plan* p, const void* q, const
   // Steps: at most N query tiles in the union of two transposed lists, times their chunks.
   prm.umax = p->N * p->nchunk;
   prm.bm_words = (p->N + 31) / 32;
-  prm.pair_axis = (p->rule.kind == BSATTN_RULE_WINDOW && p->rule.win_w == 0) ? 0 : 2;
+  prm.pair_axis = pair_axis_of(p);
   const int nd[3] = {p->nT, p->nH, p->nW};
   for (int a = 0; a < 3; ++a) prm.pdim[a] = a == prm.pair_axis ? (nd[a] + 1) / 2 : nd[a];
   return p->desc.head_dim == 128 ? run_dkdv<128>(p, q, k, v, d_o, prm, st)
