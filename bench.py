@@ -89,6 +89,22 @@ def workload_of(args):
     return dataclasses.replace(wl, heads=args.heads) if args.heads > 0 else wl
 
 
+def max_over_ranks(value: float, dist=None, device="cuda") -> float:
+    """The largest of one per-rank number over all ranks (a job's time is
+    its slowest rank's); the number itself with one rank."""
+    if not dist:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(world: int, flops_per_rank: float, ms_per_step: float) -> float:
+    """Whole-job throughput under weak scaling: every rank does
+    `flops_per_rank` per step, the step takes the slowest rank's time."""
+    return world * flops_per_rank / (ms_per_step * 1e-3) / 1e12
+
+
 def kept_pairs_from_counts(cnt: torch.Tensor) -> int:
     return int(cnt.to(torch.int64).sum().item())
 
@@ -405,11 +421,7 @@ def main():
         dist.barrier()
     torch.cuda.synchronize()
     clocks = sampler.stop() if sampler else None
-    total_ms = sum(a.elapsed_time(b) for a, b in ev)
-    if dist:
-        t = torch.tensor([total_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev), dist)
     ms_per_step = total_ms / args.steps
 
     # Per-kernel breakdown: the same layer as its C-ABI components, with
@@ -439,7 +451,7 @@ def main():
     achieved_mma = issued * pair_flops(wl.head_dim) / (attn_ms * 1e-3) / 1e12
     line = {
         "metric": METRIC,
-        "value": world * flops / (ms_per_step * 1e-3) / 1e12,
+        "value": job_tflops(world, flops, ms_per_step),
         "unit": "TFLOP/s",
         "n_gpus": world,
         "steps": args.steps,
@@ -670,16 +682,11 @@ def e2e_timing(bsattn, plan, q, k, v, ws, idx, cnt, stream, steps=10, warmup=3, 
     run(warmup)
     if dist:
         dist.barrier()
-    ms = run(steps) / steps
-    world = 1
-    if dist:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-        world = dist.get_world_size()
+    ms = max_over_ranks(run(steps) / steps, dist)
+    world = dist.get_world_size() if dist else 1
     h2d = sum(x.numel() * x.element_size() for x in hq)
     d2h = ho[0].numel() * ho[0].element_size()
-    return {"value": world * flops_per / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+    return {"value": job_tflops(world, flops_per, ms), "unit": "TFLOP/s",
             "ms_per_step": ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "note": "pinned host copies in and out every step, overlapped with the neighbouring steps' layers"}
 
