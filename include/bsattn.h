@@ -175,7 +175,7 @@ bsattn_status attn_select(const bsattn_plan* plan, const void* q_nat, const void
 /* Capacity of the library-owned scratch used by attn_select_static. */
 #define BSATTN_STATIC_SELECT_SCRATCH_BYTES (16u << 20)
 
-/* attn_select without a caller workspace (the paper has no counterpart; this
+/* attn_select without a caller workspace (the method itself has no counterpart; this
  * is a convenience of this library). For callers that cannot allocate device
  * memory themselves, e.g. code that runs where cudaMalloc is not allowed or
  * whose allocator is owned by someone else. The pooled Q/K and the score
