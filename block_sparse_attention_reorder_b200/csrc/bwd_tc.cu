@@ -6,8 +6,8 @@
 //   P_ij = 2^(scale log2(e) Q_i K_j^T - lse_i log2(e)),  Delta = rowsum(dO * O).
 //
 // Work unit, as in the forward kernel: a 128-row block of two 64-row chunks.
-// With 64-token tiles, two adjacent query tiles (w for top-k and top-p, t for
-// a window without w reach) walking the union of their kept lists (a key tile
+// With 64-token tiles, two adjacent query tiles (along t for top-k and top-p,
+// the window's widest axis for a window) walking the union of their kept lists (a key tile
 // kept by only one of the two gives zero dS to the other's rows); with tiles
 // of several chunks, chunks 2b and 2b + 1 of one query tile walking every
 // real chunk of each kept key tile.
