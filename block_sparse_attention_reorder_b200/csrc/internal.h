@@ -63,6 +63,39 @@ static inline Geom make_geom(const bsattn_plan* p) {
 
 static inline bool aligned16(const void* ptr) { return (((uintptr_t)ptr) & 15u) == 0; }
 
+// Makes `device` current for the lifetime of the object and gives the caller
+// its own current device back when the object goes out of scope, so that no
+// entry point changes the calling thread's current device. `status` is
+// BSATTN_ERR_CUDA when either runtime call failed (then nothing is switched).
+struct DeviceGuard {
+  int prev = -1;
+  bool switched = false;
+  bsattn_status status = BSATTN_OK;
+  explicit DeviceGuard(int device) {
+    if (cudaGetDevice(&prev) != cudaSuccess) {
+      status = BSATTN_ERR_CUDA;
+      return;
+    }
+    if (prev != device) {
+      if (cudaSetDevice(device) != cudaSuccess) {
+        status = BSATTN_ERR_CUDA;
+        return;
+      }
+      switched = true;
+    }
+  }
+  ~DeviceGuard() {
+    if (switched) cudaSetDevice(prev);
+  }
+  DeviceGuard(const DeviceGuard&) = delete;
+  DeviceGuard& operator=(const DeviceGuard&) = delete;
+};
+
+// Looks up, with `device` current, the device address of the library-owned
+// scratch array of attn_select_static and caches it; the lookup loads the
+// module that holds the array (reserving its memory on that device).
+bsattn_status bsattn_static_scratch_prepare(int device);
+
 #define BSATTN_CUDA_TRY(expr)                         \
   do {                                                \
     cudaError_t e_ = (expr);                          \

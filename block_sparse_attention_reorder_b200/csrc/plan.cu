@@ -91,12 +91,6 @@ BackwardWs carve_backward(const bsattn_plan* p, Carve& c) {
 
 bool ok_ptr(const void* x) { return x != nullptr && aligned16(x); }
 
-bsattn_status set_device(const bsattn_plan* p) {
-  int cur = -1;
-  BSATTN_CUDA_TRY(cudaGetDevice(&cur));
-  if (cur != p->device) BSATTN_CUDA_TRY(cudaSetDevice(p->device));
-  return BSATTN_OK;
-}
 
 }  // namespace
 
@@ -199,6 +193,10 @@ bsattn_status attn_plan_create(const bsattn_desc* d, const bsattn_rule* r, bsatt
     attn_plan_destroy(p);
     return BSATTN_ERR_CUDA;
   }
+  // Load attn_select_static's scratch array here, where the caller can
+  // allocate, so that the selection call itself reserves nothing. A failure
+  // is not the plan's: attn_select_static retries and reports it.
+  bsattn_static_scratch_prepare(p->device);
   if (r->kind == BSATTN_RULE_WINDOW) {
     // Closed-form clipped window lists, ascending because j grows with
     // (t, h, w) in row-major tile order.
@@ -268,8 +266,9 @@ bsattn_status attn_reorder(const bsattn_plan* p, const void* x_nat, void* x_tile
                            void* stream) {
   if (!p || !ok_ptr(x_nat) || !ok_ptr(x_tiled) || (pooled && !aligned16(pooled)))
     return BSATTN_ERR_INVALID_ARG;
-  bsattn_status s = set_device(p);
-  if (s) return s;
+  DeviceGuard dev(p->device);
+  if (dev.status) return dev.status;
+  bsattn_status s = BSATTN_OK;
   Geom g = make_geom(p);
   if ((s = launch_reorder(g, (const __nv_bfloat16*)x_nat, (__nv_bfloat16*)x_tiled, nullptr, nullptr,
                           RO_WRITE_TILED, (cudaStream_t)stream)))
@@ -280,8 +279,9 @@ bsattn_status attn_reorder(const bsattn_plan* p, const void* x_nat, void* x_tile
 
 bsattn_status attn_pool(const bsattn_plan* p, const void* x_nat, float* pooled, void* stream) {
   if (!p || !ok_ptr(x_nat) || !ok_ptr(pooled)) return BSATTN_ERR_INVALID_ARG;
-  bsattn_status s = set_device(p);
-  if (s) return s;
+  DeviceGuard dev(p->device);
+  if (dev.status) return dev.status;
+  bsattn_status s = BSATTN_OK;
   return launch_pool(make_geom(p), (const __nv_bfloat16*)x_nat, pooled, nullptr, nullptr,
                      (cudaStream_t)stream);
 }
@@ -289,8 +289,9 @@ bsattn_status attn_pool(const bsattn_plan* p, const void* x_nat, float* pooled, 
 bsattn_status attn_unreorder(const bsattn_plan* p, const void* x_tiled, void* x_nat,
                              void* stream) {
   if (!p || !ok_ptr(x_tiled) || !ok_ptr(x_nat)) return BSATTN_ERR_INVALID_ARG;
-  bsattn_status s = set_device(p);
-  if (s) return s;
+  DeviceGuard dev(p->device);
+  if (dev.status) return dev.status;
+  bsattn_status s = BSATTN_OK;
   return launch_unreorder(make_geom(p), (const __nv_bfloat16*)x_tiled, (__nv_bfloat16*)x_nat,
                           nullptr, nullptr, (cudaStream_t)stream);
 }
@@ -298,8 +299,9 @@ bsattn_status attn_unreorder(const bsattn_plan* p, const void* x_tiled, void* x_
 bsattn_status attn_block_scores(const bsattn_plan* p, const float* pq, const float* pk,
                                 float* S, void* stream) {
   if (!p || !ok_ptr(pq) || !ok_ptr(pk) || !ok_ptr(S)) return BSATTN_ERR_INVALID_ARG;
-  bsattn_status s = set_device(p);
-  if (s) return s;
+  DeviceGuard dev(p->device);
+  if (dev.status) return dev.status;
+  bsattn_status s = BSATTN_OK;
   return launch_block_scores(make_geom(p), pq, pk, p->scale, S, p->d_err, (cudaStream_t)stream);
 }
 
@@ -321,8 +323,9 @@ bsattn_status attn_select_from_scores(const bsattn_plan* p, const float* S, int3
                                       int32_t* cnt, void* stream) {
   if (!p || !ok_ptr(idx) || !ok_ptr(cnt)) return BSATTN_ERR_INVALID_ARG;
   if (p->rule.kind != BSATTN_RULE_WINDOW && !ok_ptr(S)) return BSATTN_ERR_INVALID_ARG;
-  bsattn_status s = set_device(p);
-  if (s) return s;
+  DeviceGuard dev(p->device);
+  if (dev.status) return dev.status;
+  bsattn_status s = BSATTN_OK;
   return select_core(p, S, idx, cnt, (cudaStream_t)stream);
 }
 
@@ -332,8 +335,9 @@ bsattn_status attn_select(const bsattn_plan* p, const void* q_nat, const void* k
   bsattn_info info;
   attn_plan_info(p, &info);
   cudaStream_t st = (cudaStream_t)stream;
-  bsattn_status s = set_device(p);
-  if (s) return s;
+  DeviceGuard dev(p->device);
+  if (dev.status) return dev.status;
+  bsattn_status s = BSATTN_OK;
   if (p->rule.kind == BSATTN_RULE_WINDOW) return select_core(p, nullptr, idx, cnt, st);
   if (!ok_ptr(q_nat) || !ok_ptr(k_nat)) return BSATTN_ERR_INVALID_ARG;
   if (!ws || !aligned16(ws) || ws_bytes < info.select_workspace_bytes) return BSATTN_ERR_WORKSPACE;
@@ -348,8 +352,9 @@ bsattn_status attn_select(const bsattn_plan* p, const void* q_nat, const void* k
 bsattn_status attn_quantize_e4m3(const bsattn_plan* p, const void* x_tiled, uint8_t* codes,
                                  float* scales, void* stream) {
   if (!p || !ok_ptr(x_tiled) || !ok_ptr(codes) || !ok_ptr(scales)) return BSATTN_ERR_INVALID_ARG;
-  bsattn_status s = set_device(p);
-  if (s) return s;
+  DeviceGuard dev(p->device);
+  if (dev.status) return dev.status;
+  bsattn_status s = BSATTN_OK;
   return launch_quant_tiled(make_geom(p), (const __nv_bfloat16*)x_tiled, codes, scales,
                             (cudaStream_t)stream);
 }
@@ -363,8 +368,9 @@ bsattn_status attn_forward(const bsattn_plan* p, const void* q, const void* k, c
   if (p->desc.qk_fp8 && (!ok_ptr(qs) || !ok_ptr(ks))) return BSATTN_ERR_INVALID_ARG;
   size_t need = attention_workspace_bytes(p);
   if (need && (!ws || !aligned16(ws) || ws_bytes < need)) return BSATTN_ERR_WORKSPACE;
-  bsattn_status s = set_device(p);
-  if (s) return s;
+  DeviceGuard dev(p->device);
+  if (dev.status) return dev.status;
+  bsattn_status s = BSATTN_OK;
   return launch_attention(p, q, k, qs, ks, (const __nv_bfloat16*)v, idx, cnt, (__nv_bfloat16*)o,
                           lse, ws, ws_bytes, (cudaStream_t)stream, AttnLayout::Tiled);
 }
@@ -379,8 +385,9 @@ bsattn_status attn_backward(const bsattn_plan* p, const void* q, const void* k, 
   bsattn_info info;
   attn_plan_info(p, &info);
   if (!ws || !aligned16(ws) || ws_bytes < info.backward_workspace_bytes) return BSATTN_ERR_WORKSPACE;
-  bsattn_status s = set_device(p);
-  if (s) return s;
+  DeviceGuard dev(p->device);
+  if (dev.status) return dev.status;
+  bsattn_status s = BSATTN_OK;
   Carve c(ws);
   const BackwardWs w = carve_backward(p, c);
   return launch_backward(p, q, k, v, o, d_o, lse, idx, cnt, dq, dk, dv, w, (cudaStream_t)stream);
@@ -396,8 +403,9 @@ bsattn_status attn_forward_natural(const bsattn_plan* p, const void* q, const vo
   if (p->desc.qk_fp8 && (!ok_ptr(qs) || !ok_ptr(ks))) return BSATTN_ERR_INVALID_ARG;
   size_t need = attention_workspace_bytes(p);
   if (need && (!ws || !aligned16(ws) || ws_bytes < need)) return BSATTN_ERR_WORKSPACE;
-  bsattn_status s = set_device(p);
-  if (s) return s;
+  DeviceGuard dev(p->device);
+  if (dev.status) return dev.status;
+  bsattn_status s = BSATTN_OK;
   return launch_attention(p, q, k, qs, ks, (const __nv_bfloat16*)v_nat, idx, cnt, (__nv_bfloat16*)o_nat,
                           lse_nat, ws, ws_bytes, (cudaStream_t)stream, AttnLayout::Natural);
 }
@@ -412,8 +420,9 @@ bsattn_status attn_layer(const bsattn_plan* p, const void* q_nat, const void* k_
   bsattn_info info;
   attn_plan_info(p, &info);
   if (!ws || !aligned16(ws) || ws_bytes < info.layer_workspace_bytes) return BSATTN_ERR_WORKSPACE;
-  bsattn_status s = set_device(p);
-  if (s) return s;
+  DeviceGuard dev(p->device);
+  if (dev.status) return dev.status;
+  bsattn_status s = BSATTN_OK;
   cudaStream_t st = (cudaStream_t)stream;
   Carve c(ws);
   LayerWs w = carve_layer(p, c);
@@ -453,8 +462,9 @@ bsattn_status attn_layer(const bsattn_plan* p, const void* q_nat, const void* k_
 
 bsattn_status attn_check_device_status(const bsattn_plan* p, void* stream) {
   if (!p) return BSATTN_ERR_INVALID_ARG;
-  bsattn_status s = set_device(p);
-  if (s) return s;
+  DeviceGuard dev(p->device);
+  if (dev.status) return dev.status;
+  bsattn_status s = BSATTN_OK;
   BSATTN_CUDA_TRY(cudaStreamSynchronize((cudaStream_t)stream));
   int h = 0;
   BSATTN_CUDA_TRY(cudaMemcpy(&h, p->d_err, sizeof(int), cudaMemcpyDeviceToHost));

@@ -30,9 +30,10 @@
  *     word and the affected work is skipped; attn_check_device_status
  *     reports it.
  *   - A plan is bound to the device that was current at attn_plan_create
- *     and is immutable afterwards, so it may be used from several streams
- *     at once (calls that share output buffers must still be ordered by the
- *     caller).
+ *     (calls switch to that device while they run and give the caller its
+ *     own current device back before returning) and is immutable
+ *     afterwards, so it may be used from several streams at once (calls
+ *     that share output buffers must still be ordered by the caller).
  *   - Block scores containing NaN give unspecified (but in-bounds) lists.
  *
  * Layouts (B batch, Hh heads, D head_dim, L = T*H*W, N = number of tiles,
@@ -149,7 +150,11 @@ bsattn_status attn_unreorder(const bsattn_plan* plan, const void* x_tiled, void*
                              void* stream);
 
 /* Step 2: block scores S = softmax_scale * pooled_q . pooled_k^T per
- * (batch, head), fp32 out. Computed on the tensor cores as three TF32
+ * (batch, head), fp32 out. The routing frontend of the FVAttn summary page
+ * (Summary and Abstract: Top-p routing with a Top-k safety floor over
+ * video-aware blocks) ranks key blocks per query block; the pages do not
+ * print the block score, and this library's reading is the scaled dot
+ * product of the tiles' mean Q and mean K. Computed on the tensor cores as three TF32
  * products per term (each input split as hi + lo, hi exact in TF32; hi*hi +
  * hi*lo + lo*hi accumulated in fp32), within about 2^-20 of
  * sum_d |q_d k_d| of the exact dot product; the result is deterministic. A
@@ -157,7 +162,12 @@ bsattn_status attn_unreorder(const bsattn_plan* plan, const void* x_tiled, void*
 bsattn_status attn_block_scores(const bsattn_plan* plan, const float* pooled_q,
                                 const float* pooled_k, float* scores, void* stream);
 
-/* Step 3 on a given score matrix: the plan's rule applied row by row.
+/* Step 3 on a given score matrix: the plan's rule applied row by row
+ * (top-p with a top-k floor: FVAttn summary page, Summary and Abstract;
+ * top-k at a fixed density: "Faster Video Diffusion with Trainable Sparse
+ * Attention" record, Dataset Splits row, final sparsity 0.9; the window:
+ * FPSAttention page, ablation rows on the (6,6,1), (6,6,6) and (3,3,1)
+ * sparsity windows).
  * Top-k: the k largest by (score descending, index ascending); -0.0 and
  * +0.0 tie. Top-p: in that order, the shortest prefix whose softmax mass
  * (fp64 exp, sum and scan) reaches p, then at least k and at most N tiles.
@@ -166,8 +176,11 @@ bsattn_status attn_block_scores(const bsattn_plan* plan, const float* pooled_q,
 bsattn_status attn_select_from_scores(const bsattn_plan* plan, const float* scores,
                                       int32_t* idx, int32_t* cnt, void* stream);
 
-/* Steps 2-3 from natural Q and K: pool, score, select. `ws` must hold
- * info.select_workspace_bytes (pooled Q/K and the score matrix). */
+/* Steps 2-3 from natural Q and K: pool, score, select (the routing
+ * frontend of the FVAttn summary page, Summary: video-aware blocks, Top-p
+ * routing, Top-k floor; see attn_block_scores and attn_select_from_scores
+ * for the readings). `ws` must hold info.select_workspace_bytes (pooled Q/K
+ * and the score matrix); the window rule reads neither q/k nor ws. */
 bsattn_status attn_select(const bsattn_plan* plan, const void* q_nat, const void* k_nat,
                           int32_t* idx, int32_t* cnt, void* ws, size_t ws_bytes,
                           void* stream);
@@ -180,11 +193,13 @@ bsattn_status attn_select(const bsattn_plan* plan, const void* q_nat, const void
  * memory themselves, e.g. code that runs where cudaMalloc is not allowed or
  * whose allocator is owned by someone else. The pooled Q/K and the score
  * matrix live in one static device array of
- * BSATTN_STATIC_SELECT_SCRATCH_BYTES bytes that every GPU loading the library
- * holds until the process exits. The call itself allocates nothing.
- * - The first call on a device looks the array's device address up (once per
- *   device, with that device current); make that first call before any
- *   stream capture.
+ * BSATTN_STATIC_SELECT_SCRATCH_BYTES bytes. The call itself allocates nothing.
+ * - The array is reserved on a device when attn_plan_create first runs there
+ *   (it looks the array's device address up, once per device, with that
+ *   device current, which loads the library module holding it); the device
+ *   then holds it until the process exits. attn_plan_create does not fail if
+ *   that memory is not available; attn_select_static then tries the lookup
+ *   again and returns BSATTN_ERR_CUDA if it still fails.
  * - Problems whose select workspace (info.select_workspace_bytes) exceeds the
  *   capacity are rejected with BSATTN_ERR_UNSUPPORTED; the window rule needs
  *   no scratch.
@@ -196,9 +211,12 @@ bsattn_status attn_select(const bsattn_plan* plan, const void* q_nat, const void
 bsattn_status attn_select_static(const bsattn_plan* plan, const void* q_nat, const void* k_nat,
                                  int32_t* idx, int32_t* cnt, void* stream);
 
-/* Per-tile e4m3 quantisation of a tiled bf16 tensor: per (b, head, tile)
- * scale = fp32(amax)/448 (amax 0 -> 1), code = e4m3(x/scale) rounded to
- * nearest even with finite saturation (OCP E4M3). */
+/* Per-tile e4m3 quantisation of a tiled bf16 tensor (FPSAttention page,
+ * Approach: FP8 quantisation and block sparsity share one 3D tile
+ * granularity): per (b, head, tile) scale = fp32(amax)/448 (amax 0 -> 1),
+ * code = e4m3(x/scale) rounded to nearest even with finite saturation (OCP
+ * E4M3; the page names FP8 without the format, this is the library's
+ * reading). */
 bsattn_status attn_quantize_e4m3(const bsattn_plan* plan, const void* x_tiled,
                                  uint8_t* codes, float* scales, void* stream);
 

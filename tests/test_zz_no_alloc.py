@@ -35,7 +35,7 @@ def _lists(bs, plan, fn, q, k):
     return lists_from_device(idx, cnt)
 
 
-@pytest.mark.parametrize("name", ["wan1.3b", "tiny", "ragged_topp", "ragged_topk"])
+@pytest.mark.parametrize("name", ["wan1.3b", "tiny", "ragged_topp", "ragged_topk", "ragged_bf16_window"])
 def test_static_scratch_matches_workspace_version_twice(bs, name):
     wl = WORKLOADS.get(name) or SMALL[name]
     plan = bs.Plan.for_workload(wl)
