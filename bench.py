@@ -5,7 +5,10 @@ and K (e4m3 tile codes with fused pooling on the FP8 workload), block
 scores, key-tile selection, and the block-sparse attention, which reads Q, K,
 V tile by tile from the natural layout and writes natural O. Inputs are seeded
 synthetic video-latent Q/K/V already resident in HBM; L2 is flushed between
-timed steps. Prints one JSON line (rank 0).
+timed steps. The headline workload is the Wan2.1-14B-shaped 720p layer
+(40 heads, 21x45x80 latent grid, top-k at sparsity 0.9); the other
+workloads (top-p, e4m3 window, Wan2.1-1.3B, tiny) follow as sub-records under
+"configs". Prints one JSON line (rank 0).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
   python bench.py --impl reference ...   # the fp64 CPU oracle on host cores
@@ -34,7 +37,9 @@ sys.path.insert(0, ROOT)
 from block_sparse_attention_reorder_b200.datagen import WORKLOADS, make_qkv  # noqa: E402
 
 METRIC = "sparse attn fwd ms/layer & achieved TFLOP/s on kept blocks vs B200 BF16 peak"
-DEFAULT_WORKLOAD = "wan1.3b"
+DEFAULT_WORKLOAD = "wan14b"
+# Other workloads timed after the headline, one sub-record each.
+OTHER_WORKLOADS = ("topp", "window_fp8", "wan1.3b", "tiny")
 L2_FLUSH_BYTES = 256 << 20
 
 
@@ -50,6 +55,8 @@ def parse():
     ap.add_argument("--no-backward", action="store_true", help="skip the backward-pass timing")
     ap.add_argument("--heads", type=int, default=0,
                     help="run a copy of the workload with this many heads (small profiling cases)")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the sub-records of the other workloads")
     return ap.parse_args()
 
 
@@ -192,6 +199,32 @@ def group_accounting(wl, plan, idx: torch.Tensor, cnt: torch.Tensor):
 
     pairs = fold(hit, pa)
     return int(pairs.sum().item()) * 2, int(pairs.sum().item())
+
+
+def tile_valid_counts(wl, plan):
+    """[N] int64: real (unpadded) tokens in each tile."""
+    import numpy as np
+
+    info = plan.info
+    tt, th, tw = wl.tile
+    j = np.arange(plan.N)
+    t0 = (j // (info.nH * info.nW)) * tt
+    h0 = ((j // info.nW) % info.nH) * th
+    w0 = (j % info.nW) * tw
+    return (np.clip(wl.T - t0, 0, tt) * np.clip(wl.H - h0, 0, th) * np.clip(wl.W - w0, 0, tw)).astype(np.int64)
+
+
+def valid_token_flops(wl, plan, idx: torch.Tensor, cnt: torch.Tensor) -> float:
+    """FLOP of the kept tile pairs counting real query x real key token
+    products only: sum over kept (i, j) of 4 * D * n_i * n_j, n = real tokens
+    of a tile (padding rows and padded keys of edge tiles not counted)."""
+    nv = torch.from_numpy(tile_valid_counts(wl, plan)).to(idx.device)
+    rows, kmax = cnt.numel(), idx.shape[-1]
+    ii = idx.reshape(rows, kmax).to(torch.int64).clamp(0, plan.N - 1)
+    keep = torch.arange(kmax, device=idx.device)[None, :] < cnt.reshape(rows, 1)
+    keys = (nv[ii] * keep).sum(dim=1)
+    own = nv.repeat(rows // plan.N)
+    return float(4.0 * wl.head_dim * (own * keys).sum().item())
 
 
 def layer_tiles_kv(plan) -> bool:
@@ -399,6 +432,7 @@ def main():
         raise SystemExit("device error word set")
     kept = kept_pairs_from_counts(cnt)
     flops = kept * pair_flops(wl.head_dim, plan.V)
+    vflops = valid_token_flops(wl, plan, idx, cnt)
     issued, loads = group_accounting(wl, plan, idx, cnt)
 
     sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
@@ -443,6 +477,12 @@ def main():
     pk = peaks()
     # The backward of the same layer (rank 0; not part of the timed step).
     bwd = None if args.no_backward else backward_timing(bsattn, plan, wl, q, k, v, idx, cnt, flush, stream, pk)
+    configs = None
+    if not args.no_configs and args.heads == 0:
+        del q, k, v, o, ws
+        torch.cuda.empty_cache()
+        configs = {n: config_record(bsattn, WORKLOADS[n], flush, stream, pk)
+                   for n in OTHER_WORKLOADS if n != wl.name}
     attn_ms = comp["attention"]
     achieved = flops / (attn_ms * 1e-3) / 1e12
     nch2 = (plan.V // 64) ** 2  # 64 x 64 chunk pairs per kept tile pair
@@ -463,6 +503,7 @@ def main():
         "dtype": "bf16+e4m3" if wl.qk_fp8 else "bf16",
         "data": "synthetic",
         "config": workload_config(wl, {"kept_pairs": kept, "kept_tflop": flops / 1e12,
+                                        "valid_token_tflop": vflops / 1e12,
                                         "mma_chunk_pairs": issued,
                                         "pair_efficiency": kept * nch2 / issued if issued else None,
                                         "kv_chunk_loads": loads,
@@ -474,10 +515,13 @@ def main():
                      "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": achieved / pk["bf16_tflops"],
                      "achieved_mma": achieved_mma,
+                     "achieved_valid_tokens": vflops / (attn_ms * 1e-3) / 1e12,
+                     "valid_token_note": "kept tile pairs counting real query x real key products only",
                      "peak_note": f"{pk['source']} bf16 burst (kernel timed alone)",
                      "traffic": measured_traffic(wl.name) if args.heads == 0 else None},
         "memory_kernels": memory_kernel_rates(wl, plan, comp, pk),
         "backward": bwd,
+        "configs": configs,
         "e2e": e2e,
         "gpu_launches": launches_per_step(wl, plan) * args.steps,
         "clocks": clocks,
@@ -490,6 +534,66 @@ def main():
     if dist:
         dist.destroy_process_group()
     return 0
+
+
+def config_record(bsattn, wl, flush, stream, pk):
+    """One other workload, timed like the headline on the same GPU (inputs
+    resident, L2 flushed between steps, CUDA events on the launching
+    stream): ms/layer, the attention kernel's TFLOP/s on kept tile pairs and
+    on real-token products, both as fractions of the bf16 peak, and the
+    memory-bound kernels' algorithmic GB/s."""
+    plan = bsattn.Plan.for_workload(wl)
+    q, k, v = make_qkv(wl, "cuda")
+    o = torch.empty_like(q)
+    ws = plan.workspace("layer")
+    si, sc = plan.list_shapes()
+    idx = torch.empty(si, dtype=torch.int32, device="cuda")
+    cnt = torch.empty(sc, dtype=torch.int32, device="cuda")
+
+    def step():
+        bsattn.attn_layer(plan, q, k, v, o, ws, idx=idx, cnt=cnt, stream=stream)
+
+    step()
+    torch.cuda.synchronize()
+    if bsattn.attn_check_device_status(plan) != 0:
+        raise SystemExit(f"device error word set ({wl.name})")
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    steps = int(min(50, max(5, 1000.0 / max(a.elapsed_time(b), 1e-3))))
+    for _ in range(3):
+        flush.fill_(1.0)
+        step()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for s_ in range(steps):
+        flush.fill_(float(s_))
+        ev[s_][0].record(stream)
+        step()
+        ev[s_][1].record(stream)
+    torch.cuda.synchronize()
+    ms = sum(x.elapsed_time(y) for x, y in ev) / steps
+    kept = kept_pairs_from_counts(cnt)
+    flops = kept * pair_flops(wl.head_dim, plan.V)
+    vflops = valid_token_flops(wl, plan, idx, cnt)
+    comp = component_timing(bsattn, plan, wl, q, k, v, flush, stream, reps=min(steps, 10))
+    attn = comp["attention"]
+    rec = {"config": workload_config(wl, {"kept_pairs": kept, "kept_tflop": flops / 1e12,
+                                          "valid_token_tflop": vflops / 1e12}),
+           "steps": steps, "warmup": 3, "ms_per_layer": ms,
+           "tflops_kept_layer": flops / (ms * 1e-3) / 1e12,
+           "attention_ms": attn,
+           "attention_tflops_kept": flops / (attn * 1e-3) / 1e12,
+           "attention_frac_kept": flops / (attn * 1e-3) / 1e12 / pk["bf16_tflops"],
+           "attention_tflops_valid_tokens": vflops / (attn * 1e-3) / 1e12,
+           "attention_frac_valid_tokens": vflops / (attn * 1e-3) / 1e12 / pk["bf16_tflops"],
+           "kernels_ms": comp,
+           "memory_kernels": memory_kernel_rates(wl, plan, comp, pk)}
+    del q, k, v, o, ws
+    plan.close()
+    torch.cuda.empty_cache()
+    return rec
 
 
 def component_timing(bsattn, plan, wl, q, k, v, flush, stream, reps=20):

@@ -83,3 +83,35 @@ def test_traffic_record_matches_the_kernel_source_or_reads_as_missing(tmp_path, 
     (tmp_path / "attn_tc_changed.cu").write_text("// another kernel\n")
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     assert bench.measured_traffic("wan1.3b") is None
+
+
+@pytest.mark.parametrize("grid,tile", [((7, 10, 13), (4, 4, 4)), ((9, 12, 13), (6, 8, 8)),
+                                       ((8, 8, 8), (4, 4, 4))])
+def test_valid_token_flops_counts_real_token_products(grid, tile):
+    """The real-token figure, against a per-token count: for every kept tile
+    pair, the number of (real query, real key) token pairs times 4 D."""
+    from oracle import tiling
+
+    T, H, W = grid
+    nT, nH, nW = (-(-n // t) for n, t in zip(grid, tile))
+    N, heads, kmax, D = nT * nH * nW, 2, 5, 128
+    rng = np.random.default_rng(3)
+    lists = [[np.sort(rng.choice(N, size=rng.integers(0, kmax + 1), replace=False)) for _ in range(N)]
+             for _ in range(heads)]
+    idx = torch.full((1, heads, N, kmax), -1, dtype=torch.int32)
+    cnt = torch.zeros((1, heads, N), dtype=torch.int32)
+    for h in range(heads):
+        for i in range(N):
+            idx[0, h, i, :len(lists[h][i])] = torch.from_numpy(lists[h][i].astype(np.int32))
+            cnt[0, h, i] = len(lists[h][i])
+    # Real tokens per tile from the oracle's token -> tile map.
+    tok_tile, _ = tiling.token_tile_and_row(T, H, W, tile)
+    real = np.bincount(tok_tile, minlength=N)
+    want = sum(4 * D * real[i] * real[j] for h in range(heads) for i in range(N) for j in lists[h][i])
+    wl = Workload("t", 1, heads, D, T, H, W, "topk", k=3, tile=tile)
+    plan = types.SimpleNamespace(N=N, V=int(np.prod(tile)), kmax=kmax,
+                                 info=types.SimpleNamespace(nT=nT, nH=nH, nW=nW))
+    assert bench.valid_token_flops(wl, plan, idx, cnt) == float(want)
+    if grid == (8, 8, 8):  # no padding: every kept pair counts in full
+        kept = sum(len(l) for hl in lists for l in hl)
+        assert want == kept * bench.pair_flops(D)
