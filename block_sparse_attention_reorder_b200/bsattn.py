@@ -88,6 +88,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "attn_schedule_plan": [P, I, ctypes.POINTER(P)],
         "attn_schedule_workspace_bytes": [P, ctypes.POINTER(Z)],
         "attn_schedule_layer": [P, I, P, P, P, P, P, P, P, P, Z, P],
+        "attn_testing_force_timeout": [I],
+        "attn_testing_set_error_word": [P, I],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -104,7 +106,7 @@ EXPORTED = ("attn_plan_create", "attn_plan_destroy", "attn_plan_info", "attn_sta
             "attn_forward", "attn_forward_natural",
             "attn_layer", "attn_check_device_status", "attn_schedule_create", "attn_schedule_destroy",
             "attn_schedule_plan", "attn_schedule_workspace_bytes", "attn_schedule_layer",
-            "attn_backward")
+            "attn_backward", "attn_testing_force_timeout", "attn_testing_set_error_word")
 
 
 def _check(code: int, where: str):
@@ -417,6 +419,17 @@ def attn_backward(plan: Plan, q_t, k_t, v_t, o_t, do_t, lse_t, idx, cnt, dq_t, d
 def attn_check_device_status(plan: Plan, stream=None) -> int:
     """Synchronise, read and clear the device error word; returns the status code."""
     return int(_lib.attn_check_device_status(plan.handle, _stream(stream)))
+
+
+def attn_testing_force_timeout(on: bool):
+    """Testing hook: attention forward launches take their bounded-wait
+    timeout path while on (see include/bsattn.h)."""
+    _check(_lib.attn_testing_force_timeout(int(bool(on))), "attn_testing_force_timeout")
+
+
+def attn_testing_set_error_word(plan: Plan, bits: int):
+    """Testing hook: write the plan's device error word."""
+    _check(_lib.attn_testing_set_error_word(plan.handle, int(bits)), "attn_testing_set_error_word")
 
 
 def attn_status_string(code: int) -> str:

@@ -73,6 +73,7 @@ constexpr int kStages = 2;
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kColS0 = 0, kColS1 = 64, kColO = 128;
 constexpr long long kWaitLimit = 4000000000LL;  // SM cycles (~2 s)
+constexpr long long kTestWaitLimit = 2000000LL;  // ~1 ms, with the testing hook on
 constexpr float kRescaleThreshold = 8.0f;        // log2 units
 
 struct TcParams {
@@ -90,6 +91,8 @@ struct TcParams {
   int bm_words;  // bitmap words per list
   int pair_axis; // 0 = t, 1 = h, 2 = w
   int pdim[3];   // work items along t, h, w (pair axis halved)
+  long long wait_limit;  // SM cycles a wait that can be aborted may take
+  int stall;             // testing: the MMA thread first waits on a barrier nothing arrives at
 };
 
 template <int D, bool FP8>
@@ -386,7 +389,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         if (m < L) {
           const int s = m % kStages;
           if (m >= kStages &&
-              !tc::mbar_wait(bar_kempty(s), ((m / kStages) - 1) & 1, abort_flag, kWaitLimit)) {
+              !tc::mbar_wait(bar_kempty(s), ((m / kStages) - 1) & 1, abort_flag, P.wait_limit)) {
             record_timeout(abort_flag, P.err);
             break;
           }
@@ -405,7 +408,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         if (m >= 1) {
           const int v = m - 1, s = v % kStages;
           if (v >= kStages &&
-              !tc::mbar_wait(bar_vempty(s), ((v / kStages) - 1) & 1, abort_flag, kWaitLimit)) {
+              !tc::mbar_wait(bar_vempty(s), ((v / kStages) - 1) & 1, abort_flag, P.wait_limit)) {
             record_timeout(abort_flag, P.err);
             break;
           }
@@ -436,10 +439,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       constexpr uint32_t idS = FP8 ? tc::instr_desc(0, 0, 0, 0, 64, 128)
                                    : tc::instr_desc(1, 1, 0, 0, 64, 128);
       constexpr uint32_t idPV = tc::instr_desc(1, 1, 0, 1, D, 128);
-      bool ok = tc::mbar_wait(bar_q, 0, abort_flag, kWaitLimit);
+      // Testing hook: bar_final gets its first arrival only from the final
+      // commit below, so this wait runs out and the CTA takes the timeout path.
+      bool ok = !P.stall || tc::mbar_wait(bar_final, 0, abort_flag, P.wait_limit);
+      ok = ok && tc::mbar_wait(bar_q, 0, abort_flag, P.wait_limit);
       auto issue_S = [&](int m) -> bool {
         const int s = m % kStages;
-        if (!tc::mbar_wait(bar_kfull(s), (m / kStages) & 1, abort_flag, kWaitLimit)) return false;
+        if (!tc::mbar_wait(bar_kfull(s), (m / kStages) & 1, abort_flag, P.wait_limit)) return false;
         tc::fence_after_sync();
         const uint32_t dS = tmem + ((m & 1) ? kColS1 : kColS0);
 #pragma unroll
@@ -462,8 +468,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       if (ok && L > 1) ok = issue_S(1);
       for (int n = 0; ok && n < L; ++n) {
         const int s = n % kStages;
-        if (!tc::mbar_wait(bar_pfull(n & 1), (n >> 1) & 1, abort_flag, kWaitLimit) ||
-            !tc::mbar_wait(bar_vfull(s), (n / kStages) & 1, abort_flag, kWaitLimit)) {
+        if (!tc::mbar_wait(bar_pfull(n & 1), (n >> 1) & 1, abort_flag, P.wait_limit) ||
+            !tc::mbar_wait(bar_vfull(s), (n / kStages) & 1, abort_flag, P.wait_limit)) {
           ok = false;
           break;
         }
@@ -501,7 +507,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       const uint32_t e = ulist[n];
       const int j = (int)(e & 0x1FFFFFu);
       const bool keep = ((e >> (30 + half)) & 1u) != 0;  // uniform within the warp
-      if (!__all_sync(0xffffffffu, tc::mbar_wait(bar_sfull(n & 1), (n >> 1) & 1, abort_flag, kWaitLimit))) {
+      if (!__all_sync(0xffffffffu, tc::mbar_wait(bar_sfull(n & 1), (n >> 1) & 1, abort_flag, P.wait_limit))) {
         ok = false;
         break;
       }
@@ -577,7 +583,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       if (__any_sync(0xffffffffu, need)) {
         // O holds PV_0..PV_{n-1} once PV_{n-1} has completed.
         if (!__all_sync(0xffffffffu,
-                        tc::mbar_wait(bar_pvdone((n - 1) & 1), ((n - 1) >> 1) & 1, abort_flag, kWaitLimit))) {
+                        tc::mbar_wait(bar_pvdone((n - 1) & 1), ((n - 1) >> 1) & 1, abort_flag, P.wait_limit))) {
           ok = false;
           break;
         }
@@ -599,7 +605,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     // ---------------------------------------------------------- epilogue
     if (ok && L > 0) {
       if (!__all_sync(0xffffffffu,
-                      tc::mbar_wait(bar_pvdone((L - 1) & 1), ((L - 1) >> 1) & 1, abort_flag, kWaitLimit))) {
+                      tc::mbar_wait(bar_pvdone((L - 1) & 1), ((L - 1) >> 1) & 1, abort_flag, P.wait_limit))) {
         record_timeout(abort_flag, P.err);
         ok = false;
       }
@@ -744,6 +750,8 @@ bsattn_status launch_attention(const bsattn_plan* p, const void* q, const void* 
                             : (p->N < p->kmax ? p->N : p->kmax) * p->nchunk;
   prm.bm_words = (p->N + 31) / 32;
   prm.pair_axis = pair_axis_of(p);
+  prm.stall = bsattn_testing_timeout_forced() ? 1 : 0;
+  prm.wait_limit = prm.stall ? kTestWaitLimit : kWaitLimit;
   const int nd[3] = {p->nT, p->nH, p->nW};
   for (int a = 0; a < 3; ++a) prm.pdim[a] = a == prm.pair_axis ? (nd[a] + 1) / 2 : nd[a];
   const bool fp8 = p->desc.qk_fp8 != 0, d128 = p->desc.head_dim == 128;

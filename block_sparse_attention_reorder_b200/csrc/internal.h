@@ -91,6 +91,10 @@ struct DeviceGuard {
   DeviceGuard& operator=(const DeviceGuard&) = delete;
 };
 
+// Testing hook (attn_testing_force_timeout): whether attention forward
+// launches should take their timeout path.
+bool bsattn_testing_timeout_forced();
+
 // Looks up, with `device` current, the device address of the library-owned
 // scratch array of attn_select_static and caches it; the lookup loads the
 // module that holds the array (reserving its memory on that device).

@@ -4,6 +4,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <atomic>
 #include <new>
 #include <vector>
 
@@ -92,9 +93,26 @@ BackwardWs carve_backward(const bsattn_plan* p, Carve& c) {
 bool ok_ptr(const void* x) { return x != nullptr && aligned16(x); }
 
 
+std::atomic<int> g_force_timeout{0};
+
 }  // namespace
 
+bool bsattn_testing_timeout_forced() { return g_force_timeout.load(std::memory_order_relaxed) != 0; }
+
 extern "C" {
+
+bsattn_status attn_testing_force_timeout(int on) {
+  g_force_timeout.store(on ? 1 : 0, std::memory_order_relaxed);
+  return BSATTN_OK;
+}
+
+bsattn_status attn_testing_set_error_word(const bsattn_plan* p, int bits) {
+  if (!p) return BSATTN_ERR_INVALID_ARG;
+  DeviceGuard dev(p->device);
+  if (dev.status) return dev.status;
+  BSATTN_CUDA_TRY(cudaMemcpy(p->d_err, &bits, sizeof(int), cudaMemcpyHostToDevice));
+  return BSATTN_OK;
+}
 
 const char* attn_status_string(bsattn_status s) {
   switch (s) {

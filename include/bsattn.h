@@ -318,6 +318,25 @@ bsattn_status attn_schedule_layer(const bsattn_schedule* schedule, int step, con
                                   float* lse_nat, int32_t* idx_out, int32_t* cnt_out, void* ws,
                                   size_t ws_bytes, void* stream);
 
+/* Testing hooks. Neither is part of the method (the pages have no
+ * counterpart); they let tests reach the failure paths without faulting a GPU.
+ *
+ * attn_testing_force_timeout(1): attention forward launches made afterwards
+ * in this process (attn_forward, attn_forward_natural, attn_layer) cap the
+ * kernel's abortable waits at about 1 ms and make each CTA's MMA-issuing
+ * thread first wait on a barrier nothing arrives at, so every CTA takes its
+ * bounded-wait timeout path: it records BSATTN_ERR_TIMEOUT in the plan's
+ * device error word, lets its own copies and MMAs finish, frees its tensor
+ * memory and returns; the outputs are then unspecified. (0) restores normal
+ * launches. Process-wide; not for use while other threads launch work.
+ *
+ * attn_testing_set_error_word: writes `bits` (BSATTN_DEVERR_* bits: 1 = bad
+ * list entry, 2 = timeout) into the plan's device error word with a
+ * synchronous copy, so that attn_check_device_status's mapping can be tested
+ * without a kernel. */
+bsattn_status attn_testing_force_timeout(int on);
+bsattn_status attn_testing_set_error_word(const bsattn_plan* plan, int bits);
+
 #ifdef __cplusplus
 }
 #endif

@@ -196,3 +196,40 @@ def test_backward_tiles_form_equals_full_mask_form():
         for j, (tok, gk, gv) in dkv_t.items():
             np.testing.assert_allclose(gk, dk[0, tok, h], rtol=1e-12, atol=1e-13)
             np.testing.assert_allclose(gv, dv[0, tok, h], rtol=1e-12, atol=1e-13)
+
+
+def test_layer_gradient_through_routing_is_the_fixed_mask_gradient():
+    """The routing (pool -> score -> select) is piecewise constant in Q and
+    K: away from score ties, a small change of Q or K leaves every kept list
+    as it is, so the derivative of the whole layer (routing included) is the
+    gradient with the kept mask held fixed, and nothing flows back through
+    the pooled scores. Central differences of the routed layer, with the
+    lists checked unchanged at every probe, against attention_backward_full
+    on the routed lists."""
+    rng = np.random.default_rng(21)
+    T, H, W, D = 4, 8, 12, 8  # 1 x 2 x 3 = 6 tiles of (4,4,4)
+    shape = (1, T * H * W, 1, D)
+    q, k, v, do = (rng.standard_normal(shape) for _ in range(4))
+
+    def routed(qq, kk):
+        return attention.route(qq, kk, T, H, W, "topk", k=2)[3]
+
+    lists = routed(q, k)
+    dq, dk, dv = attention.attention_backward_full(q, k, v, do, lists, T, H, W)
+
+    def loss(qq, kk, vv):
+        lst = routed(qq, kk)
+        assert all(np.array_equal(a, b) for a, b in zip(lst, lists)), "probe crossed a score tie"
+        return float((attention.attention_full(qq, kk, vv, lst, T, H, W)[0] * do).sum())
+
+    h = 1e-6
+    for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        for flat in rng.choice(x.size, size=12, replace=False):
+            idx = np.unravel_index(flat, x.shape)
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            args_p = {"q": (xp, k, v), "k": (q, xp, v), "v": (q, k, xp)}[name]
+            args_m = {"q": (xm, k, v), "k": (q, xm, v), "v": (q, k, xm)}[name]
+            num = (loss(*args_p) - loss(*args_m)) / (2 * h)
+            assert abs(g[idx] - num) <= 1e-6 * max(1.0, abs(num)), (name, idx, g[idx], num)
