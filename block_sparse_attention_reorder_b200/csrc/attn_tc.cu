@@ -252,9 +252,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     tc::tmem_alloc(sb + C::OFF_MISC, kTmemCols);
     tc::tmem_relinquish();
   }
-  if (tid < 64) {  // in-chunk (t, h, w) offsets of each chunk row
-    int dt = tid / (g.ch * g.cw), dh = (tid / g.cw) % g.ch, dw = tid % g.cw;
-    colc[tid] = (uint32_t)dt | ((uint32_t)dh << 8) | ((uint32_t)dw << 16);
+  if (tid < 64) colc[tid] = chunk_row_code(g, tid);  // in-chunk (t, h, w) offsets of each chunk row
+  if (g.cr < 64) {
+    // Tiles of fewer than 64 tokens: natural-layout loads fill only the
+    // chunk box's rows; the rest of every V slot must hold finite values.
+    for (int x = tid; x < kStages * C::V_BYTES / 16; x += kThreads)
+      reinterpret_cast<uint4*>(smem + C::OFF_V)[x] = make_uint4(0, 0, 0, 0);
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
   for (int w = tid; w < 2 * P.bm_words; w += kThreads) bmA[w] = 0u;
   if (!has1) {
@@ -346,7 +350,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             const int bt = j / (g.nH * g.nW), bhh = (j / g.nW) % g.nH, bw = j % g.nW;
             const int vt = min(g.T - bt * g.tt - o.dt, 255), vh = min(g.H - bhh * g.th - o.dh, 255),
                       vw = min(g.W - bw * g.tw - o.dw, 255);
-            const bool edge = vt < g.ct || vh < g.ch || vw < g.cw;
+            const bool edge = vt < g.ct || vh < g.ch || vw < g.cw || g.cr < 64;
             uext[pos] = (uint32_t)vt | ((uint32_t)vh << 8) | ((uint32_t)vw << 16) | (edge ? 1u << 31 : 0u);
           }
           ++pos;
@@ -367,7 +371,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       tc::tma_prefetch_desc(&tmQ);
       tc::tma_prefetch_desc(&tmK);
       tc::tma_prefetch_desc(&tmV);
-      tc::mbar_arrive_expect_tx(bar_q, (has1 ? 2 : 1) * 64 * C::QRB);
+      // A natural-layout load fills the chunk box's rows (cr of them).
+      const int qrows = NQO && !FP8 ? g.cr : 64, kvrows = NKV ? g.cr : 64;
+      tc::mbar_arrive_expect_tx(bar_q, (has1 ? 2 : 1) * qrows * C::QRB);
       for (int x = 0; x < (has1 ? 2 : 1); ++x) {
         const int tile = x ? i1 : i0, chunk = x ? c1 : c0;
 #pragma unroll
@@ -394,7 +400,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             break;
           }
           const int kt = (int)(ulist[m] & 0x1FFFFFu), kc = (int)((ulist[m] >> 21) & 0x1FFu);
-          tc::mbar_arrive_expect_tx(bar_kfull(s), C::K_BYTES);
+          tc::mbar_arrive_expect_tx(bar_kfull(s), FP8 ? C::K_BYTES : kvrows * C::QRB);
 #pragma unroll
           for (int cb = 0; cb < C::QBLK; ++cb) {
             const uint32_t dst = sb + C::OFF_K + s * C::K_BYTES + cb * 64 * C::SWB;
@@ -413,7 +419,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             break;
           }
           const int vt = (int)(ulist[v] & 0x1FFFFFu), vc = (int)((ulist[v] >> 21) & 0x1FFu);
-          tc::mbar_arrive_expect_tx(bar_vfull(s), C::V_BYTES);
+          tc::mbar_arrive_expect_tx(bar_vfull(s), kvrows * D * 2);
 #pragma unroll
           for (int vb = 0; vb < C::VBLK; ++vb) {
             const uint32_t dst = sb + C::OFF_V + s * C::V_BYTES + vb * 8192;
@@ -635,6 +641,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const ChunkOrigin qo0 = chunk_origin(g, c0), qo1 = chunk_origin(g, c1);
     auto token_of = [&](int rr) -> int {
       const int tile = rr >> 6 ? i1 : i0, q = rr & 63;
+      if (q >= g.cr) return -1;
       const ChunkOrigin o = rr >> 6 ? qo1 : qo0;
       const int t = (tile / (g.nH * g.nW)) * g.tt + o.dt + q / (g.ch * g.cw);
       const int h = ((tile / g.nW) % g.nH) * g.th + o.dh + (q / g.cw) % g.ch;
@@ -678,7 +685,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 
 // ---------------------------------------------------------------- host side
 // Natural-layout tensor [B, T, H, W, Hh * D] as five dimensions, innermost
-// first, with a one-tile box of 64 columns (128 bytes, one swizzle span).
+// first, with a one-chunk box of 64 columns (128 bytes, one swizzle span).
 bool make_map_nat(CUtensorMap* map, const void* base, const bsattn_plan* p) {
   auto fn = encode_fn();
   if (!fn) return false;

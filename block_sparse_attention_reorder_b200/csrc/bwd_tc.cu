@@ -172,7 +172,7 @@ __device__ __forceinline__ void compact_steps(const Geom& g, const uint32_t* bmA
           const ChunkOrigin o = chunk_origin(g, c);
           const int vt = min(g.T - bt * g.tt - o.dt, 255), vh = min(g.H - bhh * g.th - o.dh, 255),
                     vw = min(g.W - bw * g.tw - o.dw, 255);
-          const bool edge = vt < g.ct || vh < g.ch || vw < g.cw;
+          const bool edge = vt < g.ct || vh < g.ch || vw < g.cw || g.cr < 64;
           list[pos] = e | ((uint32_t)c << 21);
           ext[pos] = (uint32_t)vt | ((uint32_t)vh << 8) | ((uint32_t)vw << 16) | (edge ? 1u << 31 : 0u);
         }
@@ -238,10 +238,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     tc::tmem_alloc(sb + C::OFF_MISC, kTmemCols);
     tc::tmem_relinquish();
   }
-  if (tid < 64) {  // in-chunk (t, h, w) offsets of each chunk row
-    const int dt = tid / (g.ch * g.cw), dh = (tid / g.cw) % g.ch, dw = tid % g.cw;
-    colc[tid] = (uint32_t)dt | ((uint32_t)dh << 8) | ((uint32_t)dw << 16);
-  }
+  if (tid < 64) colc[tid] = chunk_row_code(g, tid);  // in-chunk (t, h, w) offsets of each chunk row
   for (int w = tid; w < 2 * P.bm_words; w += kThreads) bmA[w] = 0u;
   if (!has1) {  // rows 64..127 have no tile: zero their Q and dO
     for (int x = tid; x < C::QBLK * 64 * 128 / 16; x += kThreads) {
@@ -630,10 +627,7 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     tc::tmem_alloc(sb + C::OFF_MISC, kTmemCols);
     tc::tmem_relinquish();
   }
-  if (tid < 64) {  // in-chunk (t, h, w) offsets of each chunk row
-    const int dt = tid / (g.ch * g.cw), dh = (tid / g.cw) % g.ch, dw = tid % g.cw;
-    colc[tid] = (uint32_t)dt | ((uint32_t)dh << 8) | ((uint32_t)dw << 16);
-  }
+  if (tid < 64) colc[tid] = chunk_row_code(g, tid);  // in-chunk (t, h, w) offsets of each chunk row
   for (int w = tid; w < 2 * P.bm_words; w += kThreads) bmA[w] = 0u;
   if (!has1) {  // rows 64..127 have no key tile: zero their K and V
     for (int x = tid; x < C::QBLK * 64 * 128 / 16; x += kThreads) {

@@ -21,7 +21,7 @@ struct bsattn_plan {
   int device;
   int Tp, Hp, Wp, nT, nH, nW, N, V, L, kmax;
   int nchunk;          // 64-row chunks per tile (V / 64)
-  int ct, ch, cw;      // box of one chunk (t, h, w): ct * ch * cw = 64
+  int ct, ch, cw;      // box of one chunk (t, h, w): ct * ch * cw = 64, or the whole tile of fewer tokens
   float scale;
   int* d_err;        // device error word
   int32_t* d_win_idx;  // window rule: [N, kmax]
@@ -41,6 +41,7 @@ struct Geom {
   int tt, th, tw;
   int nT, nH, nW, N, L;
   int V, nchunk, ct, ch, cw;
+  int cr;  // rows of one chunk box, ct * ch * cw: 64, or fewer for a tile of fewer than 64 tokens
 };
 
 struct ChunkOrigin {
@@ -58,7 +59,17 @@ static inline Geom make_geom(const bsattn_plan* p) {
   g.tt = p->desc.tile_t; g.th = p->desc.tile_h; g.tw = p->desc.tile_w;
   g.nT = p->nT; g.nH = p->nH; g.nW = p->nW; g.N = p->N; g.L = p->L;
   g.V = p->V; g.nchunk = p->nchunk; g.ct = p->ct; g.ch = p->ch; g.cw = p->cw;
+  g.cr = p->ct * p->ch * p->cw;
   return g;
+}
+
+// Packed in-chunk offsets (t | h << 8 | w << 16) of chunk row r. Rows past
+// the chunk box (rows cr..63 of a tile of fewer than 64 tokens, stored as 64
+// rows) get 255 on every axis, which no real extent reaches.
+__host__ __device__ __forceinline__ uint32_t chunk_row_code(const Geom& g, int r) {
+  if (r >= g.cr) return 0xFFFFFFu;
+  const int dt = r / (g.ch * g.cw), dh = (r / g.cw) % g.ch, dw = r % g.cw;
+  return (uint32_t)dt | ((uint32_t)dh << 8) | ((uint32_t)dw << 16);
 }
 
 static inline bool aligned16(const void* ptr) { return (((uintptr_t)ptr) & 15u) == 0; }

@@ -154,9 +154,13 @@ bsattn_status attn_plan_create(const bsattn_desc* d, const bsattn_rule* r, bsatt
     return BSATTN_ERR_INVALID_ARG;
   if (d->head_dim != 64 && d->head_dim != 128) return BSATTN_ERR_UNSUPPORTED;
   // Tiles of 64 * nchunk tokens whose 64-row chunks are boxes of the tile.
+  // Tiles of fewer than 64 tokens are one chunk box, stored as 64 rows of
+  // which the last 64 - V are padding.
   int ct, ch, cw;
-  {
-    const long long vol = (long long)d->tile_t * d->tile_h * d->tile_w;
+  const long long vol = (long long)d->tile_t * d->tile_h * d->tile_w;
+  if (vol < 64) {
+    ct = d->tile_t; ch = d->tile_h; cw = d->tile_w;
+  } else {
     if (vol % 64 != 0 || vol > 64LL * kMaxChunks) return BSATTN_ERR_UNSUPPORTED;
     if (d->tile_t > 1024 || d->tile_h > 1024 || d->tile_w > 1024) return BSATTN_ERR_UNSUPPORTED;
     if (!chunk_box(d->tile_t, d->tile_h, d->tile_w, &ct, &ch, &cw)) return BSATTN_ERR_UNSUPPORTED;
@@ -201,7 +205,7 @@ bsattn_status attn_plan_create(const bsattn_desc* d, const bsattn_rule* r, bsatt
   p->Tp = (int)Tp; p->Hp = (int)Hp; p->Wp = (int)Wp;
   p->nT = (int)(Tp / d->tile_t); p->nH = (int)(Hp / d->tile_h); p->nW = (int)(Wp / d->tile_w);
   p->N = (int)N; p->L = (int)L; p->kmax = kmax;
-  p->V = d->tile_t * d->tile_h * d->tile_w;
+  p->V = vol < 64 ? 64 : (int)vol;  // rows per tile in the tiled layout
   p->nchunk = p->V / 64;
   p->ct = ct; p->ch = ch; p->cw = cw;
   p->scale = d->softmax_scale > 0.f ? d->softmax_scale : (float)(1.0 / sqrt((double)d->head_dim));

@@ -37,7 +37,8 @@
  *   - Block scores containing NaN give unspecified (but in-bounds) lists.
  *
  * Layouts (B batch, Hh heads, D head_dim, L = T*H*W, N = number of tiles,
- * V = tile volume = tile_t*tile_h*tile_w, a multiple of 64):
+ * V = rows per tile = tile_t*tile_h*tile_w, a multiple of 64, or 64 for a
+ * tile of fewer than 64 tokens, whose extra rows are padding):
  *   natural   [B, L, Hh, D] bf16, token n = (t*H + h)*W + w
  *   tiled     [B, Hh, N, V, D] (bf16, or u8 e4m3 codes), tile id
  *             j = ((t/tile_t)*nH + h/tile_h)*nW + w/tile_w, in-tile row
@@ -117,16 +118,16 @@ typedef struct bsattn_plan bsattn_plan;
  * padded token rows over all batches and heads), CUDA.
  *
  * Tile shapes (the pages' "3D tile granularity"; FPSAttention's tile ablation
- * compares (3,4,4) with the hardware-friendly (6,8,8)): the volume V must be
- * 64 * c with 1 <= c <= 512, each side at most 1024, and each run of 64 in-tile rows [64i, 64i + 64)
- * must be a box of the tile: 64 / (tile_h * tile_w) whole (h, w) frames when
- * tile_h * tile_w divides 64, else 64 / tile_w whole w rows when tile_w
- * divides 64 (and 64 / tile_w divides tile_h), else a 64-long run along w
- * when 64 divides tile_w.
- * (4,4,4), (2,4,8), (6,8,8), (4,8,8) and (8,8,8) qualify; (3,4,4) (V = 48)
- * does not. The attention works on these 64-row chunks: with V = 64 two
- * adjacent query tiles share a 128-row block, with V > 64 a block holds two
- * chunks of one query tile, which keep the same key tiles. */
+ * compares (3,4,4) with the hardware-friendly (6,8,8), and (3,4,4) with
+ * (24,32,32)): either fewer than 64 tokens, e.g. (3,4,4), stored as one
+ * 64-row chunk whose last 64 - V rows are padding (info.tile_volume is then
+ * 64); or a volume V = 64 * c with 1 <= c <= 512, each side at most 1024, and
+ * each run of 64 in-tile rows [64i, 64i + 64) a box of the tile: 64 /
+ * (tile_h * tile_w) whole (h, w) frames when tile_h * tile_w divides 64, else
+ * 64 / tile_w whole w rows when tile_w divides 64 (and 64 / tile_w divides
+ * tile_h), else a 64-long run along w when 64 divides tile_w. (4,4,4),
+ * (2,4,8), (6,8,8), (4,8,8), (8,8,8) and (24,32,32) qualify; (3,4,6) (V =
+ * 72) does not. The attention works on these 64-row chunks. */
 bsattn_status attn_plan_create(const bsattn_desc* desc, const bsattn_rule* rule,
                                bsattn_plan** out);
 void attn_plan_destroy(bsattn_plan* plan);

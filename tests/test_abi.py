@@ -38,7 +38,7 @@ def test_status_strings():
 
 @pytest.mark.parametrize("kw,code", [
     (dict(head_dim=96), 2),                     # unsupported head_dim
-    (dict(tile=(3, 4, 4)), 2),                  # tile volume 48, not a multiple of 64
+    (dict(tile=(3, 4, 6)), 2),                  # tile volume 72: above 64, not a multiple of 64
     (dict(tile=(2, 3, 32)), 2),                 # 64-row runs are not boxes (3 h rows of 32)
     (dict(tile=(8, 1, 24)), 2),                 # 24-token frames do not divide 64
     (dict(tile=(1, 1, 2048)), 2),               # a side above 1024

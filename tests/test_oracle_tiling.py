@@ -23,7 +23,7 @@ def test_counts_match_workload_definitions(name, golden_dir):
 
 TILE_CASES = [((5, 6, 7), (4, 4, 4)), ((8, 16, 16), (4, 4, 4)), ((1, 1, 1), (4, 4, 4)),
               ((4, 9, 4), (4, 4, 4)), ((7, 10, 9), (6, 8, 8)), ((5, 6, 11), (2, 4, 8)),
-              ((3, 5, 70), (1, 1, 128))]
+              ((3, 5, 70), (1, 1, 128)), ((7, 10, 13), (3, 4, 4))]
 
 
 @pytest.mark.parametrize("grid,tile", TILE_CASES)
@@ -71,7 +71,7 @@ def test_pool_is_valid_token_mean():
 
 
 @pytest.mark.parametrize("grid,tile", [((6, 5, 9), (4, 4, 4)), ((7, 10, 9), (6, 8, 8)),
-                                       ((5, 6, 11), (2, 4, 8))])
+                                       ((5, 6, 11), (2, 4, 8)), ((7, 10, 13), (3, 4, 4))])
 def test_pool_against_coordinate_masks(grid, tile):
     rng = np.random.default_rng(1)
     T, H, W = grid
