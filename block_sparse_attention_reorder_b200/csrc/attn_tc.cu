@@ -210,13 +210,23 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   const int head = blockIdx.y, b = blockIdx.z;
   const size_t bh = (size_t)b * g.Hh + head;
   const bool has1 = i1 >= 0;
+  // Natural-layout coordinates (w, h, t) of a chunk's first token: the tile
+  // origin plus the chunk's in-tile offset o. Computed once per chunk load
+  // (and reused by a step's V load): the one producer thread issues every
+  // load, so its integer divisions sit on the pipeline's path.
+  struct NatXYZ {
+    int x, y, z;
+  };
+  auto nat_xyz = [&](int tile, ChunkOrigin o) -> NatXYZ {
+    const int bt = tile / (g.nH * g.nW), rem = tile - bt * (g.nH * g.nW);
+    const int bhh = rem / g.nW, bw = rem - bhh * g.nW;
+    return NatXYZ{bw * g.tw + o.dw, bhh * g.th + o.dh, bt * g.tt + o.dt};
+  };
   // One chunk (64 tokens x 64 columns) of a natural-layout tensor: the box
-  // {64 columns, cw, ch, ct, 1} at the chunk's first token (tile origin plus
-  // the chunk's in-tile offset o), rows in (t, h, w) order like the tiled
-  // layout; tokens past the grid's edge read as zero.
-  auto load_nat = [&](uint32_t dst, const CUtensorMap* map, uint32_t bar, int col, int tile, ChunkOrigin o) {
-    const int bt = tile / (g.nH * g.nW), bhh = (tile / g.nW) % g.nH, bw = tile % g.nW;
-    tc::tma_load_5d(dst, map, bar, col, bw * g.tw + o.dw, bhh * g.th + o.dh, bt * g.tt + o.dt, b);
+  // {64 columns, cw, ch, ct, 1} at the chunk's first token, rows in (t, h, w)
+  // order like the tiled layout; tokens past the grid's edge read as zero.
+  auto load_nat = [&](uint32_t dst, const CUtensorMap* map, uint32_t bar, int col, NatXYZ p) {
+    tc::tma_load_5d(dst, map, bar, col, p.x, p.y, p.z, b);
   };
   // In-tile offset of a step's key chunk (packed 10 bits per axis; zero for
   // one-chunk tiles).
@@ -376,11 +386,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       tc::mbar_arrive_expect_tx(bar_q, (has1 ? 2 : 1) * qrows * C::QRB);
       for (int x = 0; x < (has1 ? 2 : 1); ++x) {
         const int tile = x ? i1 : i0, chunk = x ? c1 : c0;
+        const NatXYZ qp = NQO && !FP8 ? nat_xyz(tile, chunk_origin(g, chunk)) : NatXYZ{0, 0, 0};
 #pragma unroll
         for (int cb = 0; cb < C::QBLK; ++cb) {
           const uint32_t dst = sb + C::OFF_Q + cb * 128 * C::SWB + x * 64 * C::SWB;
           if (NQO && !FP8)
-            load_nat(dst, &tmQ, bar_q, head * D + cb * 64, tile, chunk_origin(g, chunk));
+            load_nat(dst, &tmQ, bar_q, head * D + cb * 64, qp);
           else
             tc::tma_load_2d(dst, &tmQ, bar_q, cb * C::SWB / C::ESZ, tiled_row(tile, chunk));
         }
@@ -391,7 +402,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       int lastk[kStages], lastv[kStages];
 #pragma unroll
       for (int s = 0; s < kStages; ++s) lastk[s] = lastv[s] = -1;
+      NatXYZ kp{0, 0, 0};  // coordinates of the last natural K load, reused by its step's V load
       for (int m = 0; m <= L; ++m) {
+        NatXYZ vp = kp;
         if (m < L) {
           const int s = m % kStages;
           if (m >= kStages &&
@@ -401,11 +414,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           }
           const int kt = (int)(ulist[m] & 0x1FFFFFu), kc = (int)((ulist[m] >> 21) & 0x1FFu);
           tc::mbar_arrive_expect_tx(bar_kfull(s), FP8 ? C::K_BYTES : kvrows * C::QRB);
+          if (NKV && !FP8) kp = nat_xyz(kt, step_origin(m));
 #pragma unroll
           for (int cb = 0; cb < C::QBLK; ++cb) {
             const uint32_t dst = sb + C::OFF_K + s * C::K_BYTES + cb * 64 * C::SWB;
             if (NKV && !FP8)
-              load_nat(dst, &tmK, bar_kfull(s), head * D + cb * 64, kt, step_origin(m));
+              load_nat(dst, &tmK, bar_kfull(s), head * D + cb * 64, kp);
             else
               tc::tma_load_2d(dst, &tmK, bar_kfull(s), cb * C::SWB / C::ESZ, tiled_row(kt, kc));
           }
@@ -420,11 +434,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           }
           const int vt = (int)(ulist[v] & 0x1FFFFFu), vc = (int)((ulist[v] >> 21) & 0x1FFu);
           tc::mbar_arrive_expect_tx(bar_vfull(s), kvrows * D * 2);
+          if (NKV && FP8) vp = nat_xyz(vt, step_origin(v));  // K came from tile codes: nothing to reuse
 #pragma unroll
           for (int vb = 0; vb < C::VBLK; ++vb) {
             const uint32_t dst = sb + C::OFF_V + s * C::V_BYTES + vb * 8192;
             if (NKV)
-              load_nat(dst, &tmV, bar_vfull(s), head * D + vb * 64, vt, step_origin(v));
+              load_nat(dst, &tmV, bar_vfull(s), head * D + vb * 64, vp);
             else
               tc::tma_load_2d(dst, &tmV, bar_vfull(s), vb * 64, tiled_row(vt, vc));
           }
