@@ -227,17 +227,10 @@ def valid_token_flops(wl, plan, idx: torch.Tensor, cnt: torch.Tensor) -> float:
     return float(4.0 * wl.head_dim * (own * keys).sum().item())
 
 
-def layer_tiles_kv(plan) -> bool:
-    """Whether attn_layer re-tiles K and V (kept chunks loaded 64+ times)."""
-    nch = plan.V // 64
-    return plan.kmax * (1 if nch == 1 else (nch + 1) // 2) >= 64
-
-
 def launches_per_step(wl, plan) -> int:
     pooled = wl.rule != "window"
     quant = 2 if wl.qk_fp8 else 0  # e4m3 tile codes of Q and K
-    retile = 0 if not layer_tiles_kv(plan) else (1 if wl.qk_fp8 else 2)  # K and V (or V) re-tiled once
-    return quant + (2 if pooled else 0) + retile + 1 + 1  # [pool Q+K, scores], select, attention
+    return quant + (2 if pooled else 0) + 1 + 1  # [pool Q+K, scores], select, attention
 
 
 class ClockSampler:
@@ -652,10 +645,7 @@ def component_timing(bsattn, plan, wl, q, k, v, flush, stream, reps=20):
         codes = [torch.empty(plan.tiled_shape(), dtype=torch.uint8, device="cuda") for _ in range(2)]
         scales = [torch.empty((wl.B, wl.heads, plan.N), dtype=torch.float32, device="cuda")
                   for _ in range(2)]
-    # The layer re-tiles K and V once a kept key chunk is loaded 64+ times;
-    # its attention then reads tiled K/V, timed here as attn_forward.
-    tiles_kv = layer_tiles_kv(plan)
-    names = ["pool_qk", "reorder_qk", "quantize", "reorder_kv", "block_scores", "select", "attention",
+    names = ["pool_qk", "reorder_qk", "quantize", "block_scores", "select", "attention",
              "attention_tiled", "attention_natural"]
     acc = {n: 0.0 for n in names}
 
@@ -688,10 +678,6 @@ def component_timing(bsattn, plan, wl, q, k, v, flush, stream, reps=20):
         if pooled:
             marks.append(timed("block_scores", lambda: bsattn.attn_block_scores(plan, pq, pk, S, stream)))
         marks.append(timed("select", lambda: bsattn.attn_select_from_scores(plan, S, idx, cnt, stream)))
-        if tiles_kv:
-            marks.append(timed("reorder_kv", lambda: (
-                bsattn.attn_reorder(plan, k, tiled[1], None, stream) if not wl.qk_fp8 else None,
-                bsattn.attn_reorder(plan, v, tiled[2], None, stream))))
         flush.fill_(2.0)
         marks.append(timed("attention_natural", lambda: bsattn.attn_forward_natural(
             plan, qn, kn, v, idx, cnt, o, q_scale=qs, k_scale=ks, stream=stream)))
@@ -703,7 +689,7 @@ def component_timing(bsattn, plan, wl, q, k, v, flush, stream, reps=20):
             for n, a, b in marks:
                 acc[n] += a.elapsed_time(b)
     out = {n: acc[n] / reps for n in names if acc[n] > 0}
-    out["attention"] = out["attention_tiled" if tiles_kv else "attention_natural"]
+    out["attention"] = out["attention_natural"]
     return out
 
 

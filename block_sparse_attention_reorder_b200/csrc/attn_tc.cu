@@ -135,11 +135,11 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi, float& sum) 
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// NQO: Q is read from and O (and lse) written to the natural token layout
-// [B, L, Hh, D] directly; NKV: K and V are read from it. Natural reads go
+// NAT: Q, K and V are read from and O (and lse) written to the natural token
+// layout [B, L, Hh, D] directly (else all tiled). Natural reads go
 // through five-dimensional tensor maps whose box is one tile. e4m3 Q/K are
 // always tile codes (tiled layout).
-template <int D, bool FP8, bool NQO, bool NKV>
+template <int D, bool FP8, bool NAT>
 __global__ void __launch_bounds__(kThreads, 2)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, TcParams P) {
@@ -187,7 +187,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     c0 = 2 * (blockIdx.x % per);
     c1 = c0 + 1;
     if (c1 >= nchunk) i1 = -1;
-    if (NQO) {
+    if (NAT) {
       if (i1 >= 0 && !chunk_real(i1, c1)) i1 = -1;
       if (!chunk_real(i0, c0)) {
         if (i1 < 0) return;  // uniform over the CTA, before any setup
@@ -382,15 +382,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       tc::tma_prefetch_desc(&tmK);
       tc::tma_prefetch_desc(&tmV);
       // A natural-layout load fills the chunk box's rows (cr of them).
-      const int qrows = NQO && !FP8 ? g.cr : 64, kvrows = NKV ? g.cr : 64;
+      const int qrows = NAT && !FP8 ? g.cr : 64, kvrows = NAT ? g.cr : 64;
       tc::mbar_arrive_expect_tx(bar_q, (has1 ? 2 : 1) * qrows * C::QRB);
       for (int x = 0; x < (has1 ? 2 : 1); ++x) {
         const int tile = x ? i1 : i0, chunk = x ? c1 : c0;
-        const NatXYZ qp = NQO && !FP8 ? nat_xyz(tile, chunk_origin(g, chunk)) : NatXYZ{0, 0, 0};
+        const NatXYZ qp = NAT && !FP8 ? nat_xyz(tile, chunk_origin(g, chunk)) : NatXYZ{0, 0, 0};
 #pragma unroll
         for (int cb = 0; cb < C::QBLK; ++cb) {
           const uint32_t dst = sb + C::OFF_Q + cb * 128 * C::SWB + x * 64 * C::SWB;
-          if (NQO && !FP8)
+          if (NAT && !FP8)
             load_nat(dst, &tmQ, bar_q, head * D + cb * 64, qp);
           else
             tc::tma_load_2d(dst, &tmQ, bar_q, cb * C::SWB / C::ESZ, tiled_row(tile, chunk));
@@ -414,11 +414,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           }
           const int kt = (int)(ulist[m] & 0x1FFFFFu), kc = (int)((ulist[m] >> 21) & 0x1FFu);
           tc::mbar_arrive_expect_tx(bar_kfull(s), FP8 ? C::K_BYTES : kvrows * C::QRB);
-          if (NKV && !FP8) kp = nat_xyz(kt, step_origin(m));
+          if (NAT && !FP8) kp = nat_xyz(kt, step_origin(m));
 #pragma unroll
           for (int cb = 0; cb < C::QBLK; ++cb) {
             const uint32_t dst = sb + C::OFF_K + s * C::K_BYTES + cb * 64 * C::SWB;
-            if (NKV && !FP8)
+            if (NAT && !FP8)
               load_nat(dst, &tmK, bar_kfull(s), head * D + cb * 64, kp);
             else
               tc::tma_load_2d(dst, &tmK, bar_kfull(s), cb * C::SWB / C::ESZ, tiled_row(kt, kc));
@@ -434,11 +434,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           }
           const int vt = (int)(ulist[v] & 0x1FFFFFu), vc = (int)((ulist[v] >> 21) & 0x1FFu);
           tc::mbar_arrive_expect_tx(bar_vfull(s), kvrows * D * 2);
-          if (NKV && FP8) vp = nat_xyz(vt, step_origin(v));  // K came from tile codes: nothing to reuse
+          if (NAT && FP8) vp = nat_xyz(vt, step_origin(v));  // K came from tile codes: nothing to reuse
 #pragma unroll
           for (int vb = 0; vb < C::VBLK; ++vb) {
             const uint32_t dst = sb + C::OFF_V + s * C::V_BYTES + vb * 8192;
-            if (NKV)
+            if (NAT)
               load_nat(dst, &tmV, bar_vfull(s), head * D + vb * 64, vp);
             else
               tc::tma_load_2d(dst, &tmV, bar_vfull(s), vb * 64, tiled_row(vt, vc));
@@ -665,7 +665,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     };
     const float lse_r = l > 0.f ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
     if (P.lse && row_exists) {
-      if (NQO) {
+      if (NAT) {
         const int n = token_of(r);
         if (n >= 0) P.lse[bh * (size_t)g.L + n] = lse_r;
       } else {
@@ -678,7 +678,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     for (int e2 = r; e2 < rows * CPR; e2 += 128) {
       const int rr = e2 / CPR, cc = e2 % CPR;
       const uint4 val = *reinterpret_cast<const uint4*>(smem + C::OFF_K + rr * C::O_PITCH + cc * 16);
-      if (NQO) {
+      if (NAT) {
         const int n = token_of(rr);
         if (n >= 0)
           reinterpret_cast<uint4*>(P.o + (((size_t)b * g.L + n) * g.Hh + head) * D)[cc] = val;
@@ -717,7 +717,7 @@ bool make_map_nat(CUtensorMap* map, const void* base, const bsattn_plan* p) {
   return r == CUDA_SUCCESS;
 }
 
-template <int D, bool FP8, bool NQO, bool NKV>
+template <int D, bool FP8, bool NAT>
 bsattn_status run(const bsattn_plan* p, const void* q, const void* k, const __nv_bfloat16* v,
                   TcParams prm, cudaStream_t st) {
   using C = Cfg<D, FP8>;
@@ -726,18 +726,18 @@ bsattn_status run(const bsattn_plan* p, const void* q, const void* k, const __nv
   CUtensorMap mq, mk, mv;
   const CUtensorMapDataType dqk = FP8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const CUtensorMapSwizzle sw = C::SWB == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
-  if (NQO && !FP8 ? !make_map_nat(&mq, q, p) : !bsattn_make_map_2d(&mq, q, dqk, C::ESZ, D, rows, C::SWB / C::ESZ, 64, sw))
+  if (NAT && !FP8 ? !make_map_nat(&mq, q, p) : !bsattn_make_map_2d(&mq, q, dqk, C::ESZ, D, rows, C::SWB / C::ESZ, 64, sw))
     return BSATTN_ERR_CUDA;
-  if (NKV && !FP8 ? !make_map_nat(&mk, k, p) : !bsattn_make_map_2d(&mk, k, dqk, C::ESZ, D, rows, C::SWB / C::ESZ, 64, sw))
+  if (NAT && !FP8 ? !make_map_nat(&mk, k, p) : !bsattn_make_map_2d(&mk, k, dqk, C::ESZ, D, rows, C::SWB / C::ESZ, 64, sw))
     return BSATTN_ERR_CUDA;
-  if (NKV ? !make_map_nat(&mv, v, p)
+  if (NAT ? !make_map_nat(&mv, v, p)
           : !bsattn_make_map_2d(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, rows, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B))
     return BSATTN_ERR_CUDA;
   // Step list, extents and (tiles of several chunks) chunk offsets.
   size_t smem = 1024 + C::OFF_DYN + (size_t)prm.bm_words * 8 + (size_t)prm.umax * (p->nchunk > 1 ? 12 : 8);
   if (smem < 80 * 1024) smem = 80 * 1024;  // at most two CTAs (2 x 256 TMEM columns) per SM
   if (smem > 227 * 1024) return BSATTN_ERR_UNSUPPORTED;
-  auto kern = attn_tc_kernel<D, FP8, NQO, NKV>;
+  auto kern = attn_tc_kernel<D, FP8, NAT>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return BSATTN_ERR_CUDA;
   const int items = p->nchunk > 1 ? p->N * ((p->nchunk + 1) / 2) : prm.pdim[0] * prm.pdim[1] * prm.pdim[2];
@@ -777,16 +777,10 @@ bsattn_status launch_attention(const bsattn_plan* p, const void* q, const void* 
   const int nd[3] = {p->nT, p->nH, p->nW};
   for (int a = 0; a < 3; ++a) prm.pdim[a] = a == prm.pair_axis ? (nd[a] + 1) / 2 : nd[a];
   const bool fp8 = p->desc.qk_fp8 != 0, d128 = p->desc.head_dim == 128;
-#define BSATTN_RUN(QO, KV)                                                                          \
-  return d128 ? (fp8 ? run<128, true, QO, KV>(p, q, k, v, prm, st) : run<128, false, QO, KV>(p, q, k, v, prm, st)) \
-              : (fp8 ? run<64, true, QO, KV>(p, q, k, v, prm, st) : run<64, false, QO, KV>(p, q, k, v, prm, st))
-  switch (lay) {
-    case AttnLayout::Natural:
-      BSATTN_RUN(true, true);
-    case AttnLayout::NaturalQO:
-      BSATTN_RUN(true, false);
-    default:
-      BSATTN_RUN(false, false);
-  }
+#define BSATTN_RUN(NATV)                                                                            \
+  return d128 ? (fp8 ? run<128, true, NATV>(p, q, k, v, prm, st) : run<128, false, NATV>(p, q, k, v, prm, st)) \
+              : (fp8 ? run<64, true, NATV>(p, q, k, v, prm, st) : run<64, false, NATV>(p, q, k, v, prm, st))
+  if (lay == AttnLayout::Natural) BSATTN_RUN(true);
+  BSATTN_RUN(false);
 #undef BSATTN_RUN
 }

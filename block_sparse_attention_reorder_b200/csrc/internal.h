@@ -144,19 +144,14 @@ bsattn_status launch_broadcast_lists(int bh, int N, int kmax, const int32_t* src
                                      const int32_t* src_cnt, int32_t* idx, int32_t* cnt,
                                      cudaStream_t st);
 // Where the attention's tensors live. Tiled: all tiled. Natural: Q, K, V, O
-// and lse in the natural layout ([B, L, Hh, D], [B, Hh, L]). NaturalQO: Q, O
-// and lse natural, K and V tiled. e4m3 Q/K are tile codes in every layout.
-enum class AttnLayout { Tiled, Natural, NaturalQO };
+// and lse in the natural layout ([B, L, Hh, D], [B, Hh, L]). e4m3 Q/K are
+// tile codes in both layouts.
+enum class AttnLayout { Tiled, Natural };
 bsattn_status launch_attention(const bsattn_plan* p, const void* q, const void* k,
                                const float* qs, const float* ks, const __nv_bfloat16* v,
                                const int32_t* idx, const int32_t* cnt, __nv_bfloat16* o,
                                float* lse, void* ws, size_t ws_bytes, cudaStream_t st,
                                AttnLayout lay);
-// Whether attn_layer re-tiles K and V: natural chunk loads cost more per load
-// than tiled ones, which outweighs the one-off reorder once a key chunk is
-// loaded about 40+ times: kmax >= 64 with one-chunk tiles (two query tiles
-// per block), kmax * ceil(nchunk / 2) >= 64 otherwise (every block of a query
-// tile loads each kept chunk).
 // Tile axis (0 = t, 1 = h, 2 = w) along which two 64-token tiles are stacked
 // into one 128-row block (attention: query tiles; dK/dV: key tiles). Top-k and
 // top-p: t, whose neighbouring tiles keep the most key tiles in common on the
@@ -170,10 +165,6 @@ static inline int pair_axis_of(const bsattn_plan* p) {
   for (int x = 1; x < 3; ++x)
     if (w[x] > w[a]) a = x;
   return a;
-}
-
-static inline bool layer_tiles_kv(const bsattn_plan* p) {
-  return (long long)p->kmax * (p->nchunk == 1 ? 1 : (p->nchunk + 1) / 2) >= 64;
 }
 size_t attention_workspace_bytes(const bsattn_plan* p);
 // Scratch of the backward pass (carved from the caller's workspace).

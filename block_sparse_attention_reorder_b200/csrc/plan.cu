@@ -42,16 +42,13 @@ SelectWs carve_select(const bsattn_plan* p, Carve& c) {
   return w;
 }
 
-// The layer reads Q and writes O in the natural layout; K and V too unless
-// layer_tiles_kv(), which re-tiles them once. e4m3 Q/K codes (with their
-// tile scales) are tiled.
+// The layer reads Q, K, V and writes O in the natural layout; e4m3 Q/K codes
+// (with their tile scales) are tiled.
 struct LayerWs {
   uint8_t* qt;  // e4m3 tile codes (qk_fp8 only)
   uint8_t* kt;
   float* qs;
   float* ks;
-  __nv_bfloat16* kb;  // tiled bf16 K (layer_tiles_kv, bf16 Q/K)
-  __nv_bfloat16* vt;  // tiled V (layer_tiles_kv)
   SelectWs sel;
   int32_t* idx;
   int32_t* cnt;
@@ -66,9 +63,6 @@ LayerWs carve_layer(const bsattn_plan* p, Carve& c) {
   w.kt = (uint8_t*)c.take(p->desc.qk_fp8 ? elems : 0);
   w.qs = (float*)c.take(p->desc.qk_fp8 ? bh * p->N * sizeof(float) : 0);
   w.ks = (float*)c.take(p->desc.qk_fp8 ? bh * p->N * sizeof(float) : 0);
-  const bool tkv = layer_tiles_kv(p);
-  w.kb = (__nv_bfloat16*)c.take(tkv && !p->desc.qk_fp8 ? elems * 2 : 0);
-  w.vt = (__nv_bfloat16*)c.take(tkv ? elems * 2 : 0);
   if (p->rule.kind == BSATTN_RULE_WINDOW) {
     w.sel.pq = w.sel.pk = w.sel.S = nullptr;
   } else {
@@ -464,22 +458,10 @@ bsattn_status attn_layer(const bsattn_plan* p, const void* q_nat, const void* k_
   // Tile means for the scores; the attention reads natural tensors tile by tile.
   if (pool && (s = launch_pool(g, (const __nv_bfloat16*)q_nat, w.sel.pq, (const __nv_bfloat16*)k_nat, w.sel.pk, st)))
     return s;
-  const void* v = v_nat;
-  const bool tkv = layer_tiles_kv(p);
-  if (tkv) {
-    // Many loads per key tile: one reorder of K and V is cheaper than natural tile loads.
-    if (!p->desc.qk_fp8) {
-      if ((s = launch_reorder(g, (const __nv_bfloat16*)k_nat, w.kb, nullptr, nullptr, RO_WRITE_TILED, st))) return s;
-      k = w.kb;
-    }
-    if ((s = launch_reorder(g, (const __nv_bfloat16*)v_nat, w.vt, nullptr, nullptr, RO_WRITE_TILED, st))) return s;
-    v = w.vt;
-  }
   if (pool && (s = launch_block_scores(g, w.sel.pq, w.sel.pk, p->scale, w.sel.S, p->d_err, st))) return s;
   if ((s = select_core(p, w.sel.S, idx, cnt, st))) return s;
-  return launch_attention(p, q, k, w.qs, w.ks, (const __nv_bfloat16*)v, idx, cnt, (__nv_bfloat16*)o_nat,
-                          lse_nat, w.attn_ws, attention_workspace_bytes(p), st,
-                          tkv ? AttnLayout::NaturalQO : AttnLayout::Natural);
+  return launch_attention(p, q, k, w.qs, w.ks, (const __nv_bfloat16*)v_nat, idx, cnt, (__nv_bfloat16*)o_nat,
+                          lse_nat, w.attn_ws, attention_workspace_bytes(p), st, AttnLayout::Natural);
 }
 
 bsattn_status attn_check_device_status(const bsattn_plan* p, void* stream) {

@@ -250,10 +250,7 @@ bsattn_status attn_forward_natural(const bsattn_plan* plan, const void* q, const
  * attention reads each 64-token chunk of Q straight from the natural layout
  * (the tile reorder happens in its loads; tokens past the grid's edge read
  * as zero and are masked) and writes natural bf16 O and, if non-NULL,
- * natural fp32 lse [B, Hh, L]. K and V are read the same way, or re-tiled
- * once into the workspace when each kept key chunk is loaded 64 or more
- * times (kmax >= 64 for 64-token tiles, kmax * ceil(c/2) >= 64 for tiles of
- * c chunks), which is cheaper than that many natural-layout loads. Results
+ * natural fp32 lse [B, Hh, L]. K and V are read the same way. Results
  * equal the step-by-step path (reorder, attn_forward, unreorder). If idx_out/cnt_out
  * are non-NULL the kept lists are also copied there. `ws` must hold
  * info.layer_workspace_bytes. */
