@@ -117,7 +117,8 @@ struct Cfg {
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base, abort, L, pad
   static constexpr int OFF_COL = OFF_MISC + 16;         // 64 packed column coords
   static constexpr int OFF_SCAN = OFF_COL + 256;        // block-scan scratch
-  static constexpr int OFF_DYN = OFF_SCAN + 64;         // bitmaps, union list
+  static constexpr int OFF_TOK = OFF_SCAN + 64;         // epilogue: natural token of each block row
+  static constexpr int OFF_DYN = OFF_TOK + 512;         // bitmaps, union list
   static constexpr int O_PITCH = D * 2 + 16;            // epilogue staging row pitch
   static_assert(OFF_Q % 1024 == 0 && OFF_K % 1024 == 0 && OFF_V % 1024 == 0, "alignment");
   static_assert(128 * O_PITCH <= OFF_BAR - OFF_K, "epilogue staging fits in the ring");
@@ -664,10 +665,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       return (t < g.T && h < g.H && w < g.W) ? (t * g.H + h) * g.W + w : -1;
     };
     const float lse_r = l > 0.f ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
+    // Each row's token once (its integer divisions would otherwise repeat
+    // for every 16-byte piece of the row in the store loop below).
+    int* tokrow = reinterpret_cast<int*>(smem + C::OFF_TOK);
+    const int tok = NAT && row_exists ? token_of(r) : -1;
+    if (NAT) tokrow[r] = tok;
     if (P.lse && row_exists) {
       if (NAT) {
-        const int n = token_of(r);
-        if (n >= 0) P.lse[bh * (size_t)g.L + n] = lse_r;
+        if (tok >= 0) P.lse[bh * (size_t)g.L + tok] = lse_r;
       } else {
         P.lse[(size_t)tiled_row(half ? i1 : i0, half ? c1 : c0) + (r & 63)] = lse_r;
       }
@@ -679,7 +684,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       const int rr = e2 / CPR, cc = e2 % CPR;
       const uint4 val = *reinterpret_cast<const uint4*>(smem + C::OFF_K + rr * C::O_PITCH + cc * 16);
       if (NAT) {
-        const int n = token_of(rr);
+        const int n = tokrow[rr];
         if (n >= 0)
           reinterpret_cast<uint4*>(P.o + (((size_t)b * g.L + n) * g.Hh + head) * D)[cc] = val;
       } else {
