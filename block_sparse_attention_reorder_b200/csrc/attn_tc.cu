@@ -236,9 +236,31 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const uint32_t v = uorg[n];
     return ChunkOrigin{(int)(v & 0x3FFu), (int)((v >> 10) & 0x3FFu), (int)(v >> 20)};
   };
+  // Real extent of a key chunk (tile j, in-tile offset o) from its first
+  // token along t, h, w (capped at 255), bit 31 set when it is smaller than
+  // the chunk box along some axis (padded keys to mask).
+  auto chunk_ext = [&](int j, ChunkOrigin o) -> uint32_t {
+    const int bt = j / (g.nH * g.nW), rem = j - bt * (g.nH * g.nW);
+    const int bhh = rem / g.nW, bw = rem - bhh * g.nW;
+    const int vt = min(g.T - bt * g.tt - o.dt, 255), vh = min(g.H - bhh * g.th - o.dh, 255),
+              vw = min(g.W - bw * g.tw - o.dw, 255);
+    const bool edge = vt < g.ct || vh < g.ch || vw < g.cw || g.cr < 64;
+    return (uint32_t)vt | ((uint32_t)vh << 8) | ((uint32_t)vw << 16) | (edge ? 1u << 31 : 0u);
+  };
   // First tiled-layout row of chunk c of tile j.
   auto tiled_row = [&](int j, int c) -> int { return (int)((bh * g.N + j) * g.V) + 64 * c; };
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  // The two kept-list counts and this thread's first entry of each list are
+  // read first, so that their latency overlaps the set-up below: an entry's
+  // address does not depend on the counts (entries at and beyond a count
+  // are read but not used).
+  const int32_t* lA = P.idx + (bh * g.N + i0) * (size_t)P.kmax;
+  const int32_t* lB = has1 ? P.idx + (bh * g.N + i1) * (size_t)P.kmax : lA;
+  int nA = P.cnt[bh * g.N + i0];
+  int nB = has1 ? P.cnt[bh * g.N + i1] : 0;
+  int jA = tid < P.kmax ? __ldg(lA + tid) : 0;
+  int jB = has1 && tid < P.kmax ? __ldg(lB + tid) : 0;
 
   // ------------------------------------------------------------ setup
   if (tid == 0) {
@@ -287,23 +309,25 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   // into the step list: one entry per real 64-key chunk of each kept key
   // tile, key tile in bits 0-20, chunk in bits 21-29, bit 30 (31) set when
   // the first (second) query half keeps the tile.
-  int nA = P.cnt[bh * g.N + i0];
-  int nB = has1 ? P.cnt[bh * g.N + i1] : 0;
   if (nA < 0 || nA > P.kmax || nB < 0 || nB > P.kmax) {
     if (tid == 0) atomicOr(P.err, BSATTN_DEVERR_BAD_INDEX);
     nA = min(max(nA, 0), P.kmax);
     nB = min(max(nB, 0), P.kmax);
   }
-  {
-    const int32_t* lA = P.idx + (bh * g.N + i0) * (size_t)P.kmax;
-    const int32_t* lB = has1 ? P.idx + (bh * g.N + i1) * (size_t)P.kmax : lA;
-    for (int e = tid; e < nA + nB; e += kThreads) {
-      int j = e < nA ? __ldg(lA + e) : __ldg(lB + (e - nA));
+  for (int e = tid; e < max(nA, nB); e += kThreads) {
+    if (e != tid) {
+      jA = e < nA ? __ldg(lA + e) : 0;
+      jB = e < nB ? __ldg(lB + e) : 0;
+    }
+#pragma unroll
+    for (int x = 0; x < 2; ++x) {
+      if (e >= (x ? nB : nA)) continue;
+      const int j = x ? jB : jA;
       if (j < 0 || j >= g.N) {
         atomicOr(P.err, BSATTN_DEVERR_BAD_INDEX);
         continue;
       }
-      atomicOr(e < nA ? &bmA[j >> 5] : &bmB[j >> 5], 1u << (j & 31));
+      atomicOr(x ? &bmB[j >> 5] : &bmA[j >> 5], 1u << (j & 31));
     }
   }
   __syncthreads();
@@ -353,16 +377,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           if (nchunk > 1 && !chunk_real(j, c)) continue;
           if (pos < P.umax) {
             ulist[pos] = e | ((uint32_t)c << 21);
-            const ChunkOrigin o = nchunk > 1 ? chunk_origin(g, c) : ChunkOrigin{0, 0, 0};
-            if (nchunk > 1) uorg[pos] = (uint32_t)o.dt | ((uint32_t)o.dh << 10) | ((uint32_t)o.dw << 20);
-            // Real extent of the key chunk from its first token along t, h, w
-            // (capped at 255), bit 31 set when it is smaller than the chunk
-            // box along some axis (padded keys to mask).
-            const int bt = j / (g.nH * g.nW), bhh = (j / g.nW) % g.nH, bw = j % g.nW;
-            const int vt = min(g.T - bt * g.tt - o.dt, 255), vh = min(g.H - bhh * g.th - o.dh, 255),
-                      vw = min(g.W - bw * g.tw - o.dw, 255);
-            const bool edge = vt < g.ct || vh < g.ch || vw < g.cw || g.cr < 64;
-            uext[pos] = (uint32_t)vt | ((uint32_t)vh << 8) | ((uint32_t)vw << 16) | (edge ? 1u << 31 : 0u);
+            if (nchunk > 1) {
+              const ChunkOrigin o = chunk_origin(g, c);
+              uorg[pos] = (uint32_t)o.dt | ((uint32_t)o.dh << 10) | ((uint32_t)o.dw << 20);
+              uext[pos] = chunk_ext(j, o);
+            }
           }
           ++pos;
         }
@@ -523,6 +542,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const bool row_exists = half == 0 || has1;
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
     const float qsc = (FP8 && row_exists) ? P.qs[bh * g.N + (half ? i1 : i0)] : 1.f;
+    if (nchunk == 1) {
+      // Extents of one-chunk tiles, spread over the softmax threads (the
+      // compaction above leaves them out: a dense bitmap word would put up
+      // to 32 entries' divisions on one thread ahead of the CTA barrier).
+      for (int n = r; n < L; n += 128) uext[n] = chunk_ext((int)(ulist[n] & 0x1FFFFFu), ChunkOrigin{0, 0, 0});
+      asm volatile("bar.sync 2, 128;" ::: "memory");
+    }
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int n = 0; n < L; ++n) {
@@ -672,7 +698,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     if (NAT) tokrow[r] = tok;
     if (P.lse && row_exists) {
       if (NAT) {
-        if (tok >= 0) P.lse[bh * (size_t)g.L + tok] = lse_r;
+        if (tok >= 0) P.lse[bh * (size_t)g.L + (size_t)tok] = lse_r;
       } else {
         P.lse[(size_t)tiled_row(half ? i1 : i0, half ? c1 : c0) + (r & 63)] = lse_r;
       }
