@@ -502,8 +502,11 @@ topk_kernel(int rows, int N, int k, const float* __restrict__ S, int32_t* __rest
 // float4 (lane l holds tiles 128c + 4l .. 4l+3 of 128-tile chunk c), binning
 // uses 128 bins so that four bin indices pack into one 32-bit word, and the
 // second pass compares four packed bins with the boundary bin per SWAR
-// subtraction instead of binning every score again. The general search
-// (lane-strided view of the same staged row) covers crowded boundary bins.
+// subtraction instead of binning every score again. The row is not staged in
+// shared memory (which keeps eight warps per CTA and the registers low): the
+// few boundary-bin candidates and the general search for crowded boundary
+// bins (lane-strided view) read it again from global memory, where it is
+// still cached.
 constexpr int kBins7 = 128;
 
 struct Binning7 {  // Binning with 128 bins (indices fit 7 bits)
@@ -556,7 +559,7 @@ __device__ __forceinline__ int find_bin128(const uint32_t* h, int r, int lane, i
 
 template <int C4>
 struct Shape4 {
-  static constexpr int per_warp = 128 * C4 * 4 + 128 * C4 + 2 * 4 * C4 * 4 + kBins * 4 + kCand * 8;
+  static constexpr int per_warp = 128 * C4 + 2 * 4 * C4 * 4 + kBins * 4 + kCand * 8;
   static constexpr int warps = (8 * per_warp <= 48 * 1024) ? 8 : 4;
   static_assert(warps * per_warp <= 48 * 1024, "selection shared memory");
 };
@@ -566,7 +569,6 @@ __global__ void __launch_bounds__(32 * Shape4<C4>::warps)
 topk4_kernel(int rows, int N, int k, const float* __restrict__ S, int32_t* __restrict__ idx,
              int32_t* __restrict__ cnt, int kmax) {
   constexpr int W = Shape4<C4>::warps, VPT = 4 * C4;
-  __shared__ __align__(16) float vals_s[W][128 * C4];
   __shared__ uint32_t bins_s[W][32 * C4];
   __shared__ uint32_t gt_s[W][4 * C4];
   __shared__ uint32_t eq_s[W][4 * C4];
@@ -576,26 +578,28 @@ topk4_kernel(int rows, int N, int k, const float* __restrict__ S, int32_t* __res
   const int r0 = blockIdx.x * W + w;
   if (r0 >= rows) return;
   const float* s = S + (size_t)r0 * N;
-  float* slice = vals_s[w];
   uint32_t* hist = hcnt_s[w];
   const float qnan = __int_as_float(0x7fc00000);
+  auto load4 = [&](int c) -> float4 {
+    const int j0 = 128 * c + 4 * lane;  // N % 4 == 0: a float4 is all in or all out
+    return j0 < N ? __ldg(reinterpret_cast<const float4*>(s + j0)) : make_float4(qnan, qnan, qnan, qnan);
+  };
 
-  // Pass 1: all float4 loads in flight; bins over the extent of an evenly
-  // strided sample of chunks (tiles outside it land in the edge bins).
+  // Pass 1: bins over the extent of an evenly strided sample of chunks (tiles
+  // outside it land in the edge bins), then every chunk binned, loaded in
+  // groups of four float4 so that few registers hold the row.
   constexpr int B0 = C4 < 4 ? C4 : 4;
   constexpr int STEP = C4 / B0;
-  float4 v[C4];
-#pragma unroll
-  for (int c = 0; c < C4; ++c) {
-    const int j0 = 128 * c + 4 * lane;  // N % 4 == 0: a float4 is all in or all out
-    v[c] = j0 < N ? __ldg(reinterpret_cast<const float4*>(s + j0)) : make_float4(qnan, qnan, qnan, qnan);
-  }
   float mn = qnan, mx = qnan;
+  {
+    float4 u[B0];
 #pragma unroll
-  for (int t = 0; t < B0; ++t) {
-    const float4 u = v[t * STEP];
-    mn = fminf(fminf(mn, fminf(u.x, u.y)), fminf(u.z, u.w));
-    mx = fmaxf(fmaxf(mx, fmaxf(u.x, u.y)), fmaxf(u.z, u.w));
+    for (int t = 0; t < B0; ++t) u[t] = load4(t * STEP);
+#pragma unroll
+    for (int t = 0; t < B0; ++t) {
+      mn = fminf(fminf(mn, fminf(u[t].x, u[t].y)), fminf(u[t].z, u[t].w));
+      mx = fmaxf(fmaxf(mx, fmaxf(u[t].x, u[t].y)), fmaxf(u[t].z, u[t].w));
+    }
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
@@ -607,20 +611,27 @@ topk4_kernel(int rows, int N, int k, const float* __restrict__ S, int32_t* __res
 #pragma unroll
   for (int q = 0; q < kBins7 / 32; ++q) hist[lane + 32 * q] = 0;
   __syncwarp();
+  constexpr int G = 4;  // float4 loads in flight per group
 #pragma unroll
-  for (int c = 0; c < C4; ++c) {
-    const int j0 = 128 * c + 4 * lane;
-    uint32_t word = 0;
-    if (j0 < N) {
-      *reinterpret_cast<float4*>(slice + j0) = v[c];
-      const uint32_t b0 = bin(v[c].x), b1 = bin(v[c].y), b2 = bin(v[c].z), b3 = bin(v[c].w);
-      atomicAdd(&hist[b0], 1u);
-      atomicAdd(&hist[b1], 1u);
-      atomicAdd(&hist[b2], 1u);
-      atomicAdd(&hist[b3], 1u);
-      word = b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
+  for (int c0 = 0; c0 < C4; c0 += G) {
+    float4 v[G];
+#pragma unroll
+    for (int t = 0; t < G; ++t) v[t] = c0 + t < C4 ? load4(c0 + t) : make_float4(qnan, qnan, qnan, qnan);
+#pragma unroll
+    for (int t = 0; t < G; ++t) {
+      const int c = c0 + t;
+      if (c >= C4) break;
+      uint32_t word = 0;
+      if (128 * c + 4 * lane < N) {
+        const uint32_t b0 = bin(v[t].x), b1 = bin(v[t].y), b2 = bin(v[t].z), b3 = bin(v[t].w);
+        atomicAdd(&hist[b0], 1u);
+        atomicAdd(&hist[b1], 1u);
+        atomicAdd(&hist[b2], 1u);
+        atomicAdd(&hist[b3], 1u);
+        word = b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
+      }
+      bins_s[w][32 * c + lane] = word;
     }
-    bins_s[w][32 * c + lane] = word;
   }
   __syncwarp();
 
@@ -669,7 +680,7 @@ topk4_kernel(int rows, int N, int k, const float* __restrict__ S, int32_t* __res
       const int wbase = 32 * (lane + 32 * t);
       while (m) {
         const int j = wbase + __ffs(m) - 1;
-        if (pos < kCand) cand_s[w][pos] = comp_key(slice[j], j);
+        if (pos < kCand) cand_s[w][pos] = comp_key(__ldg(s + j), j);
         ++pos;
         m &= m - 1;
       }
@@ -688,8 +699,8 @@ topk4_kernel(int rows, int N, int k, const float* __restrict__ S, int32_t* __res
     __syncwarp();
     n = compact_mask<VPT>(gt_s[w], N, lane, out, kmax);
   } else if (r >= 1) {
-    // General search over the exact extent on the same staged row.
-    const Row row{&slice[lane], N, lane};
+    // General search over the exact extent, reading the row from global memory.
+    const Row row{s + lane, N, lane};
     float lo, hi;
     row_extent<VPT>(row, &lo, &hi);
     const Hist h{hist, nullptr};
