@@ -712,15 +712,23 @@ topk4_kernel(int rows, int N, int k, const float* __restrict__ S, int32_t* __res
   if (lane == 0) cnt[r0] = n;
 }
 
+// Rows per CTA of the top-p kernel, whose row is not staged in shared memory.
+template <int VPT>
+struct ShapeP {
+  static constexpr int per_warp = VPT * 4 + kBins * 4 + kBins * 8 + kCand * 8;
+  static constexpr int warps = (8 * per_warp <= 48 * 1024) ? 8 : 4;
+  static_assert(warps * per_warp <= 48 * 1024, "selection shared memory");
+};
+
 // Top-p with a top-k floor: in descending order keep the shortest prefix
 // whose softmax mass reaches p of the row's total, then at least k and at
-// most N tiles.
+// most N tiles. Every pass reads the row from global memory (still cached
+// after the first): staging it in shared memory would halve the warps per SM.
 template <int VPT>
-__global__ void __launch_bounds__(32 * Shape<VPT, true>::warps)
+__global__ void __launch_bounds__(32 * ShapeP<VPT>::warps, 4)
 topp_kernel(int rows, int N, int k, double p, const float* __restrict__ S, int32_t* __restrict__ idx,
             int32_t* __restrict__ cnt, int kmax) {
-  constexpr int W = Shape<VPT, true>::warps;
-  __shared__ float vals_s[W][32 * VPT];
+  constexpr int W = ShapeP<VPT>::warps;
   __shared__ uint32_t hcnt_s[W][kBins];
   __shared__ uint64_t hwt_s[W][kBins];
   __shared__ uint32_t mask_s[W][VPT];
@@ -729,9 +737,8 @@ topp_kernel(int rows, int N, int k, double p, const float* __restrict__ S, int32
   const int r0 = blockIdx.x * W + w;
   if (r0 >= rows) return;
   const float* s = S + (size_t)r0 * N;
-  float* slice = vals_s[w];
-  const Row row{&slice[lane], N, lane};
-  // Pass 1: stage the row; the exact max is needed before any mass.
+  const Row row{s + lane, N, lane};
+  // Pass 1: the exact max is needed before any mass.
   float v[VPT];
 #pragma unroll
   for (int i = 0; i < VPT; ++i) {
@@ -744,7 +751,7 @@ topp_kernel(int rows, int N, int k, double p, const float* __restrict__ S, int32
     const int j = lane + 32 * i;
     lo = fminf(lo, v[i]);
     hi = fmaxf(hi, v[i]);
-    if (j < N) slice[j] = v[i];
+    (void)j;
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
@@ -875,7 +882,7 @@ bsattn_status run_topk4(int rows, int N, int k, const float* S, int32_t* idx, in
 template <int VPT>
 bsattn_status run_topp(int rows, int N, int k, double p, const float* S, int32_t* idx, int32_t* cnt, int kmax,
                        cudaStream_t st) {
-  constexpr int W = Shape<VPT, true>::warps;
+  constexpr int W = ShapeP<VPT>::warps;
   topp_kernel<VPT><<<(rows + W - 1) / W, 32 * W, 0, st>>>(rows, N, k, p, S, idx, cnt, kmax);
   return cudaGetLastError() == cudaSuccess ? BSATTN_OK : BSATTN_ERR_CUDA;
 }
