@@ -501,6 +501,7 @@ def main():
     pk = peaks()
     # The backward of the same layer (rank 0; not part of the timed step).
     bwd = None if args.no_backward else backward_timing(bsattn, plan, wl, q, k, v, idx, cnt, flush, stream, pk)
+    routing = routing_timing(bsattn, plan, wl, q, k, flush, stream)
     configs = None
     if not args.no_configs and args.heads == 0:
         del q, k, v, o, ws
@@ -545,6 +546,7 @@ def main():
                      "traffic": measured_traffic(wl.name) if args.heads == 0 else None},
         "memory_kernels": memory_kernel_rates(wl, plan, comp, pk),
         "backward": bwd,
+        "routing": routing,
         "configs": configs,
         "e2e": e2e,
         "gpu_launches": launches_per_step(wl, plan) * args.steps,
@@ -690,6 +692,37 @@ def component_timing(bsattn, plan, wl, q, k, v, flush, stream, reps=20):
                 acc[n] += a.elapsed_time(b)
     out = {n: acc[n] / reps for n in names if acc[n] > 0}
     out["attention"] = out["attention_natural"]
+    return out
+
+
+def routing_timing(bsattn, plan, wl, q, k, flush, stream, reps=10):
+    """Pool + score + select of the layer's Q and K two ways (top-k plans):
+    attn_select (the score matrix written and read back) and
+    attn_select_fused (scores recomputed in three passes, never written).
+    Device time per call, L2 flushed before each, CUDA events."""
+    if wl.rule != "topk":
+        return None
+    ws = plan.workspace("select")
+    si, sc = plan.list_shapes()
+    idx = torch.empty(si, dtype=torch.int32, device="cuda")
+    cnt = torch.empty(sc, dtype=torch.int32, device="cuda")
+    out = {}
+    for name, fn in (("unfused_ms", lambda: bsattn.attn_select(plan, q, k, idx, cnt, ws, stream)),
+                     ("fused_ms", lambda: bsattn.attn_select_fused(plan, q, k, idx, cnt, ws, stream=stream))):
+        fn()
+        tot = 0.0
+        for _ in range(reps):
+            flush.fill_(1.0)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            torch.cuda.synchronize()
+            tot += a.elapsed_time(b)
+        out[name] = tot / reps
+    assert bsattn.attn_check_device_status(plan) == 0
+    out["note"] = ("pool + block scores + top-k through attn_select (S written and read back) "
+                   "and attn_select_fused (S recomputed three times on chip, never written)")
     return out
 
 

@@ -77,6 +77,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "attn_select_from_scores": [P, P, P, P, P],
         "attn_select": [P, P, P, P, P, P, Z, P],
         "attn_select_static": [P, P, P, P, P, P],
+        "attn_select_fused": [P, P, P, P, P, P, P, Z, P],
         "attn_quantize_e4m3": [P, P, P, P, P],
         "attn_forward": [P, P, P, P, P, P, P, P, P, P, P, Z, P],
         "attn_forward_natural": [P, P, P, P, P, P, P, P, P, P, P, Z, P],
@@ -102,7 +103,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
 _lib = load_library()
 EXPORTED = ("attn_plan_create", "attn_plan_destroy", "attn_plan_info", "attn_status_string",
             "attn_reorder", "attn_pool", "attn_unreorder", "attn_block_scores",
-            "attn_select_from_scores", "attn_select", "attn_select_static", "attn_quantize_e4m3",
+            "attn_select_from_scores", "attn_select", "attn_select_static", "attn_select_fused",
+            "attn_quantize_e4m3",
             "attn_forward", "attn_forward_natural",
             "attn_layer", "attn_check_device_status", "attn_schedule_create", "attn_schedule_destroy",
             "attn_schedule_plan", "attn_schedule_workspace_bytes", "attn_schedule_layer",
@@ -323,6 +325,19 @@ def attn_select(plan: Plan, q_nat, k_nat, idx, cnt, ws, stream=None):
     _want(cnt, torch.int32, sc, "cnt")
     _check(_lib.attn_select(plan.handle, _ptr(q_nat), _ptr(k_nat), _ptr(idx), _ptr(cnt), _ptr(ws),
                             ws.numel() * ws.element_size(), _stream(stream)), "attn_select")
+
+
+def attn_select_fused(plan: Plan, q_nat, k_nat, idx, cnt, ws, scores_debug=None, stream=None):
+    _want(q_nat, torch.bfloat16, plan.natural_shape(), "q_nat")
+    _want(k_nat, torch.bfloat16, plan.natural_shape(), "k_nat")
+    si, sc = plan.list_shapes()
+    _want(idx, torch.int32, si, "idx")
+    _want(cnt, torch.int32, sc, "cnt")
+    if scores_debug is not None:
+        _want(scores_debug, torch.float32, (plan.B, plan.heads, plan.N, plan.N), "scores_debug")
+    _check(_lib.attn_select_fused(plan.handle, _ptr(q_nat), _ptr(k_nat), _ptr(idx), _ptr(cnt),
+                                  _ptr(scores_debug), _ptr(ws), ws.numel() * ws.element_size(),
+                                  _stream(stream)), "attn_select_fused")
 
 
 STATIC_SELECT_SCRATCH_BYTES = 16 << 20

@@ -138,6 +138,15 @@ bsattn_status launch_block_scores(const Geom& g, const float* pq, const float* p
                                   float* S, int* err, cudaStream_t st);
 bsattn_status launch_select_topk(int rows, int N, int k, const float* S, int32_t* idx,
                                  int32_t* cnt, int kmax, cudaStream_t st);
+// Top-k of the rows listed in rlist[0, *rcount) only (rows <= total rows;
+// the count is read on the device).
+bsattn_status launch_select_topk_rows(int rows, int N, int k, const float* S, int32_t* idx, int32_t* cnt,
+                                      int kmax, const int32_t* rlist, const int* rcount, cudaStream_t st);
+// Fused block scores + top-k (S not materialised except for rows the fused
+// kernel hands to the row-wise fallback, or every row when debug_s).
+bsattn_status launch_fused_topk(const Geom& g, const float* pq, const float* pk, float scale, int k, int kmax,
+                                int32_t* idx, int32_t* cnt, float* S, bool debug_s, int32_t* fb_rows, int* fb_count,
+                                int* err, cudaStream_t st);
 bsattn_status launch_select_topp(int rows, int N, int k, double p, const float* S, int32_t* idx,
                                  int32_t* cnt, int kmax, cudaStream_t st);
 bsattn_status launch_broadcast_lists(int bh, int N, int kmax, const int32_t* src_idx,

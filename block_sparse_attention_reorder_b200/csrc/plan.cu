@@ -31,6 +31,8 @@ struct SelectWs {
   float* pq;
   float* pk;
   float* S;
+  int32_t* fb_rows;  // top-k: rows attn_select_fused hands to the row-wise selection
+  int* fb_count;
 };
 
 SelectWs carve_select(const bsattn_plan* p, Carve& c) {
@@ -39,6 +41,9 @@ SelectWs carve_select(const bsattn_plan* p, Carve& c) {
   w.pq = (float*)c.take(bh * p->N * p->desc.head_dim * sizeof(float));
   w.pk = (float*)c.take(bh * p->N * p->desc.head_dim * sizeof(float));
   w.S = (float*)c.take(bh * p->N * p->N * sizeof(float));
+  const bool topk = p->rule.kind == BSATTN_RULE_TOPK;
+  w.fb_rows = (int32_t*)c.take(topk ? bh * p->N * sizeof(int32_t) : 0);
+  w.fb_count = (int*)c.take(topk ? sizeof(int) : 0);
   return w;
 }
 
@@ -363,6 +368,29 @@ bsattn_status attn_select(const bsattn_plan* p, const void* q_nat, const void* k
   if ((s = launch_pool(g, (const __nv_bfloat16*)q_nat, w.pq, (const __nv_bfloat16*)k_nat, w.pk, st))) return s;
   if ((s = launch_block_scores(g, w.pq, w.pk, p->scale, w.S, p->d_err, st))) return s;
   return select_core(p, w.S, idx, cnt, st);
+}
+
+bsattn_status attn_select_fused(const bsattn_plan* p, const void* q_nat, const void* k_nat, int32_t* idx,
+                                int32_t* cnt, float* scores_debug, void* ws, size_t ws_bytes, void* stream) {
+  if (!p || !ok_ptr(idx) || !ok_ptr(cnt) || (scores_debug && !aligned16(scores_debug)))
+    return BSATTN_ERR_INVALID_ARG;
+  if (p->rule.kind == BSATTN_RULE_TOPP) return BSATTN_ERR_UNSUPPORTED;
+  bsattn_info info;
+  attn_plan_info(p, &info);
+  cudaStream_t st = (cudaStream_t)stream;
+  DeviceGuard dev(p->device);
+  if (dev.status) return dev.status;
+  bsattn_status s = BSATTN_OK;
+  if (p->rule.kind == BSATTN_RULE_WINDOW) return select_core(p, nullptr, idx, cnt, st);
+  if (!ok_ptr(q_nat) || !ok_ptr(k_nat)) return BSATTN_ERR_INVALID_ARG;
+  if (!ws || !aligned16(ws) || ws_bytes < info.select_workspace_bytes) return BSATTN_ERR_WORKSPACE;
+  Carve c(ws);
+  SelectWs w = carve_select(p, c);
+  Geom g = make_geom(p);
+  if ((s = launch_pool(g, (const __nv_bfloat16*)q_nat, w.pq, (const __nv_bfloat16*)k_nat, w.pk, st))) return s;
+  return launch_fused_topk(g, w.pq, w.pk, p->scale, p->rule.k, p->kmax, idx, cnt,
+                           scores_debug ? scores_debug : w.S, scores_debug != nullptr, w.fb_rows, w.fb_count,
+                           p->d_err, st);
 }
 
 bsattn_status attn_quantize_e4m3(const bsattn_plan* p, const void* x_tiled, uint8_t* codes,

@@ -23,6 +23,18 @@
 // Every block is accumulated in the same order (slices ascending, then the
 // 8-wide K steps, hi*hi, hi*lo, lo*hi), so the result does not depend on how
 // blocks are shared among CTAs.
+//
+// Fused score + top-k (FUSED): S is never written. A CTA takes whole 128-row
+// blocks of S and computes every block of the row three times, with the same
+// products in the same order as above (so every score is bit-identical to
+// the materialised S); the epilogue threads (thread = row) select on the
+// fly: pass 0 the row's exact min and max, pass 1 a 128-bin histogram over
+// that range, pass 2 the tiles above the bin where the count from the top
+// reaches k (written to the list in ascending order) and the tiles of that
+// bin as 64-bit keys, ranked exactly at the end and merged into the list. A
+// row whose boundary bin holds more than 32 tiles (runs of equal scores, a
+// constant or non-finite row) writes its S row in pass 2 instead and is
+// handed, through a row list, to the row-wise top-k kernel.
 #include "internal.h"
 #include "tc_common.cuh"
 
@@ -31,23 +43,30 @@ namespace {
 constexpr int kRows = 128;                       // output block edge (M = N = 128)
 constexpr int kSlice = 32;                       // fp32 columns of D per slice (128 bytes)
 constexpr int kSliceBytes = kRows * kSlice * 4;  // 16 KB per operand slice
-constexpr int kStages = 4;                       // Pk slice ring
 constexpr int kThreads = 320;
 constexpr int kSplitThreads = 128;
 constexpr int kEpiBytes = 32 * 128;              // one warp's 32 x 32 transpose buffer
 constexpr long long kWaitLimit = 4000000000LL;   // SM cycles (~2 s)
 
-template <int D>
+constexpr int kFusedPasses = 3;                  // min/max, histogram, collect
+constexpr int kFusedBins = 128;
+constexpr int kFusedCand = 32;                   // boundary-bin tiles ranked in the kernel
+
+template <int D, bool FUSED>
 struct ScoresCfg {
+  static constexpr int STAGES = FUSED ? 3 : 4;            // Pk slice ring
   static constexpr int KS = D / kSlice;                   // slices per block
   static constexpr int OFF_ASTG = 0;                      // Pq block staging, KS slices
   static constexpr int OFF_RING = KS * kSliceBytes;       // stage s: Pk hi, then Pk lo
   static constexpr int STAGE = 2 * kSliceBytes;
-  static constexpr int OFF_EPI = OFF_RING + kStages * STAGE;
-  static constexpr int OFF_BAR = OFF_EPI + 4 * kEpiBytes;
+  static constexpr int OFF_EPI = OFF_RING + STAGES * STAGE;
+  // Epilogue: the transpose buffers, or (fused) per-row state: a 16-bit
+  // histogram [bin][row] and the boundary-bin keys [slot][row].
+  static constexpr int EPI_BYTES = FUSED ? kFusedBins * kRows * 2 + kFusedCand * kRows * 8 : 4 * kEpiBytes;
+  static constexpr int OFF_BAR = OFF_EPI + EPI_BYTES;
   // a_full, a_stage_free, a_split, a_free, b_full[S], b_split[S], b_empty[S], acc_full[2],
   // acc_empty[2], final
-  static constexpr int NBAR = 4 + 3 * kStages + 4 + 1;
+  static constexpr int NBAR = 4 + 3 * STAGES + 4 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;     // TMEM base, abort flag, a word that stays 0
   static constexpr int SMEM = OFF_MISC + 16 + 1024;       // + alignment slack
   // TMEM columns: Pq hi [0, D), Pq lo [D, 2D), accumulators at 2D and 2D + 128.
@@ -61,9 +80,23 @@ struct ScoresParams {
   int nb;             // 128-row blocks per (batch, head)
   long long blocks;   // B * Hh * nb * nb
   float scale;
-  float* S;
+  float* S;           // fused: rows handed to the fallback (every row when debug_s)
   int* err;
+  // fused top-k only
+  long long rblocks;  // B * Hh * nb row blocks
+  int k, kmax;
+  int32_t* idx;
+  int32_t* cnt;
+  int debug_s;        // 1: every row's S is written as well
+  int32_t* fb_rows;   // rows for the row-wise fallback, *fb_count of them
+  int* fb_count;
 };
+
+__device__ __forceinline__ uint32_t fused_order_key(float x) {
+  uint32_t u = __float_as_uint(x);
+  if (u == 0x80000000u) u = 0u;  // -0.0 ties with +0.0
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
 
 // D[tmem] (+)= A[tmem] * B[smem desc], TF32 operands.
 __device__ __forceinline__ void mma_ts_tf32(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc,
@@ -97,11 +130,12 @@ __device__ __forceinline__ void split_slice(uint8_t* hi, int t) {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-template <int D>
+template <int D, bool FUSED>
 __global__ void __launch_bounds__(kThreads, 1)
 block_scores_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                        ScoresParams P) {
-  using C = ScoresCfg<D>;
+  using C = ScoresCfg<D, FUSED>;
+  constexpr int kStages = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -118,10 +152,13 @@ block_scores_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
   volatile int* never = reinterpret_cast<volatile int*>(misc + 2);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // This CTA's contiguous run of blocks; block = ((bh * nb) + bi) * nb + bj.
-  const long long blk0 = P.blocks * blockIdx.x / gridDim.x;
-  const long long blk1 = P.blocks * (blockIdx.x + 1) / gridDim.x;
+  // This CTA's contiguous run of blocks; block = ((bh * nb) + bi) * PN + pass * nb + bj
+  // (fused: whole row blocks, each computed in kFusedPasses passes; else one pass).
   const int nb = P.nb;
+  const int PN = (FUSED ? kFusedPasses : 1) * nb;
+  const long long blk0 = FUSED ? P.rblocks * blockIdx.x / gridDim.x * PN : P.blocks * blockIdx.x / gridDim.x;
+  const long long blk1 =
+      FUSED ? P.rblocks * (blockIdx.x + 1) / gridDim.x * PN : P.blocks * (blockIdx.x + 1) / gridDim.x;
 
   if (tid == 0) {
     tc::mbar_init(bar_afull, 1);
@@ -161,7 +198,7 @@ block_scores_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
       for (int s = 0; s < kStages; ++s) last_b[s] = -1;
       bool ok = true;
       for (long long blk = blk0; ok && blk < blk1; ++blk) {
-        const long long rk = blk / nb, bh = rk / nb;
+        const long long rk = blk / PN, bh = rk / nb;
         const int bi = (int)(rk % nb), bj = (int)(blk % nb);
         if (rk != prev) {
           // The split warps must have read the previous Pq block out of staging.
@@ -207,7 +244,7 @@ block_scores_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
       int arow = 0, t = 0;
       bool ok = true;
       for (long long blk = blk0; ok && blk < blk1; ++blk, ++t) {
-        const long long rk = blk / nb;
+        const long long rk = blk / PN;
         if (rk != prev) {
           if (!tc::mbar_wait(bar_asplit, arow & 1, abort_flag, kWaitLimit)) {
             ok = false;
@@ -246,7 +283,7 @@ block_scores_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
         tc::mma_commit(bar_accfull(a));
         // Pq columns of TMEM are rewritten for the next row block only after
         // this one's MMAs are done.
-        if (blk + 1 < blk1 && (blk + 1) / nb != rk) tc::mma_commit(bar_afree);
+        if (blk + 1 < blk1 && (blk + 1) / PN != rk) tc::mma_commit(bar_afree);
       }
       if (!ok) {
         *abort_flag = 1;
@@ -264,7 +301,7 @@ block_scores_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
     int arow = 0;
     bool ok = true;
     for (long long blk = blk0; ok && blk < blk1; ++blk) {
-      const long long rk = blk / nb;
+      const long long rk = blk / PN;
       if (rk != prev) {
         if (!__all_sync(0xffffffffu, tc::mbar_wait(bar_afull, arow & 1, abort_flag, kWaitLimit)) ||
             (arow > 0 && !__all_sync(0xffffffffu, tc::mbar_wait(bar_afree, (arow - 1) & 1, abort_flag, kWaitLimit)))) {
@@ -306,6 +343,167 @@ block_scores_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
         }
         split_slice(smem + C::OFF_RING + s * C::STAGE, t);
         tc::mbar_arrive(bar_bsplit(s));
+      }
+    }
+    if (!ok) {
+      *abort_flag = 1;
+      if (lane == 0) atomicOr(P.err, BSATTN_DEVERR_TIMEOUT);
+    }
+  } else if constexpr (FUSED) {
+    // ------------------------------------------------------------ fused top-k epilogue
+    // Thread r owns row r of the current 128-row block (TMEM lane r).
+    const int r = tid;
+    uint16_t* hist = reinterpret_cast<uint16_t*>(smem + C::OFF_EPI);  // [bin][row]
+    uint64_t* cand = reinterpret_cast<uint64_t*>(smem + C::OFF_EPI + kFusedBins * kRows * 2);  // [slot][row]
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23: bin index in the low mantissa bits
+    const float qnan = __int_as_float(0x7fc00000);
+    const int rr = min(P.k, P.N);
+    float mn = qnan, mx = qnan, sc = 0.f, offm = kMagic;
+    int bstar = -1, need = 0, outpos = 0, ncand = 0;
+    bool crowded = false;
+    // Equal-width bins over [mn, mx], monotone in the score (one FMA; NaN and
+    // a range that overflows land in bin 0).
+    auto bin_of = [&](float x) -> int {
+      const float u = fminf(fmaxf(fmaf(x, sc, offm), kMagic), kMagic + (float)(kFusedBins - 1));
+      return __float_as_int(u) - __float_as_int(kMagic);
+    };
+    int t = 0;
+    bool ok = true;
+    for (long long blk = blk0; blk < blk1; ++blk, ++t) {
+      const int a = t & 1;
+      if (!__all_sync(0xffffffffu, tc::mbar_wait(bar_accfull(a), (t >> 1) & 1, abort_flag, kWaitLimit))) {
+        ok = false;
+        break;
+      }
+      tc::fence_after_sync();
+      const long long rk = blk / PN, bh = rk / nb;
+      const int pass = (int)((blk / nb) % kFusedPasses), bj = (int)(blk % nb);
+      const int i = (int)(rk % nb) * kRows + r;  // this thread's row within its (batch, head)
+      const bool row_ok = i < P.N;
+      const size_t grow = (size_t)bh * P.N + i;  // row of the whole score matrix
+      if (bj == 0 && pass == 0) {
+        mn = mx = qnan;
+        crowded = false;
+      }
+      if (bj == 0 && pass == 1) {
+        // A constant or non-finite row has no range to bin: fallback.
+        crowded = !(mn < mx) || !(mx - mn <= 3.0e38f);
+        sc = crowded ? 0.f : (float)kFusedBins / (mx - mn);
+        if (!(sc <= 3.0e38f)) crowded = true;
+        if (crowded) sc = 0.f;
+        offm = crowded ? kMagic : fmaf(-mn, sc, kMagic);
+        for (int q = 0; q < kFusedBins; ++q) hist[q * kRows + r] = 0;
+      }
+      if (bj == 0 && pass == 2) {
+        // The bin in which the count, taken from the top bin down, reaches rr.
+        int run = 0;
+        bstar = -1;
+        for (int q = kFusedBins - 1; q >= 0; --q) {
+          const int c = hist[q * kRows + r];
+          if (run + c >= rr) {
+            bstar = q;
+            need = rr - run;
+            crowded = crowded || c > kFusedCand;
+            break;
+          }
+          run += c;
+        }
+        if (bstar < 0) crowded = true;
+        outpos = 0;
+        ncand = 0;
+      }
+      int32_t* out = P.idx + grow * P.kmax;
+      float* srow = P.S + grow * P.N;
+      // One straight-line loop per pass over 32 columns at a time (the
+      // columns past N are masked, not branched out of).
+#pragma unroll 1
+      for (int c0 = 0; c0 < kRows; c0 += 32) {
+        uint32_t v[32];
+        tc::tmem_ld32_wait(tmem + lane_base + C::COL_ACC + (uint32_t)(a * kRows + c0), v);
+        const int j0 = bj * kRows + c0;
+        const int jn = row_ok ? min(32, P.N - j0) : 0;  // valid columns of this piece
+        if (pass == 0) {
+          float lo = mn, hi = mx;
+#pragma unroll
+          for (int q = 0; q < 32; ++q) {
+            const float x = q < jn ? __uint_as_float(v[q]) * P.scale : qnan;
+            lo = fminf(lo, x);
+            hi = fmaxf(hi, x);
+          }
+          mn = lo;
+          mx = hi;
+        } else if (pass == 1) {
+          if (!crowded) {
+#pragma unroll
+            for (int q = 0; q < 32; ++q)
+              if (q < jn) ++hist[bin_of(__uint_as_float(v[q]) * P.scale) * kRows + r];
+          }
+        } else if (jn > 0) {
+          if (crowded || P.debug_s) {
+#pragma unroll
+            for (int q = 0; q < 32; ++q)
+              if (q < jn) srow[j0 + q] = __uint_as_float(v[q]) * P.scale;
+          }
+          if (!crowded) {
+#pragma unroll
+            for (int q = 0; q < 32; ++q) {
+              const float x = __uint_as_float(v[q]) * P.scale;
+              const int bx = q < jn ? bin_of(x) : -1;
+              if (bx > bstar) {
+                if (outpos < P.kmax) out[outpos] = j0 + q;
+                ++outpos;
+              } else if (bx == bstar) {
+                if (ncand < kFusedCand)
+                  cand[ncand * kRows + r] =
+                      ((uint64_t)fused_order_key(x) << 32) | (uint64_t)(0xffffffffu - (uint32_t)(j0 + q));
+                ++ncand;
+              }
+            }
+          }
+        }
+      }
+      tc::fence_before_sync();
+      tc::mbar_arrive(bar_accempty(a));
+      if (pass == kFusedPasses - 1 && bj == nb - 1 && row_ok) {
+        if (crowded) {
+          P.fb_rows[atomicAdd(P.fb_count, 1)] = (int32_t)grow;
+        } else {
+          // The boundary bin's keys are unique; the `need` largest are kept.
+          // Their tile indices, ascending, go into the histogram's column r
+          // (free now) and are merged behind the tiles above the bin.
+          uint16_t* kept = hist + r;
+          const int nc = min(ncand, kFusedCand);
+          int nk = 0;
+          for (int x1 = 0; x1 < nc; ++x1) {
+            const uint64_t kx = cand[x1 * kRows + r];
+            int rank = 0;
+            for (int x2 = 0; x2 < nc; ++x2) rank += cand[x2 * kRows + r] > kx ? 1 : 0;
+            if (rank < need) {
+              const uint16_t jj = (uint16_t)(0xffffffffu - (uint32_t)kx);
+              int pos = nk++;
+              while (pos > 0 && kept[(pos - 1) * kRows] > jj) {
+                kept[pos * kRows] = kept[(pos - 1) * kRows];
+                --pos;
+              }
+              kept[pos * kRows] = jj;
+            }
+          }
+          const int na = min(outpos, P.kmax), total = min(na + nk, P.kmax);
+          int ia = na - 1, ib = nk - 1;
+          for (int wpos = total - 1; wpos >= 0 && ib >= 0; --wpos) {
+            const int ja = ia >= 0 ? out[ia] : -1;
+            const int jb = kept[ib * kRows];
+            if (ja > jb) {
+              out[wpos] = ja;
+              --ia;
+            } else {
+              out[wpos] = jb;
+              --ib;
+            }
+          }
+          P.cnt[grow] = total;
+        }
       }
     }
     if (!ok) {
@@ -376,10 +574,20 @@ block_scores_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
   }
 }
 
-template <int D>
+// The fused top-k's outputs (FUSED kernels only).
+struct FusedArgs {
+  int k, kmax;
+  int32_t* idx;
+  int32_t* cnt;
+  int debug_s;
+  int32_t* fb_rows;
+  int* fb_count;
+};
+
+template <int D, bool FUSED>
 bsattn_status run_scores(const Geom& g, const float* pq, const float* pk, float scale, float* S, int* err,
-                         cudaStream_t st) {
-  using C = ScoresCfg<D>;
+                         const FusedArgs* fa, cudaStream_t st) {
+  using C = ScoresCfg<D, FUSED>;
   const uint64_t rows = (uint64_t)g.B * g.Hh * g.N;
   CUtensorMap ma, mb;
   if (!bsattn_make_map_2d(&ma, pq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, D, rows, kSlice, kRows,
@@ -387,21 +595,32 @@ bsattn_status run_scores(const Geom& g, const float* pq, const float* pk, float 
       !bsattn_make_map_2d(&mb, pk, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, D, rows, kSlice, kRows,
                           CU_TENSOR_MAP_SWIZZLE_128B))
     return BSATTN_ERR_CUDA;
-  auto kern = block_scores_tc_kernel<D>;
+  auto kern = block_scores_tc_kernel<D, FUSED>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
     return BSATTN_ERR_CUDA;
   int dev = 0, sms = 0;
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
     return BSATTN_ERR_CUDA;
-  ScoresParams prm;
+  ScoresParams prm{};
   prm.N = g.N;
   prm.nb = (g.N + kRows - 1) / kRows;
   prm.blocks = (long long)g.B * g.Hh * prm.nb * prm.nb;
+  prm.rblocks = (long long)g.B * g.Hh * prm.nb;
   prm.scale = scale;
   prm.S = S;
   prm.err = err;
-  const int grid = (int)(prm.blocks < sms ? prm.blocks : sms);
+  if (FUSED) {
+    prm.k = fa->k;
+    prm.kmax = fa->kmax;
+    prm.idx = fa->idx;
+    prm.cnt = fa->cnt;
+    prm.debug_s = fa->debug_s;
+    prm.fb_rows = fa->fb_rows;
+    prm.fb_count = fa->fb_count;
+  }
+  const long long units = FUSED ? prm.rblocks : prm.blocks;  // fused CTAs take whole row blocks
+  const int grid = (int)(units < sms ? units : sms);
   kern<<<grid, kThreads, C::SMEM, st>>>(ma, mb, prm);
   return cudaGetLastError() == cudaSuccess ? BSATTN_OK : BSATTN_ERR_CUDA;
 }
@@ -413,6 +632,20 @@ bsattn_status launch_block_scores(const Geom& g, const float* pq, const float* p
   // Row coordinates of the tensor maps (B * Hh * N rows, plus a block) stay in int32.
   if ((uint64_t)g.B * g.Hh * g.N + kRows >= (1ull << 31)) return BSATTN_ERR_UNSUPPORTED;
   if (g.B <= 0 || g.Hh <= 0 || g.N <= 0) return BSATTN_OK;
-  return g.D == 128 ? run_scores<128>(g, pq, pk, scale, S, err, st)
-                    : run_scores<64>(g, pq, pk, scale, S, err, st);
+  return g.D == 128 ? run_scores<128, false>(g, pq, pk, scale, S, err, nullptr, st)
+                    : run_scores<64, false>(g, pq, pk, scale, S, err, nullptr, st);
+}
+
+bsattn_status launch_fused_topk(const Geom& g, const float* pq, const float* pk, float scale, int k, int kmax,
+                                int32_t* idx, int32_t* cnt, float* S, bool debug_s, int32_t* fb_rows, int* fb_count,
+                                int* err, cudaStream_t st) {
+  if ((uint64_t)g.B * g.Hh * g.N + kRows >= (1ull << 31)) return BSATTN_ERR_UNSUPPORTED;
+  if (g.B <= 0 || g.Hh <= 0 || g.N <= 0) return BSATTN_OK;
+  if (cudaMemsetAsync(fb_count, 0, sizeof(int), st) != cudaSuccess) return BSATTN_ERR_CUDA;
+  const FusedArgs fa{k, kmax, idx, cnt, debug_s ? 1 : 0, fb_rows, fb_count};
+  bsattn_status s = g.D == 128 ? run_scores<128, true>(g, pq, pk, scale, S, err, &fa, st)
+                               : run_scores<64, true>(g, pq, pk, scale, S, err, &fa, st);
+  if (s != BSATTN_OK) return s;
+  // Rows the kernel could not settle: the row-wise top-k over their S rows.
+  return launch_select_topk_rows((int)((uint64_t)g.B * g.Hh * g.N), g.N, k, S, idx, cnt, kmax, fb_rows, fb_count, st);
 }

@@ -422,15 +422,23 @@ struct Shape {
 template <int VPT>
 __global__ void __launch_bounds__(32 * Shape<VPT, false>::warps)
 topk_kernel(int rows, int N, int k, const float* __restrict__ S, int32_t* __restrict__ idx,
-            int32_t* __restrict__ cnt, int kmax) {
+            int32_t* __restrict__ cnt, int kmax, const int32_t* __restrict__ rlist,
+            const int* __restrict__ rcount) {
   constexpr int W = Shape<VPT, false>::warps;
   __shared__ float vals_s[W][32 * VPT];
   __shared__ uint32_t hcnt_s[W][kBins];
   __shared__ uint32_t mask_s[W][VPT];
   __shared__ uint64_t cand_s[W][kCand];
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int r0 = blockIdx.x * W + w;
-  if (r0 >= rows) return;
+  // With a row list, warp x takes the list's x-th row (the list's length is
+  // read on the device); otherwise row x.
+  int r0 = blockIdx.x * W + w;
+  if (rlist) {
+    if (r0 >= *rcount) return;
+    r0 = rlist[r0];
+  } else if (r0 >= rows) {
+    return;
+  }
   const float* s = S + (size_t)r0 * N;
   float* slice = vals_s[w];
   uint32_t* hist = hcnt_s[w];
@@ -567,7 +575,8 @@ struct Shape4 {
 template <int C4>
 __global__ void __launch_bounds__(32 * Shape4<C4>::warps)
 topk4_kernel(int rows, int N, int k, const float* __restrict__ S, int32_t* __restrict__ idx,
-             int32_t* __restrict__ cnt, int kmax) {
+             int32_t* __restrict__ cnt, int kmax, const int32_t* __restrict__ rlist,
+             const int* __restrict__ rcount) {
   constexpr int W = Shape4<C4>::warps, VPT = 4 * C4;
   __shared__ uint32_t bins_s[W][32 * C4];
   __shared__ uint32_t gt_s[W][4 * C4];
@@ -575,8 +584,15 @@ topk4_kernel(int rows, int N, int k, const float* __restrict__ S, int32_t* __res
   __shared__ uint32_t hcnt_s[W][kBins];
   __shared__ uint64_t cand_s[W][kCand];
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int r0 = blockIdx.x * W + w;
-  if (r0 >= rows) return;
+  // With a row list, warp x takes the list's x-th row (the list's length is
+  // read on the device); otherwise row x.
+  int r0 = blockIdx.x * W + w;
+  if (rlist) {
+    if (r0 >= *rcount) return;
+    r0 = rlist[r0];
+  } else if (r0 >= rows) {
+    return;
+  }
   const float* s = S + (size_t)r0 * N;
   uint32_t* hist = hcnt_s[w];
   const float qnan = __int_as_float(0x7fc00000);
@@ -865,17 +881,17 @@ __global__ void broadcast_lists_kernel(int N, int kmax, const int32_t* __restric
 
 template <int VPT>
 bsattn_status run_topk(int rows, int N, int k, const float* S, int32_t* idx, int32_t* cnt, int kmax,
-                       cudaStream_t st) {
+                       const int32_t* rlist, const int* rcount, cudaStream_t st) {
   constexpr int W = Shape<VPT, false>::warps;
-  topk_kernel<VPT><<<(rows + W - 1) / W, 32 * W, 0, st>>>(rows, N, k, S, idx, cnt, kmax);
+  topk_kernel<VPT><<<(rows + W - 1) / W, 32 * W, 0, st>>>(rows, N, k, S, idx, cnt, kmax, rlist, rcount);
   return cudaGetLastError() == cudaSuccess ? BSATTN_OK : BSATTN_ERR_CUDA;
 }
 
 template <int C4>
 bsattn_status run_topk4(int rows, int N, int k, const float* S, int32_t* idx, int32_t* cnt, int kmax,
-                        cudaStream_t st) {
+                        const int32_t* rlist, const int* rcount, cudaStream_t st) {
   constexpr int W = Shape4<C4>::warps;
-  topk4_kernel<C4><<<(rows + W - 1) / W, 32 * W, 0, st>>>(rows, N, k, S, idx, cnt, kmax);
+  topk4_kernel<C4><<<(rows + W - 1) / W, 32 * W, 0, st>>>(rows, N, k, S, idx, cnt, kmax, rlist, rcount);
   return cudaGetLastError() == cudaSuccess ? BSATTN_OK : BSATTN_ERR_CUDA;
 }
 
@@ -889,32 +905,37 @@ bsattn_status run_topp(int rows, int N, int k, double p, const float* S, int32_t
 
 }  // namespace
 
-bsattn_status launch_select_topk(int rows, int N, int k, const float* S, int32_t* idx, int32_t* cnt, int kmax,
-                                 cudaStream_t st) {
+bsattn_status launch_select_topk_rows(int rows, int N, int k, const float* S, int32_t* idx, int32_t* cnt,
+                                      int kmax, const int32_t* rlist, const int* rcount, cudaStream_t st) {
   if (rows <= 0 || N <= 0) return BSATTN_OK;
   if (N % 4 == 0 && N >= 128 && ((uintptr_t)S & 15u) == 0) {
     const int c4 = (N + 127) / 128;
-    if (c4 <= 1) return run_topk4<1>(rows, N, k, S, idx, cnt, kmax, st);
-    if (c4 <= 2) return run_topk4<2>(rows, N, k, S, idx, cnt, kmax, st);
-    if (c4 <= 3) return run_topk4<3>(rows, N, k, S, idx, cnt, kmax, st);
-    if (c4 <= 4) return run_topk4<4>(rows, N, k, S, idx, cnt, kmax, st);
-    if (c4 <= 6) return run_topk4<6>(rows, N, k, S, idx, cnt, kmax, st);
-    if (c4 <= 8) return run_topk4<8>(rows, N, k, S, idx, cnt, kmax, st);
-    if (c4 <= 12) return run_topk4<12>(rows, N, k, S, idx, cnt, kmax, st);
-    if (c4 <= 16) return run_topk4<16>(rows, N, k, S, idx, cnt, kmax, st);
+    if (c4 <= 1) return run_topk4<1>(rows, N, k, S, idx, cnt, kmax, rlist, rcount, st);
+    if (c4 <= 2) return run_topk4<2>(rows, N, k, S, idx, cnt, kmax, rlist, rcount, st);
+    if (c4 <= 3) return run_topk4<3>(rows, N, k, S, idx, cnt, kmax, rlist, rcount, st);
+    if (c4 <= 4) return run_topk4<4>(rows, N, k, S, idx, cnt, kmax, rlist, rcount, st);
+    if (c4 <= 6) return run_topk4<6>(rows, N, k, S, idx, cnt, kmax, rlist, rcount, st);
+    if (c4 <= 8) return run_topk4<8>(rows, N, k, S, idx, cnt, kmax, rlist, rcount, st);
+    if (c4 <= 12) return run_topk4<12>(rows, N, k, S, idx, cnt, kmax, rlist, rcount, st);
+    if (c4 <= 16) return run_topk4<16>(rows, N, k, S, idx, cnt, kmax, rlist, rcount, st);
   }
   const int vpt = (N + 31) / 32;
-  if (vpt <= 1) return run_topk<1>(rows, N, k, S, idx, cnt, kmax, st);
-  if (vpt <= 2) return run_topk<2>(rows, N, k, S, idx, cnt, kmax, st);
-  if (vpt <= 4) return run_topk<4>(rows, N, k, S, idx, cnt, kmax, st);
-  if (vpt <= 8) return run_topk<8>(rows, N, k, S, idx, cnt, kmax, st);
-  if (vpt <= 12) return run_topk<12>(rows, N, k, S, idx, cnt, kmax, st);
-  if (vpt <= 16) return run_topk<16>(rows, N, k, S, idx, cnt, kmax, st);
-  if (vpt <= 24) return run_topk<24>(rows, N, k, S, idx, cnt, kmax, st);
-  if (vpt <= 32) return run_topk<32>(rows, N, k, S, idx, cnt, kmax, st);
-  if (vpt <= 48) return run_topk<48>(rows, N, k, S, idx, cnt, kmax, st);
-  if (vpt <= 64) return run_topk<64>(rows, N, k, S, idx, cnt, kmax, st);
+  if (vpt <= 1) return run_topk<1>(rows, N, k, S, idx, cnt, kmax, rlist, rcount, st);
+  if (vpt <= 2) return run_topk<2>(rows, N, k, S, idx, cnt, kmax, rlist, rcount, st);
+  if (vpt <= 4) return run_topk<4>(rows, N, k, S, idx, cnt, kmax, rlist, rcount, st);
+  if (vpt <= 8) return run_topk<8>(rows, N, k, S, idx, cnt, kmax, rlist, rcount, st);
+  if (vpt <= 12) return run_topk<12>(rows, N, k, S, idx, cnt, kmax, rlist, rcount, st);
+  if (vpt <= 16) return run_topk<16>(rows, N, k, S, idx, cnt, kmax, rlist, rcount, st);
+  if (vpt <= 24) return run_topk<24>(rows, N, k, S, idx, cnt, kmax, rlist, rcount, st);
+  if (vpt <= 32) return run_topk<32>(rows, N, k, S, idx, cnt, kmax, rlist, rcount, st);
+  if (vpt <= 48) return run_topk<48>(rows, N, k, S, idx, cnt, kmax, rlist, rcount, st);
+  if (vpt <= 64) return run_topk<64>(rows, N, k, S, idx, cnt, kmax, rlist, rcount, st);
   return BSATTN_ERR_UNSUPPORTED;
+}
+
+bsattn_status launch_select_topk(int rows, int N, int k, const float* S, int32_t* idx, int32_t* cnt, int kmax,
+                                 cudaStream_t st) {
+  return launch_select_topk_rows(rows, N, k, S, idx, cnt, kmax, nullptr, nullptr, st);
 }
 
 bsattn_status launch_select_topp(int rows, int N, int k, double p, const float* S, int32_t* idx, int32_t* cnt,

@@ -186,6 +186,24 @@ bsattn_status attn_select(const bsattn_plan* plan, const void* q_nat, const void
                           int32_t* idx, int32_t* cnt, void* ws, size_t ws_bytes,
                           void* stream);
 
+/* attn_select with the scoring and the top-k selection fused (the same
+ * routing frontend, FVAttn summary page, Summary, and the same top-k rule as
+ * attn_select_from_scores): the score matrix is not written. The kernel
+ * computes each 128-row block of S three times with the products and order
+ * of attn_block_scores (every score bit-identical) and selects per row on
+ * the fly; a row it cannot settle in three passes (more than 32 tiles in the
+ * bin where its k-th largest score falls: runs of equal scores, a constant
+ * or non-finite row) has its S row written to the workspace and is selected
+ * by the row-wise kernel afterwards. Results equal attn_select's for the
+ * same inputs. Top-k plans; the window rule as attn_select; top-p plans:
+ * BSATTN_ERR_UNSUPPORTED. `ws` as for attn_select (info.select_workspace_bytes
+ * also covers this call's list of rows to settle). scores_debug, if
+ * non-NULL (16-byte aligned, [B, Hh, N, N] fp32), receives every row of S
+ * as attn_block_scores writes it. */
+bsattn_status attn_select_fused(const bsattn_plan* plan, const void* q_nat, const void* k_nat,
+                                int32_t* idx, int32_t* cnt, float* scores_debug, void* ws,
+                                size_t ws_bytes, void* stream);
+
 /* Capacity of the library-owned scratch used by attn_select_static. */
 #define BSATTN_STATIC_SELECT_SCRATCH_BYTES (16u << 20)
 
