@@ -104,6 +104,7 @@ reorder_kernel(Geom g, const __nv_bfloat16* __restrict__ x_nat, __nv_bfloat16* _
   constexpr int ITER = 64 * CH / kThreads;  // chunks per thread
   constexpr int RSTEP = kThreads / CH;      // row stride between a thread's chunks
   __shared__ float wred[kThreads / 32];
+  __shared__ int rowtok[64];  // token of each row of the chunk, -1 for a padded slot
 
   const int j = blockIdx.x / g.nchunk, head = blockIdx.y, b = blockIdx.z;
   const int c = threadIdx.x % CH;
@@ -111,12 +112,16 @@ reorder_kernel(Geom g, const __nv_bfloat16* __restrict__ x_nat, __nv_bfloat16* _
   const TileCoord tc = tile_coord(g, j);
   const int row0 = 64 * (blockIdx.x % g.nchunk);  // first in-tile row of the chunk
   const size_t tile_off = (((size_t)b * g.Hh + head) * g.N + j) * g.V + row0;
+  // Each row's token once per CTA: the CH threads of a row would otherwise
+  // all repeat its integer divisions.
+  if (threadIdx.x < 64) rowtok[threadIdx.x] = row_token(g, tc, row0 + threadIdx.x);
+  __syncthreads();
 
   uint4 v[ITER];
 #pragma unroll
   for (int i = 0; i < ITER; ++i) {
     int r = r0 + RSTEP * i;
-    int n = row_token(g, tc, row0 + r);
+    int n = rowtok[r];
     if (n >= 0) {
       const uint4* src = reinterpret_cast<const uint4*>(x_nat + (((size_t)b * g.L + n) * g.Hh + head) * D) + c;
       v[i] = __ldg(src);
@@ -159,22 +164,25 @@ unreorder_kernel(Geom g, const __nv_bfloat16* __restrict__ x_tiled, __nv_bfloat1
   constexpr int CH = D / 8;
   constexpr int ITER = 64 * CH / kThreads;
   constexpr int RSTEP = kThreads / CH;
+  __shared__ int rowtok[64];  // token of each row of the chunk, -1 for a padded slot
   const int j = blockIdx.x / g.nchunk, head = blockIdx.y, b = blockIdx.z;
   const int c = threadIdx.x % CH;
   const int r0 = threadIdx.x / CH;
   const TileCoord tc = tile_coord(g, j);
   const int row0 = 64 * (blockIdx.x % g.nchunk);
   const size_t tile_off = (((size_t)b * g.Hh + head) * g.N + j) * g.V + row0;
+  if (threadIdx.x < 64) rowtok[threadIdx.x] = row_token(g, tc, row0 + threadIdx.x);
+  __syncthreads();
 #pragma unroll
   for (int i = 0; i < ITER; ++i) {
     int r = r0 + RSTEP * i;
-    int n = row_token(g, tc, row0 + r);
+    int n = rowtok[r];
     if (n < 0) continue;
     uint4 v = __ldg(reinterpret_cast<const uint4*>(x_tiled + (tile_off + r) * D) + c);
     reinterpret_cast<uint4*>(x_nat + (((size_t)b * g.L + n) * g.Hh + head) * D)[c] = v;
   }
   if (lse_tiled && threadIdx.x < 64) {
-    int n = row_token(g, tc, row0 + threadIdx.x);
+    int n = rowtok[threadIdx.x];
     if (n >= 0) lse_nat[((size_t)b * g.Hh + head) * g.L + n] = lse_tiled[tile_off + threadIdx.x];
   }
 }
