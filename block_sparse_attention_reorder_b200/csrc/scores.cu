@@ -29,9 +29,9 @@
 // products in the same order as above (so every score is bit-identical to
 // the materialised S); the epilogue threads (thread = row) select on the
 // fly: pass 0 the row's exact min and max, pass 1 a 128-bin histogram over
-// that range, pass 2 the tiles above the bin where the count from the top
-// reaches k (written to the list in ascending order) and the tiles of that
-// bin as 64-bit keys, ranked exactly at the end and merged into the list. A
+// that range, pass 2 a bit mask of the tiles above the bin where the count
+// from the top reaches k and the tiles of that bin as 64-bit keys, ranked
+// exactly at the end; their bits join the mask, written out ascending. A
 // row whose boundary bin holds more than 32 tiles (runs of equal scores, a
 // constant or non-finite row) writes its S row in pass 2 instead and is
 // handed, through a row list, to the row-wise top-k kernel.
@@ -51,6 +51,10 @@ constexpr long long kWaitLimit = 4000000000LL;   // SM cycles (~2 s)
 constexpr int kFusedPasses = 3;                  // min/max, histogram, collect
 constexpr int kFusedBins = 128;
 constexpr int kFusedCand = 32;                   // boundary-bin tiles ranked in the kernel
+// Per-row state words (one row per epilogue thread): the 128 16-bit bin
+// counts of pass 1, then the 64 kept-tile mask words of pass 2 (N <= 2048),
+// plus one word of padding so that the rows fall on different banks.
+constexpr int kStateWords = 65;
 
 template <int D, bool FUSED>
 struct ScoresCfg {
@@ -60,9 +64,9 @@ struct ScoresCfg {
   static constexpr int OFF_RING = KS * kSliceBytes;       // stage s: Pk hi, then Pk lo
   static constexpr int STAGE = 2 * kSliceBytes;
   static constexpr int OFF_EPI = OFF_RING + STAGES * STAGE;
-  // Epilogue: the transpose buffers, or (fused) per-row state: a 16-bit
-  // histogram [bin][row] and the boundary-bin keys [slot][row].
-  static constexpr int EPI_BYTES = FUSED ? kFusedBins * kRows * 2 + kFusedCand * kRows * 8 : 4 * kEpiBytes;
+  // Epilogue: the transpose buffers, or (fused) per-row state words and the
+  // boundary-bin keys [slot][row].
+  static constexpr int EPI_BYTES = FUSED ? kRows * kStateWords * 4 + kFusedCand * kRows * 8 : 4 * kEpiBytes;
   static constexpr int OFF_BAR = OFF_EPI + EPI_BYTES;
   // a_full, a_stage_free, a_split, a_free, b_full[S], b_split[S], b_empty[S], acc_full[2],
   // acc_empty[2], final
@@ -353,14 +357,18 @@ block_scores_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
     // ------------------------------------------------------------ fused top-k epilogue
     // Thread r owns row r of the current 128-row block (TMEM lane r).
     const int r = tid;
-    uint16_t* hist = reinterpret_cast<uint16_t*>(smem + C::OFF_EPI);  // [bin][row]
-    uint64_t* cand = reinterpret_cast<uint64_t*>(smem + C::OFF_EPI + kFusedBins * kRows * 2);  // [slot][row]
+    // This row's state: bin counts in pass 1, then its kept-tile mask (one
+    // bit per tile, ascending) in pass 2; only this thread touches it.
+    uint32_t* rowstate = reinterpret_cast<uint32_t*>(smem + C::OFF_EPI) + r * kStateWords;
+    uint16_t* hist = reinterpret_cast<uint16_t*>(rowstate);
+    uint32_t* bmask = rowstate;
+    uint64_t* cand = reinterpret_cast<uint64_t*>(smem + C::OFF_EPI + kRows * kStateWords * 4);  // [slot][row]
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
     constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23: bin index in the low mantissa bits
     const float qnan = __int_as_float(0x7fc00000);
     const int rr = min(P.k, P.N);
     float mn = qnan, mx = qnan, sc = 0.f, offm = kMagic;
-    int bstar = -1, need = 0, outpos = 0, ncand = 0;
+    int bstar = -1, need = 0, ncand = 0;
     bool crowded = false;
     // Equal-width bins over [mn, mx], monotone in the score (one FMA; NaN and
     // a range that overflows land in bin 0).
@@ -393,14 +401,14 @@ block_scores_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
         if (!(sc <= 3.0e38f)) crowded = true;
         if (crowded) sc = 0.f;
         offm = crowded ? kMagic : fmaf(-mn, sc, kMagic);
-        for (int q = 0; q < kFusedBins; ++q) hist[q * kRows + r] = 0;
+        for (int q = 0; q < kFusedBins / 2; ++q) rowstate[q] = 0u;
       }
       if (bj == 0 && pass == 2) {
         // The bin in which the count, taken from the top bin down, reaches rr.
         int run = 0;
         bstar = -1;
         for (int q = kFusedBins - 1; q >= 0; --q) {
-          const int c = hist[q * kRows + r];
+          const int c = hist[q];
           if (run + c >= rr) {
             bstar = q;
             need = rr - run;
@@ -410,7 +418,6 @@ block_scores_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
           run += c;
         }
         if (bstar < 0) crowded = true;
-        outpos = 0;
         ncand = 0;
       }
       int32_t* out = P.idx + grow * P.kmax;
@@ -437,7 +444,13 @@ block_scores_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
           if (!crowded) {
 #pragma unroll
             for (int q = 0; q < 32; ++q)
-              if (q < jn) ++hist[bin_of(__uint_as_float(v[q]) * P.scale) * kRows + r];
+              if (q < jn) {
+                // 16-bit counts, two to a word (at most 2,048 each): an atomic
+                // add that returns nothing, so the thread does not wait for
+                // its previous increment to land.
+                const int bx = bin_of(__uint_as_float(v[q]) * P.scale);
+                atomicAdd(rowstate + (bx >> 1), 1u << (16 * (bx & 1)));
+              }
           }
         } else if (jn > 0) {
           if (crowded || P.debug_s) {
@@ -446,20 +459,22 @@ block_scores_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
               if (q < jn) srow[j0 + q] = __uint_as_float(v[q]) * P.scale;
           }
           if (!crowded) {
+            // Tiles above the boundary bin as one 32-bit mask word per piece;
+            // the boundary bin's tiles as keys.
+            uint32_t above_bits = 0;
 #pragma unroll
             for (int q = 0; q < 32; ++q) {
               const float x = __uint_as_float(v[q]) * P.scale;
               const int bx = q < jn ? bin_of(x) : -1;
-              if (bx > bstar) {
-                if (outpos < P.kmax) out[outpos] = j0 + q;
-                ++outpos;
-              } else if (bx == bstar) {
+              above_bits |= (bx > bstar ? 1u : 0u) << q;
+              if (bx == bstar) {
                 if (ncand < kFusedCand)
                   cand[ncand * kRows + r] =
                       ((uint64_t)fused_order_key(x) << 32) | (uint64_t)(0xffffffffu - (uint32_t)(j0 + q));
                 ++ncand;
               }
             }
+            bmask[j0 >> 5] = above_bits;
           }
         }
       }
@@ -469,40 +484,29 @@ block_scores_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
         if (crowded) {
           P.fb_rows[atomicAdd(P.fb_count, 1)] = (int32_t)grow;
         } else {
-          // The boundary bin's keys are unique; the `need` largest are kept.
-          // Their tile indices, ascending, go into the histogram's column r
-          // (free now) and are merged behind the tiles above the bin.
-          uint16_t* kept = hist + r;
+          // The boundary bin's keys are unique; the `need` largest are kept:
+          // their bits join the mask, which is then written out ascending.
           const int nc = min(ncand, kFusedCand);
-          int nk = 0;
           for (int x1 = 0; x1 < nc; ++x1) {
             const uint64_t kx = cand[x1 * kRows + r];
             int rank = 0;
             for (int x2 = 0; x2 < nc; ++x2) rank += cand[x2 * kRows + r] > kx ? 1 : 0;
             if (rank < need) {
-              const uint16_t jj = (uint16_t)(0xffffffffu - (uint32_t)kx);
-              int pos = nk++;
-              while (pos > 0 && kept[(pos - 1) * kRows] > jj) {
-                kept[pos * kRows] = kept[(pos - 1) * kRows];
-                --pos;
-              }
-              kept[pos * kRows] = jj;
+              const uint32_t jj = 0xffffffffu - (uint32_t)kx;
+              bmask[jj >> 5] |= 1u << (jj & 31);
             }
           }
-          const int na = min(outpos, P.kmax), total = min(na + nk, P.kmax);
-          int ia = na - 1, ib = nk - 1;
-          for (int wpos = total - 1; wpos >= 0 && ib >= 0; --wpos) {
-            const int ja = ia >= 0 ? out[ia] : -1;
-            const int jb = kept[ib * kRows];
-            if (ja > jb) {
-              out[wpos] = ja;
-              --ia;
-            } else {
-              out[wpos] = jb;
-              --ib;
+          int total = 0;
+          const int nwords = (P.N + 31) >> 5;
+          for (int wd = 0; wd < nwords; ++wd) {
+            uint32_t bits = bmask[wd];
+            while (bits) {
+              if (total < P.kmax) out[total] = wd * 32 + __ffs(bits) - 1;
+              ++total;
+              bits &= bits - 1;
             }
           }
-          P.cnt[grow] = total;
+          P.cnt[grow] = min(total, P.kmax);
         }
       }
     }
