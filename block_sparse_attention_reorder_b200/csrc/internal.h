@@ -118,13 +118,13 @@ bsattn_status bsattn_static_scratch_prepare(int device);
   } while (0)
 
 // Launch wrappers (each returns BSATTN_OK or BSATTN_ERR_CUDA).
-// flags for launch_reorder
-enum : int {
-  RO_WRITE_TILED = 1,  // write the tiled bf16 copy
-  RO_QUANT = 4,        // write e4m3 codes + tile scales
-};
+// Natural -> tiled bf16 copy (padded slots zero).
 bsattn_status launch_reorder(const Geom& g, const __nv_bfloat16* x_nat, __nv_bfloat16* x_tiled,
-                             uint8_t* codes, float* scales, int flags, cudaStream_t st);
+                             cudaStream_t st);
+// e4m3 tile codes (tiled layout) and per-tile scales of natural Q and K, one launch.
+bsattn_status launch_reorder_quant(const Geom& g, const __nv_bfloat16* q_nat, const __nv_bfloat16* k_nat,
+                                   uint8_t* q_codes, uint8_t* k_codes, float* q_scales, float* k_scales,
+                                   cudaStream_t st);
 // fp32 tile means of one or two natural tensors (x1/p1 may be null).
 bsattn_status launch_pool(const Geom& g, const __nv_bfloat16* x0, float* p0, const __nv_bfloat16* x1,
                           float* p1, cudaStream_t st);

@@ -291,8 +291,7 @@ bsattn_status attn_reorder(const bsattn_plan* p, const void* x_nat, void* x_tile
   if (dev.status) return dev.status;
   bsattn_status s = BSATTN_OK;
   Geom g = make_geom(p);
-  if ((s = launch_reorder(g, (const __nv_bfloat16*)x_nat, (__nv_bfloat16*)x_tiled, nullptr, nullptr,
-                          RO_WRITE_TILED, (cudaStream_t)stream)))
+  if ((s = launch_reorder(g, (const __nv_bfloat16*)x_nat, (__nv_bfloat16*)x_tiled, (cudaStream_t)stream)))
     return s;
   return pooled ? launch_pool(g, (const __nv_bfloat16*)x_nat, pooled, nullptr, nullptr, (cudaStream_t)stream)
                 : BSATTN_OK;
@@ -478,8 +477,9 @@ bsattn_status attn_layer(const bsattn_plan* p, const void* q_nat, const void* k_
   const void* k = k_nat;
   if (p->desc.qk_fp8) {
     // e4m3 tile codes and scales.
-    if ((s = launch_reorder(g, (const __nv_bfloat16*)q_nat, nullptr, w.qt, w.qs, RO_QUANT, st))) return s;
-    if ((s = launch_reorder(g, (const __nv_bfloat16*)k_nat, nullptr, w.kt, w.ks, RO_QUANT, st))) return s;
+    if ((s = launch_reorder_quant(g, (const __nv_bfloat16*)q_nat, (const __nv_bfloat16*)k_nat, w.qt, w.kt, w.qs,
+                                  w.ks, st)))
+      return s;
     q = w.qt;
     k = w.kt;
   }

@@ -7,7 +7,8 @@
 // are one contiguous 64*D*2-byte block, so both sides use full 32-byte
 // sectors. e4m3 quantisation needs the whole tile's amax: with one chunk per
 // tile the values stay in registers, with several a CTA takes the tile and
-// reads it twice (the second time mostly from L2).
+// reads it twice (the second time mostly from L2). Q and K are quantised by
+// one launch (the grid's z covers both tensors).
 #include <cuda_fp8.h>
 
 #include "internal.h"
@@ -46,6 +47,15 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float* f) {
   }
 }
 
+// max(|x|) of 8 bf16 values, taken on bf16 pairs (exact: the maximum of bf16
+// magnitudes is one of them; a NaN is passed over, as fmaxf does).
+__device__ __forceinline__ __nv_bfloat162 absmax8(__nv_bfloat162 m, const uint4& u) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) m = __hmax2(m, __habs2(h[i]));
+  return m;
+}
+
 __device__ __forceinline__ float block_max(float v, float* red) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
@@ -58,23 +68,31 @@ __device__ __forceinline__ float block_max(float v, float* red) {
   return m;
 }
 
-// x / scale as the e4m3 conversion sees it. The code is that of the IEEE
-// fp32 quotient fl(x / scale); the product p = x * rscale (rscale the
-// correctly rounded 1 / scale) is within 3 fp32 ulps of that quotient (two
-// roundings of 2^-24 relative each, plus the quotient's own half ulp), so it
-// rounds to the same e4m3 code unless it lies within a few ulps of an e4m3
-// rounding midpoint (fp32 mantissa bits 19..0 equal to 0x80000 for e4m3
-// normals) or in the e4m3 subnormal range (|p| < 2^-6); those rare values
-// take the exact division. Zero is exact either way.
+// x / scale as the e4m3 conversion sees it: the IEEE fp32 quotient
+// fl(x / scale), computed without a division by Markstein's FMA correction.
+// With y = rscale the correctly rounded 1/scale and p = fl(x * y), p is
+// within an ulp of x / scale, the residual x - p * scale is exact in fp32 and
+// fl(p + r * y) is the correctly rounded quotient. The residual is exact when
+// ulp(p) * ulp(scale) >= 2^-149; for codes that can be nonzero (|p| >= 2^-11)
+// that holds once scale >= 2^-92. Tiles with a smaller scale, or with one
+// above 2^126 (reciprocal subnormal or zero, e.g. an infinite amax), divide
+// instead; the test is per tile, hence uniform across the CTA. r is written
+// as -(p * scale - x) so that x = -0 keeps its sign.
+constexpr float kFmaQuotientMinScale = 0x1p-92f, kFmaQuotientMaxScale = 0x1p126f;
+
 __device__ __forceinline__ float e4m3_quotient(float x, float scale, float rscale) {
-  const float p = x * rscale;
-  const uint32_t a = __float_as_uint(p) & 0x7fffffffu;
-  const uint32_t low = a & 0xFFFFFu;
-  const bool safe = a == 0u || (a >= 0x3C800000u && low + 4u - 0x80000u > 8u);
-  return safe ? p : __fdiv_rn(x, scale);
+  const float p = __fmul_rn(x, rscale);
+  const float r = -fmaf(p, scale, -x);
+  return fmaf(r, rscale, p);
 }
 
-// e4m3 codes of 8 values divided by `scale` (as the IEEE fp32 division), RNE, satfinite.
+__device__ __forceinline__ bool fma_quotient_ok(float scale) {
+  return scale >= kFmaQuotientMinScale && scale <= kFmaQuotientMaxScale;
+}
+
+// e4m3 codes of 8 values divided by `scale` (as the IEEE fp32 division), RNE,
+// satfinite; FMA: through e4m3_quotient (the tile passed fma_quotient_ok).
+template <bool FMA>
 __device__ __forceinline__ uint2 quant8(const float* f, float scale, float rscale) {
   uint32_t w[2];
 #pragma unroll
@@ -82,8 +100,9 @@ __device__ __forceinline__ uint2 quant8(const float* f, float scale, float rscal
     uint32_t acc = 0;
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
-      float2 x = make_float2(e4m3_quotient(f[4 * h + 2 * i], scale, rscale),
-                             e4m3_quotient(f[4 * h + 2 * i + 1], scale, rscale));
+      const float a = f[4 * h + 2 * i], b = f[4 * h + 2 * i + 1];
+      float2 x = FMA ? make_float2(e4m3_quotient(a, scale, rscale), e4m3_quotient(b, scale, rscale))
+                          : make_float2(__fdiv_rn(a, scale), __fdiv_rn(b, scale));
       __nv_fp8x2_storage_t p = __nv_cvt_float2_to_fp8x2(x, __NV_SATFINITE, __NV_E4M3);
       acc |= (uint32_t)p << (16 * i);
     }
@@ -98,12 +117,10 @@ __device__ __forceinline__ float tile_scale_from_amax(float amax) {
 
 template <int D>
 __global__ void __launch_bounds__(kThreads)
-reorder_kernel(Geom g, const __nv_bfloat16* __restrict__ x_nat, __nv_bfloat16* __restrict__ x_tiled,
-               uint8_t* __restrict__ codes, float* __restrict__ scales, int flags) {
+reorder_kernel(Geom g, const __nv_bfloat16* __restrict__ x_nat, __nv_bfloat16* __restrict__ x_tiled) {
   constexpr int CH = D / 8;                 // 16-byte chunks per row
   constexpr int ITER = 64 * CH / kThreads;  // chunks per thread
   constexpr int RSTEP = kThreads / CH;      // row stride between a thread's chunks
-  __shared__ float wred[kThreads / 32];
   __shared__ int rowtok[64];  // token of each row of the chunk, -1 for a padded slot
 
   const int j = blockIdx.x / g.nchunk, head = blockIdx.y, b = blockIdx.z;
@@ -120,41 +137,66 @@ reorder_kernel(Geom g, const __nv_bfloat16* __restrict__ x_nat, __nv_bfloat16* _
   uint4 v[ITER];
 #pragma unroll
   for (int i = 0; i < ITER; ++i) {
-    int r = r0 + RSTEP * i;
-    int n = rowtok[r];
-    if (n >= 0) {
-      const uint4* src = reinterpret_cast<const uint4*>(x_nat + (((size_t)b * g.L + n) * g.Hh + head) * D) + c;
-      v[i] = __ldg(src);
-    } else {
-      v[i] = make_uint4(0, 0, 0, 0);
-    }
+    int n = rowtok[r0 + RSTEP * i];
+    v[i] = n >= 0 ? __ldg(reinterpret_cast<const uint4*>(x_nat + (((size_t)b * g.L + n) * g.Hh + head) * D) + c)
+                  : make_uint4(0, 0, 0, 0);
   }
-  if (flags & RO_WRITE_TILED) {
 #pragma unroll
-    for (int i = 0; i < ITER; ++i) {
-      int r = r0 + RSTEP * i;
-      reinterpret_cast<uint4*>(x_tiled + (tile_off + r) * D)[c] = v[i];
-    }
+  for (int i = 0; i < ITER; ++i)
+    reinterpret_cast<uint4*>(x_tiled + (tile_off + r0 + RSTEP * i) * D)[c] = v[i];
+}
+
+// Source and destination of the e4m3 quantisation of one or two tensors
+// (Q and K); blockIdx.z = batch * ntensor + tensor.
+struct QuantPair {
+  const __nv_bfloat16* src[2];
+  uint8_t* codes[2];
+  float* scales[2];
+};
+
+// e4m3 codes and tile scales of one-chunk tiles straight from the natural
+// layout: one CTA per (tile, head, tensor, batch) holds the tile's 64 rows in
+// registers, takes their amax, and writes the codes as one contiguous block.
+// Capped at 40 registers so six CTAs share an SM and keep loads in flight
+// across each CTA's amax barrier.
+template <int D>
+__global__ void __launch_bounds__(kThreads, 6)
+reorder_quant_kernel(Geom g, QuantPair qp) {
+  constexpr int CH = D / 8;
+  constexpr int ITER = 64 * CH / kThreads;
+  constexpr int RSTEP = kThreads / CH;
+  __shared__ float wred[kThreads / 32];
+  __shared__ int rowtok[64];
+  const int nt = gridDim.z / g.B;
+  const int tensor = blockIdx.z % nt, b = blockIdx.z / nt;
+  const int j = blockIdx.x, head = blockIdx.y;
+  const int c = threadIdx.x % CH;
+  const int r0 = threadIdx.x / CH;
+  const size_t tile = ((size_t)b * g.Hh + head) * g.N + j;
+  if (threadIdx.x < 64) rowtok[threadIdx.x] = row_token(g, tile_coord(g, j), threadIdx.x);
+  __syncthreads();
+  const __nv_bfloat16* x_nat = qp.src[tensor];
+  uint4 v[ITER];
+#pragma unroll
+  for (int i = 0; i < ITER; ++i) {
+    int n = rowtok[r0 + RSTEP * i];
+    v[i] = n >= 0 ? __ldg(reinterpret_cast<const uint4*>(x_nat + (((size_t)b * g.L + n) * g.Hh + head) * D) + c)
+                  : make_uint4(0, 0, 0, 0);
   }
-  if (flags & RO_QUANT) {
-    float m = 0.f;
+  __nv_bfloat162 m2 = __float2bfloat162_rn(0.f);
 #pragma unroll
-    for (int i = 0; i < ITER; ++i) {
-      float f[8];
-      bf16x8_to_f32(v[i], f);
+  for (int i = 0; i < ITER; ++i) m2 = absmax8(m2, v[i]);
+  const float m = fmaxf(__low2float(m2), __high2float(m2));
+  const float scale = tile_scale_from_amax(block_max(m, wred)), rscale = __frcp_rn(scale);
+  uint2* dst = reinterpret_cast<uint2*>(qp.codes[tensor] + tile * 64 * D);
+  const bool fma = fma_quotient_ok(scale);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(f[e]));
-    }
-    const float scale = tile_scale_from_amax(block_max(m, wred)), rscale = __frcp_rn(scale);
-#pragma unroll
-    for (int i = 0; i < ITER; ++i) {
-      int r = r0 + RSTEP * i;
-      float f[8];
-      bf16x8_to_f32(v[i], f);
-      reinterpret_cast<uint2*>(codes + (tile_off + r) * D)[c] = quant8(f, scale, rscale);
-    }
-    if (threadIdx.x == 0) scales[((size_t)b * g.Hh + head) * g.N + j] = scale;
+  for (int i = 0; i < ITER; ++i) {
+    float f[8];
+    bf16x8_to_f32(v[i], f);
+    dst[(r0 + RSTEP * i) * CH + c] = fma ? quant8<true>(f, scale, rscale) : quant8<false>(f, scale, rscale);
   }
+  if (threadIdx.x == 0) qp.scales[tensor][tile] = scale;
 }
 
 template <int D>
@@ -208,32 +250,35 @@ quant_tiled_kernel(Geom g, const __nv_bfloat16* __restrict__ x_tiled, uint8_t* _
   }
   const float scale = tile_scale_from_amax(block_max(m, wred)), rscale = __frcp_rn(scale);
   uint2* dst = reinterpret_cast<uint2*>(codes + tile * 64 * D);
+  const bool fma = fma_quotient_ok(scale);
 #pragma unroll
   for (int i = 0; i < ITER; ++i) {
     float f[8];
     bf16x8_to_f32(v[i], f);
-    dst[threadIdx.x + kThreads * i] = quant8(f, scale, rscale);
+    dst[threadIdx.x + kThreads * i] = fma ? quant8<true>(f, scale, rscale) : quant8<false>(f, scale, rscale);
   }
   if (threadIdx.x == 0) scales[tile] = scale;
 }
 
 // e4m3 codes of tiles of several chunks: pass 1 takes the tile's amax, pass 2
-// reads the tile again and writes the codes (and, for NAT sources with
-// x_tiled set, the tiled bf16 copy). NAT: the source is the natural layout
-// (padded rows read as zero); else it is the tiled bf16 layout.
+// reads the tile again (mostly from L2) and writes the codes. NAT: the
+// sources are natural-layout tensors (padded rows read as zero); else tiled
+// bf16 tensors.
 template <int D, bool NAT>
 __global__ void __launch_bounds__(kThreads)
-quant_multi_kernel(Geom g, const __nv_bfloat16* __restrict__ src, __nv_bfloat16* __restrict__ x_tiled,
-                   uint8_t* __restrict__ codes, float* __restrict__ scales) {
+quant_multi_kernel(Geom g, QuantPair qp) {
   constexpr int CH = D / 8;
   constexpr int ITER = 64 * CH / kThreads;
   constexpr int RSTEP = kThreads / CH;
   __shared__ float wred[kThreads / 32];
-  const int j = blockIdx.x, head = blockIdx.y, b = blockIdx.z;
+  const int nt = gridDim.z / g.B;
+  const int tensor = blockIdx.z % nt, b = blockIdx.z / nt;
+  const int j = blockIdx.x, head = blockIdx.y;
   const int c = threadIdx.x % CH;
   const int r0 = threadIdx.x / CH;
   const TileCoord tc = tile_coord(g, j);
   const size_t tile = ((size_t)b * g.Hh + head) * g.N + j;
+  const __nv_bfloat16* src = qp.src[tensor];
   auto load = [&](int r) -> uint4 {
     if (NAT) {
       const int n = row_token(g, tc, r);
@@ -242,20 +287,18 @@ quant_multi_kernel(Geom g, const __nv_bfloat16* __restrict__ src, __nv_bfloat16*
     }
     return __ldg(reinterpret_cast<const uint4*>(src + (tile * g.V + r) * D) + c);
   };
-  float m = 0.f;
+  __nv_bfloat162 m2 = __float2bfloat162_rn(0.f);
   for (int row0 = 0; row0 < g.V; row0 += 64) {
     uint4 v[ITER];
 #pragma unroll
     for (int i = 0; i < ITER; ++i) v[i] = load(row0 + r0 + RSTEP * i);
 #pragma unroll
-    for (int i = 0; i < ITER; ++i) {
-      float f[8];
-      bf16x8_to_f32(v[i], f);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(f[e]));
-    }
+    for (int i = 0; i < ITER; ++i) m2 = absmax8(m2, v[i]);
   }
+  const float m = fmaxf(__low2float(m2), __high2float(m2));
   const float scale = tile_scale_from_amax(block_max(m, wred)), rscale = __frcp_rn(scale);
+  uint8_t* codes = qp.codes[tensor];
+  const bool fma = fma_quotient_ok(scale);
   for (int row0 = 0; row0 < g.V; row0 += 64) {
     uint4 v[ITER];
 #pragma unroll
@@ -263,13 +306,13 @@ quant_multi_kernel(Geom g, const __nv_bfloat16* __restrict__ src, __nv_bfloat16*
 #pragma unroll
     for (int i = 0; i < ITER; ++i) {
       const size_t row = tile * g.V + row0 + r0 + RSTEP * i;
-      if (NAT && x_tiled) reinterpret_cast<uint4*>(x_tiled + row * D)[c] = v[i];
       float f[8];
       bf16x8_to_f32(v[i], f);
-      reinterpret_cast<uint2*>(codes + row * D)[c] = quant8(f, scale, rscale);
+      reinterpret_cast<uint2*>(codes + row * D)[c] =
+          fma ? quant8<true>(f, scale, rscale) : quant8<false>(f, scale, rscale);
     }
   }
-  if (threadIdx.x == 0) scales[tile] = scale;
+  if (threadIdx.x == 0) qp.scales[tensor][tile] = scale;
 }
 
 // Tile means of natural bf16 tokens. A token row holds all heads
@@ -346,21 +389,30 @@ bsattn_status launch_pool(const Geom& g, const __nv_bfloat16* x0, float* p0, con
 }
 
 bsattn_status launch_reorder(const Geom& g, const __nv_bfloat16* x_nat, __nv_bfloat16* x_tiled,
-                             uint8_t* codes, float* scales, int flags, cudaStream_t st) {
-  if ((flags & RO_QUANT) && g.nchunk > 1) {
-    __nv_bfloat16* xt = (flags & RO_WRITE_TILED) ? x_tiled : nullptr;
-    dim3 grid(g.N, g.Hh, g.B);
-    if (g.D == 128)
-      quant_multi_kernel<128, true><<<grid, kThreads, 0, st>>>(g, x_nat, xt, codes, scales);
-    else
-      quant_multi_kernel<64, true><<<grid, kThreads, 0, st>>>(g, x_nat, xt, codes, scales);
-    return cudaGetLastError() == cudaSuccess ? BSATTN_OK : BSATTN_ERR_CUDA;
-  }
+                             cudaStream_t st) {
   dim3 grid(g.N * g.nchunk, g.Hh, g.B);
   if (g.D == 128)
-    reorder_kernel<128><<<grid, kThreads, 0, st>>>(g, x_nat, x_tiled, codes, scales, flags);
+    reorder_kernel<128><<<grid, kThreads, 0, st>>>(g, x_nat, x_tiled);
   else
-    reorder_kernel<64><<<grid, kThreads, 0, st>>>(g, x_nat, x_tiled, codes, scales, flags);
+    reorder_kernel<64><<<grid, kThreads, 0, st>>>(g, x_nat, x_tiled);
+  return cudaGetLastError() == cudaSuccess ? BSATTN_OK : BSATTN_ERR_CUDA;
+}
+
+bsattn_status launch_reorder_quant(const Geom& g, const __nv_bfloat16* q_nat, const __nv_bfloat16* k_nat,
+                                   uint8_t* q_codes, uint8_t* k_codes, float* q_scales, float* k_scales,
+                                   cudaStream_t st) {
+  const QuantPair qp{{q_nat, k_nat}, {q_codes, k_codes}, {q_scales, k_scales}};
+  dim3 grid(g.N, g.Hh, 2 * g.B);
+  if (g.nchunk > 1) {
+    if (g.D == 128)
+      quant_multi_kernel<128, true><<<grid, kThreads, 0, st>>>(g, qp);
+    else
+      quant_multi_kernel<64, true><<<grid, kThreads, 0, st>>>(g, qp);
+  } else if (g.D == 128) {
+    reorder_quant_kernel<128><<<grid, kThreads, 0, st>>>(g, qp);
+  } else {
+    reorder_quant_kernel<64><<<grid, kThreads, 0, st>>>(g, qp);
+  }
   return cudaGetLastError() == cudaSuccess ? BSATTN_OK : BSATTN_ERR_CUDA;
 }
 
@@ -378,10 +430,11 @@ bsattn_status launch_quant_tiled(const Geom& g, const __nv_bfloat16* x_tiled, ui
                                  float* scales, cudaStream_t st) {
   dim3 grid(g.N, g.Hh, g.B);
   if (g.nchunk > 1) {
+    const QuantPair qp{{x_tiled, x_tiled}, {codes, codes}, {scales, scales}};
     if (g.D == 128)
-      quant_multi_kernel<128, false><<<grid, kThreads, 0, st>>>(g, x_tiled, nullptr, codes, scales);
+      quant_multi_kernel<128, false><<<grid, kThreads, 0, st>>>(g, qp);
     else
-      quant_multi_kernel<64, false><<<grid, kThreads, 0, st>>>(g, x_tiled, nullptr, codes, scales);
+      quant_multi_kernel<64, false><<<grid, kThreads, 0, st>>>(g, qp);
     return cudaGetLastError() == cudaSuccess ? BSATTN_OK : BSATTN_ERR_CUDA;
   }
   if (g.D == 128)

@@ -185,13 +185,38 @@ def test_quantize_e4m3_bytes(bs, name):
     np.testing.assert_array_equal(codes.cpu().numpy(), rc)
 
 
-def test_quantize_e4m3_every_bf16_magnitude(bs):
+def _bf16(x):
+    return (np.array([x], np.float32).view(np.uint32) & 0xFFFF0000).view(np.float32)[0]
+
+
+def _bf16_step(x, n):
+    """The bf16 value n representable steps above (n > 0) or below x > 0."""
+    return (np.array([x], np.float32).view(np.uint32) + np.uint32(n << 16) if n > 0 else
+            np.array([x], np.float32).view(np.uint32) - np.uint32((-n) << 16)).view(np.float32)[0]
+
+
+# Tile amax values away from the common range: the exact-division fallback of
+# the quantiser (scale below 2^-92, or infinite) and the values next to that
+# bound, the bf16 extremes, and ordinary ones; 24 tiles.
+_GUARD = np.float32(448.0) * np.float32(2.0) ** -92  # scale exactly 2^-92
+_BF16_MAX = np.array([0x7F7F0000], np.uint32).view(np.float32)[0]
+_EDGE_AMAX = [_GUARD, _bf16_step(_GUARD, -1), _bf16_step(_GUARD, 1), _bf16_step(_GUARD, -2),
+              np.float32(2.0) ** -100, _bf16(1e-30), _bf16(1e-35), _bf16(1.2e-38), _bf16(9.2e-41),
+              _BF16_MAX, _bf16(1e38), np.float32(2.0) ** 100, np.float32(1.0), np.float32(448.0),
+              np.float32(0.5), _bf16(3e-20), _bf16(7e15), np.float32(np.inf), np.float32(np.inf), _bf16(5e-3),
+              _bf16(123.0), _bf16(2e-27), _bf16(6e-26), _bf16(1e-24)]
+
+
+@pytest.mark.parametrize("amax_set", ["random", "edges"])
+def test_quantize_e4m3_every_bf16_magnitude(bs, amax_set):
     """Tiles holding every bf16 magnitude of the 32 binades up to the tile's
-    amax (both signs, zeros to fill the 64 x 128 tile), under 24 different
-    amax values: e4m3 codes byte-identical to the oracle's fp32-division
-    quantisation. Many of these quotients fall exactly on, or next to, e4m3
-    rounding midpoints (bf16 ratios have short binary expansions), and the
-    smallest ones in the e4m3 subnormal range and below it."""
+    amax (both signs, +0 and -0 filling the 64 x 128 tile), under 24 amax
+    values (random ones between 5e-5 and 2e4, or the edge set above, where a
+    tile with an infinite amax holds +inf and -inf): e4m3 codes byte-identical
+    to the oracle's fp32-division quantisation. Many of these quotients fall
+    exactly on, or next to, e4m3 rounding midpoints (bf16 ratios have short
+    binary expansions), and the smallest ones in the e4m3 subnormal range and
+    below it."""
     T, H, W = 4, 4, 4 * 12  # 12 tiles of 64 tokens
     heads = 2
     plan = bs.Plan(1, heads, 128, T, H, W, rule="window", win=(0, 0, 1), qk_fp8=True)
@@ -199,22 +224,28 @@ def test_quantize_e4m3_every_bf16_magnitude(bs):
     tiles = np.zeros((1, heads, plan.N, 64, 128), dtype=np.float32)
     for h in range(heads):
         for t in range(plan.N):
-            amax = np.float32(rng.uniform(0.5, 2.0) * 10.0 ** rng.uniform(-4, 4))
-            amax = (np.array([amax], np.float32).view(np.uint32) & 0xFFFF0000).view(np.float32)[0]  # bf16
-            e = int(np.frexp(amax)[1]) - 1
-            base = (np.float32(2.0) ** np.arange(e - 31, e + 1, dtype=np.float32)).view(np.uint32)
+            if amax_set == "random":
+                amax = _bf16(np.float32(rng.uniform(0.5, 2.0) * 10.0 ** rng.uniform(-4, 4)))
+            else:
+                amax = _EDGE_AMAX[h * plan.N + t]
+            top = amax if np.isfinite(amax) else _BF16_MAX
+            e = int(np.frexp(top)[1]) - 1
+            # binade bases as bf16 (those below the smallest bf16 subnormal are 0)
+            base = (np.float32(2.0) ** np.arange(e - 31, e + 1, dtype=np.float32)).view(np.uint32) & 0xFFFF0000
             mags = (base[:, None] + (np.arange(128, dtype=np.uint32) << 16)[None, :]).reshape(-1).view(np.float32)
-            mags = mags[mags < amax]
+            mags = np.unique(mags[mags < amax])
             vals = np.concatenate([[amax, -amax], mags, -mags])[:8192].astype(np.float32)
             flat = np.zeros(8192, np.float32)
             flat[:vals.size] = vals
+            flat[vals.size::2] = -0.0
             tiles[0, h, t] = rng.permutation(flat).reshape(64, 128)
     xt = torch.from_numpy(tiles).to(torch.bfloat16).cuda()
     assert torch.equal(xt.float().cpu(), torch.from_numpy(tiles))  # every value is a bf16 value
     codes = torch.empty(plan.tiled_shape(), dtype=torch.uint8, device="cuda")
     scales = torch.empty((1, heads, plan.N), dtype=torch.float32, device="cuda")
     bs.attn_quantize_e4m3(plan, xt, codes, scales)
-    rc, rs = e4m3.quantize_tiled(tiles)
+    with np.errstate(invalid="ignore"):  # inf / inf in the tiles with an infinite amax: NaN, code 0x7F
+        rc, rs = e4m3.quantize_tiled(tiles)
     np.testing.assert_array_equal(scales.cpu().numpy(), rs)
     np.testing.assert_array_equal(codes.cpu().numpy(), rc)
     # attn_layer quantises while it reorders (natural source): its output is
@@ -234,7 +265,7 @@ def test_quantize_e4m3_every_bf16_magnitude(bs):
     o_chain = torch.empty_like(x_nat)
     bs.attn_unreorder(plan, ot, o_chain)
     assert bs.attn_check_device_status(plan) == 0
-    assert torch.equal(o_layer, o_chain)
+    assert torch.equal(o_layer.view(torch.int16), o_chain.view(torch.int16))  # bitwise: NaN rows included
 
 
 def _oracle_inputs(wl):
