@@ -401,6 +401,40 @@ def test_forward_natural_equals_tiled_path(bs, name):
     assert torch.equal(lse_nat.cpu(), lse_ref)
 
 
+@pytest.mark.parametrize("name", ["ragged_window_fp8", "ragged_d64_fp8", "tile248_window_fp8",
+                                  "tile688_window_fp8"])
+def test_layer_e4m3_equals_quantize_chain(bs, name):
+    """attn_layer quantises Q and K in one launch straight from the natural
+    layout (tiles of one chunk and of several); its output is bit-identical
+    to reorder -> attn_quantize_e4m3 -> attn_forward -> unreorder on the same
+    kept lists."""
+    wl = SMALL[name]
+    plan = _plan(bs, wl)
+    assert plan.qk_fp8
+    q, k, v = make_qkv(wl, "cuda")
+    si, sc = plan.list_shapes()
+    idx = torch.empty(si, dtype=torch.int32, device="cuda")
+    cnt = torch.empty(sc, dtype=torch.int32, device="cuda")
+    o_layer = torch.full_like(q, float("nan"))
+    bs.attn_layer(plan, q, k, v, o_layer, plan.workspace("layer"), idx=idx, cnt=cnt)
+    ts = plan.tiled_shape()
+    tiled = []
+    for x in (q, k, v):
+        t = torch.empty(ts, dtype=torch.bfloat16, device="cuda")
+        bs.attn_reorder(plan, x, t)
+        tiled.append(t)
+    codes = [torch.empty(ts, dtype=torch.uint8, device="cuda") for _ in range(2)]
+    scales = [torch.empty((wl.B, wl.heads, plan.N), dtype=torch.float32, device="cuda") for _ in range(2)]
+    for t, c, s_ in zip(tiled[:2], codes, scales):
+        bs.attn_quantize_e4m3(plan, t, c, s_)
+    ot = torch.empty(ts, dtype=torch.bfloat16, device="cuda")
+    bs.attn_forward(plan, codes[0], codes[1], tiled[2], idx, cnt, ot, q_scale=scales[0], k_scale=scales[1])
+    o_chain = torch.empty_like(q)
+    bs.attn_unreorder(plan, ot, o_chain)
+    assert bs.attn_check_device_status(plan) == 0
+    assert torch.equal(o_layer.view(torch.int16), o_chain.view(torch.int16))
+
+
 def tiling_lse_natural(lse_t, wl, plan):
     """Tiled lse [B, Hh, N, V] -> natural [B, Hh, L] (oracle's tile order)."""
     x = to64(lse_t)
