@@ -168,6 +168,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   uint32_t* ulist = bmB + P.bm_words;
   uint32_t* uext = ulist + P.umax;  // real extent of each step's key chunk (see below)
   uint32_t* uorg = uext + P.umax;   // packed in-tile offsets of the steps' key chunks (several-chunk tiles)
+  float* uks = reinterpret_cast<float*>(uorg + (P.g.nchunk > 1 ? P.umax : 0));  // e4m3: each step's key-tile scale
 
   const Geom& g = P.g;
   const int nchunk = g.nchunk;
@@ -542,18 +543,23 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const bool row_exists = half == 0 || has1;
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
     const float qsc = (FP8 && row_exists) ? P.qs[bh * g.N + (half ? i1 : i0)] : 1.f;
-    if (nchunk == 1) {
+    if (nchunk == 1 || FP8) {
       // Extents of one-chunk tiles, spread over the softmax threads (the
       // compaction above leaves them out: a dense bitmap word would put up
-      // to 32 entries' divisions on one thread ahead of the CTA barrier).
-      for (int n = r; n < L; n += 128) uext[n] = chunk_ext((int)(ulist[n] & 0x1FFFFFu), ChunkOrigin{0, 0, 0});
+      // to 32 entries' divisions on one thread ahead of the CTA barrier),
+      // and on the e4m3 path each step's key-tile scale, all fetched here
+      // at once rather than one global load per step on the critical path.
+      for (int n = r; n < L; n += 128) {
+        const int jn = (int)(ulist[n] & 0x1FFFFFu);
+        if (nchunk == 1) uext[n] = chunk_ext(jn, ChunkOrigin{0, 0, 0});
+        if (FP8) uks[n] = __ldg(P.ks + bh * g.N + jn);
+      }
       asm volatile("bar.sync 2, 128;" ::: "memory");
     }
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int n = 0; n < L; ++n) {
       const uint32_t e = ulist[n];
-      const int j = (int)(e & 0x1FFFFFu);
       const bool keep = ((e >> (30 + half)) & 1u) != 0;  // uniform within the warp
       if (!__all_sync(0xffffffffu, tc::mbar_wait(bar_sfull(n & 1), (n >> 1) & 1, abort_flag, P.wait_limit))) {
         ok = false;
@@ -567,7 +573,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       if (keep) {
         uint32_t sr[64];
         tc::tmem_ld64_wait(sbuf, sr);
-        const float c = P.scale_log2 * (FP8 ? qsc * __ldg(P.ks + bh * g.N + j) : 1.f);
+        const float c = P.scale_log2 * (FP8 ? qsc * uks[n] : 1.f);
         const uint32_t ext = uext[n];
         const bool edge = (ext >> 31) != 0;
         if (edge) {  // padded keys of an edge chunk
@@ -765,7 +771,8 @@ bsattn_status run(const bsattn_plan* p, const void* q, const void* k, const __nv
           : !bsattn_make_map_2d(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, rows, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B))
     return BSATTN_ERR_CUDA;
   // Step list, extents and (tiles of several chunks) chunk offsets.
-  size_t smem = 1024 + C::OFF_DYN + (size_t)prm.bm_words * 8 + (size_t)prm.umax * (p->nchunk > 1 ? 12 : 8);
+  size_t smem = 1024 + C::OFF_DYN + (size_t)prm.bm_words * 8 + (size_t)prm.umax * (p->nchunk > 1 ? 12 : 8) +
+                (FP8 ? (size_t)prm.umax * 4 : 0);
   if (smem < 80 * 1024) smem = 80 * 1024;  // at most two CTAs (2 x 256 TMEM columns) per SM
   if (smem > 227 * 1024) return BSATTN_ERR_UNSUPPORTED;
   auto kern = attn_tc_kernel<D, FP8, NAT>;

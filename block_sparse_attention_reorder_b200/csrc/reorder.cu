@@ -76,37 +76,48 @@ __device__ __forceinline__ float block_max(float v, float* red) {
 // ulp(p) * ulp(scale) >= 2^-149; for codes that can be nonzero (|p| >= 2^-11)
 // that holds once scale >= 2^-92. Tiles with a smaller scale, or with one
 // above 2^126 (reciprocal subnormal or zero, e.g. an infinite amax), divide
-// instead; the test is per tile, hence uniform across the CTA. r is written
-// as -(p * scale - x) so that x = -0 keeps its sign.
+// instead; the test is per tile, hence uniform across the CTA. The kernels
+// form t = p * scale - x (exact, t = -r) and q = p + t * (-y), so that x = -0
+// gives -0, on packed pairs of values.
 constexpr float kFmaQuotientMinScale = 0x1p-92f, kFmaQuotientMaxScale = 0x1p126f;
-
-__device__ __forceinline__ float e4m3_quotient(float x, float scale, float rscale) {
-  const float p = __fmul_rn(x, rscale);
-  const float r = -fmaf(p, scale, -x);
-  return fmaf(r, rscale, p);
-}
 
 __device__ __forceinline__ bool fma_quotient_ok(float scale) {
   return scale >= kFmaQuotientMinScale && scale <= kFmaQuotientMaxScale;
 }
 
 // e4m3 codes of 8 values divided by `scale` (as the IEEE fp32 division), RNE,
-// satfinite; FMA: through e4m3_quotient (the tile passed fma_quotient_ok).
+// satfinite; FMA: by the correction above (the tile passed fma_quotient_ok),
+// else by division.
 template <bool FMA>
 __device__ __forceinline__ uint2 quant8(const float* f, float scale, float rscale) {
   uint32_t w[2];
+  if constexpr (FMA) {
+    const float2 y2 = make_float2(rscale, rscale), s2 = make_float2(scale, scale),
+                 ny2 = make_float2(-rscale, -rscale);
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    uint32_t acc = 0;
+    for (int h = 0; h < 2; ++h) {
+      uint32_t acc = 0;
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const float a = f[4 * h + 2 * i], b = f[4 * h + 2 * i + 1];
-      float2 x = FMA ? make_float2(e4m3_quotient(a, scale, rscale), e4m3_quotient(b, scale, rscale))
-                          : make_float2(__fdiv_rn(a, scale), __fdiv_rn(b, scale));
-      __nv_fp8x2_storage_t p = __nv_cvt_float2_to_fp8x2(x, __NV_SATFINITE, __NV_E4M3);
-      acc |= (uint32_t)p << (16 * i);
+      for (int i = 0; i < 2; ++i) {
+        const float2 x = make_float2(f[4 * h + 2 * i], f[4 * h + 2 * i + 1]);
+        const float2 p = __fmul2_rn(x, y2);
+        const float2 t = __ffma2_rn(p, s2, make_float2(-x.x, -x.y));
+        const float2 q = __ffma2_rn(t, ny2, p);
+        acc |= (uint32_t)__nv_cvt_float2_to_fp8x2(q, __NV_SATFINITE, __NV_E4M3) << (16 * i);
+      }
+      w[h] = acc;
     }
-    w[h] = acc;
+  } else {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      uint32_t acc = 0;
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const float2 q = make_float2(__fdiv_rn(f[4 * h + 2 * i], scale), __fdiv_rn(f[4 * h + 2 * i + 1], scale));
+        acc |= (uint32_t)__nv_cvt_float2_to_fp8x2(q, __NV_SATFINITE, __NV_E4M3) << (16 * i);
+      }
+      w[h] = acc;
+    }
   }
   return make_uint2(w[0], w[1]);
 }

@@ -5,9 +5,10 @@ page, Approach: per-tile e4m3 quantisation) by the IEEE fp32 quotient
 fl(x / s). The kernels compute it without a division, by Markstein's FMA
 correction: with y = fl(1 / s) correctly rounded,
 
-    p = fl(x * y),   r = fl(-(p * s - x)),   q = fl(p + r * y),
+    p = fl(x * y),   t = fl(p * s - x),   q = fl(p + t * (-y)),
 
-the two last steps single-rounded FMAs, and they take the plain division in
+the two last steps single-rounded FMAs (t is minus the residual x - p * s, and
+this form keeps the sign of x = -0), and they take the plain division in
 tiles whose scale is below 2^-92 or above 2^126. Here the three roundings are
 redone exactly in numpy (products of two fp32 values are exact in fp64; the
 last sum is rounded to fp32 from an exact two-term sum) and the codes from q
@@ -43,8 +44,8 @@ def _rn32_of_sum(a, b):
 
 def _fma_quotient(x, scale, y):
     p = (x * y).astype(np.float32).astype(np.float64)
-    r = (-(p * scale - x)).astype(np.float32).astype(np.float64)
-    return _rn32_of_sum(p, r * y)
+    t = (p * scale - x).astype(np.float32).astype(np.float64)
+    return _rn32_of_sum(p, t * -y)
 
 
 def _bf16_from_bits(bits):
