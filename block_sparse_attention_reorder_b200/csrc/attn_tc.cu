@@ -70,6 +70,7 @@ namespace {
 
 constexpr int kThreads = 192;
 constexpr int kStages = 2;
+static_assert(kStages == 2, "K/V slots are freed through the S / PV barriers of the same step parity");
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kColS0 = 0, kColS1 = 64, kColO = 128;
 constexpr long long kWaitLimit = 4000000000LL;  // SM cycles (~2 s)
@@ -112,8 +113,8 @@ struct Cfg {
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
   static constexpr int OFF_V = OFF_K + kStages * K_BYTES;
   static constexpr int OFF_BAR = OFF_V + kStages * V_BYTES;
-  // barriers: q, kfull[S], kempty[S], vfull[S], vempty[S], sfull[2], pfull[2], pvdone[2], final
-  static constexpr int NBAR = 1 + 4 * kStages + 7;
+  // barriers: q, kfull[S], vfull[S], sfull[2], pfull[2], pvdone[2], final
+  static constexpr int NBAR = 1 + 2 * kStages + 7;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base, abort, L, pad
   static constexpr int OFF_COL = OFF_MISC + 16;         // 64 packed column coords
   static constexpr int OFF_SCAN = OFF_COL + 256;        // block-scan scratch
@@ -150,14 +151,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const uint32_t sb = tc::smem_addr(smem);
   const uint32_t bar_q = sb + C::OFF_BAR;
+  // A K slot is free again when the S product that read it has completed,
+  // a V slot when its PV product has: with kStages = 2 S buffers and ring
+  // slots share the step parity, so the producer waits on sfull / pvdone
+  // (their next phase needs its own next load first, so it cannot miss one).
   auto bar_kfull = [&](int s) { return sb + C::OFF_BAR + 8u * (1 + s); };
-  auto bar_kempty = [&](int s) { return sb + C::OFF_BAR + 8u * (1 + kStages + s); };
-  auto bar_vfull = [&](int s) { return sb + C::OFF_BAR + 8u * (1 + 2 * kStages + s); };
-  auto bar_vempty = [&](int s) { return sb + C::OFF_BAR + 8u * (1 + 3 * kStages + s); };
-  auto bar_sfull = [&](int b) { return sb + C::OFF_BAR + 8u * (1 + 4 * kStages + b); };
-  auto bar_pfull = [&](int b) { return sb + C::OFF_BAR + 8u * (3 + 4 * kStages + b); };
-  auto bar_pvdone = [&](int b) { return sb + C::OFF_BAR + 8u * (5 + 4 * kStages + b); };
-  const uint32_t bar_final = sb + C::OFF_BAR + 8u * (7 + 4 * kStages);
+  auto bar_vfull = [&](int s) { return sb + C::OFF_BAR + 8u * (1 + kStages + s); };
+  auto bar_sfull = [&](int b) { return sb + C::OFF_BAR + 8u * (1 + 2 * kStages + b); };
+  auto bar_pfull = [&](int b) { return sb + C::OFF_BAR + 8u * (3 + 2 * kStages + b); };
+  auto bar_pvdone = [&](int b) { return sb + C::OFF_BAR + 8u * (5 + 2 * kStages + b); };
+  const uint32_t bar_final = sb + C::OFF_BAR + 8u * (7 + 2 * kStages);
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
   volatile int* never = reinterpret_cast<volatile int*>(misc + 3);  // stays 0: waits that ignore abort
@@ -268,9 +271,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     tc::mbar_init(bar_q, 1);
     for (int s = 0; s < kStages; ++s) {
       tc::mbar_init(bar_kfull(s), 1);
-      tc::mbar_init(bar_kempty(s), 1);
       tc::mbar_init(bar_vfull(s), 1);
-      tc::mbar_init(bar_vempty(s), 1);
     }
     for (int x = 0; x < 2; ++x) {
       tc::mbar_init(bar_sfull(x), 1);
@@ -429,7 +430,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         if (m < L) {
           const int s = m % kStages;
           if (m >= kStages &&
-              !tc::mbar_wait(bar_kempty(s), ((m / kStages) - 1) & 1, abort_flag, P.wait_limit)) {
+              !tc::mbar_wait(bar_sfull(s), ((m / kStages) - 1) & 1, abort_flag, P.wait_limit)) {
             record_timeout(abort_flag, P.err);
             break;
           }
@@ -449,7 +450,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         if (m >= 1) {
           const int v = m - 1, s = v % kStages;
           if (v >= kStages &&
-              !tc::mbar_wait(bar_vempty(s), ((v / kStages) - 1) & 1, abort_flag, P.wait_limit)) {
+              !tc::mbar_wait(bar_pvdone(s), ((v / kStages) - 1) & 1, abort_flag, P.wait_limit)) {
             record_timeout(abort_flag, P.err);
             break;
           }
@@ -503,7 +504,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             tc::mma_ss_f16(dS, da, db, idS, kk > 0 ? 1u : 0u);
         }
         tc::mma_commit(bar_sfull(m & 1));
-        tc::mma_commit(bar_kempty(s));
         return true;
       };
       if (ok) ok = issue_S(0);
@@ -524,7 +524,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           tc::mma_ts_f16(tmem + kColO, pA + kk * 8, dv, idPV, (n > 0 || kk > 0) ? 1u : 0u);
         }
         tc::mma_commit(bar_pvdone(n & 1));
-        tc::mma_commit(bar_vempty(s));
         if (n + 2 < L && !issue_S(n + 2)) {
           ok = false;
           break;
