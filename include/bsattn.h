@@ -233,7 +233,8 @@ bsattn_status attn_select_static(const bsattn_plan* plan, const void* q_nat, con
 /* Per-tile e4m3 quantisation of a tiled bf16 tensor (FPSAttention page,
  * Approach: FP8 quantisation and block sparsity share one 3D tile
  * granularity): per (b, head, tile) scale = fp32(amax)/448 (amax 0 -> 1),
- * code = e4m3(x/scale) rounded to nearest even with finite saturation (OCP
+ * code = e4m3 of the IEEE fp32 quotient x/scale (computed without a division,
+ * same bits), rounded to nearest even with finite saturation (OCP
  * E4M3; the page names FP8 without the format, this is the library's
  * reading). */
 bsattn_status attn_quantize_e4m3(const bsattn_plan* plan, const void* x_tiled,
